@@ -1,0 +1,194 @@
+"""Oracle for the Titans neural long-term memory -- TEST INFRASTRUCTURE ONLY.
+
+Only tests/, the smoke check (``__graft_entry__.smoke``) and bench.py's CPU
+baseline leg may import this package. The product (the CUDA library and its
+Python binding) never imports it and shares no code with it.
+
+Two fp64 paths, both from the pages on "Titans: Learning to Memorize at Test Time":
+
+* :func:`forward` -- the defining recurrence, token by token, in plain C
+  (``titans_oracle.c``): per-token gradients at the chunk-start weights
+  (walk-through sec. 3.2, t' = t - mod(t, b)), momentum S_t = eta_t S_{t-1} -
+  theta_t grad (sec. 3.1), forgetting W_t = (1 - alpha_t) W_{t-1} + S_t
+  (sec. 3.1 "Forgetting Mechanism"), retrieval y_t = M*(q_t) (sec. 3.1
+  "Retrieving a Memory").
+* :func:`forward_closed_form` -- the same chunk semantics unrolled over one
+  chunk (the tensorized mini-batch form of sec. 3.2, extended with momentum):
+  every per-token gradient is taken at the chunk-start weights, so the n
+  updates of a chunk fold into per-token coefficients c_j, d_j and three
+  per-chunk scalars. It is pinned to :func:`forward` by the tests (1e-12) and
+  is used where the token loop would take too long.
+
+Pins against things other than the oracle itself are in tests/test_oracle_pins.py.
+Parity of the oracle on the full-size workloads is "unpinned" beyond those pins:
+no page prints a worked numerical example.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Dict, Optional
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+
+def _open(path: str):
+    lib = ctypes.CDLL(path)
+    f = lib.titans_oracle_forward
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_long, ctypes.c_long, ctypes.c_int, ctypes.c_int, ctypes.c_int] + \
+        [ctypes.c_void_p] * 11 + [ctypes.c_int]
+    lib.titans_oracle_threads.restype = ctypes.c_int
+    return lib
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        _lib = _open(_build.build())
+    return _lib
+
+
+def forward_from_library(path: str):
+    """A forward() bound to another build of titans_oracle.c (used by the mutation tests)."""
+    lib = _open(path)
+
+    def fwd(*args, **kw):
+        return forward(*args, _lib_override=lib, **kw)
+    return fwd
+
+
+def threads() -> int:
+    return _load().titans_oracle_threads()
+
+
+def _np(x, dtype) -> np.ndarray:
+    try:
+        import torch
+        if isinstance(x, torch.Tensor):
+            x = x.detach().to("cpu")
+            x = x.to(torch.float64 if dtype == np.float64 else torch.float32).numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    return np.ascontiguousarray(np.asarray(x, dtype=dtype))
+
+
+def _ptr(a: Optional[np.ndarray]):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def forward(k, q, v, alpha, eta, theta, state: Dict, chunk: int, want_y: bool = True,
+            n_threads: int = 0, _lib_override=None):
+    """Token-by-token fp64 recurrence.
+
+    k, q, v: [U, T, d]; alpha, eta, theta: [U, T]; state: dict with W1, S1 (and W2, S2 for
+    the MLP), each [U, ...]. Returns (y [U, T, d] float64 or None, new state dict float64).
+    """
+    kf, qf, vf = (_np(x, np.float32) for x in (k, q, v))
+    al, et, th = (_np(x, np.float32) for x in (alpha, eta, theta))
+    U, T, d = kf.shape
+    linear = "W2" not in state
+    W1 = _np(state["W1"], np.float64).copy()
+    S1 = _np(state["S1"], np.float64).copy()
+    W2 = None if linear else _np(state["W2"], np.float64).copy()
+    S2 = None if linear else _np(state["S2"], np.float64).copy()
+    h = 0 if linear else W1.shape[1]
+    y = np.zeros((U, T, d), np.float64) if want_y else None
+    lib = _load() if _lib_override is None else _lib_override
+    rc = lib.titans_oracle_forward(U, T, d, h, int(chunk), _ptr(kf), _ptr(qf), _ptr(vf),
+                                       _ptr(al), _ptr(et), _ptr(th), _ptr(W1), _ptr(W2), _ptr(S1),
+                                       _ptr(S2), _ptr(y), int(n_threads))
+    if rc != 0:
+        raise RuntimeError("oracle: bad arguments or out of memory")
+    st = {"W1": W1, "S1": S1}
+    if not linear:
+        st.update(W2=W2, S2=S2)
+    return y, st
+
+
+def chunk_scalars(alpha: np.ndarray, eta: np.ndarray, theta: np.ndarray):
+    """Coefficients of one chunk (last axis = the chunk's tokens, 0-based j = 0..n-1).
+
+    Unrolling S_j = eta_j S_{j-1} - theta_j g_j and W_j = (1 - alpha_j) W_{j-1} + S_j over
+    the chunk with every g_j fixed at the chunk-start weights gives
+        W_end = A * W_0 + sigma * S_0 - sum_j c_j g_j
+        S_end = E * S_0 - sum_j d_j g_j
+    with P_j = prod_{l>j} (1 - alpha_l), Q_j = prod_{l>j} eta_l,
+         r_{n-1} = 1, r_j = P_j + eta_{j+1} r_{j+1},
+         c_j = theta_j r_j, d_j = theta_j Q_j,
+         A = (1 - alpha_0) P_0, E = eta_0 Q_0, sigma = eta_0 r_0.
+    Division-free; valid for eta = 0 and alpha = 1.
+    """
+    alpha = np.asarray(alpha, np.float64)
+    eta = np.asarray(eta, np.float64)
+    theta = np.asarray(theta, np.float64)
+    n = alpha.shape[-1]
+    P = np.ones_like(alpha)
+    Q = np.ones_like(alpha)
+    r = np.ones_like(alpha)
+    for j in range(n - 2, -1, -1):
+        P[..., j] = P[..., j + 1] * (1.0 - alpha[..., j + 1])
+        Q[..., j] = Q[..., j + 1] * eta[..., j + 1]
+        r[..., j] = P[..., j] + eta[..., j + 1] * r[..., j + 1]
+    c = theta * r
+    dd = theta * Q
+    A = (1.0 - alpha[..., 0]) * P[..., 0]
+    E = eta[..., 0] * Q[..., 0]
+    sig = eta[..., 0] * r[..., 0]
+    return c, dd, A, E, sig
+
+
+def _silu_parts(Z):
+    s = 1.0 / (1.0 + np.exp(-Z))
+    return s, Z * s
+
+
+def forward_closed_form(k, q, v, alpha, eta, theta, state: Dict, chunk: int, want_y: bool = True):
+    """Chunk closed form in fp64, batched over units with numpy matmuls. Same arguments as forward."""
+    K, Qm, V = (_np(x, np.float64) for x in (k, q, v))
+    al, et, th = (_np(x, np.float64) for x in (alpha, eta, theta))
+    U, T, d = K.shape
+    linear = "W2" not in state
+    W1 = _np(state["W1"], np.float64).copy()
+    S1 = _np(state["S1"], np.float64).copy()
+    if not linear:
+        W2 = _np(state["W2"], np.float64).copy()
+        S2 = _np(state["S2"], np.float64).copy()
+    y = np.zeros((U, T, d), np.float64) if want_y else None
+    tr = lambda x: np.swapaxes(x, -1, -2)
+    for t0 in range(0, T, chunk):
+        t1 = min(t0 + chunk, T)
+        Kc, Qc, Vc = K[:, t0:t1], Qm[:, t0:t1], V[:, t0:t1]
+        c, dd, A, E, sig = chunk_scalars(al[:, t0:t1], et[:, t0:t1], th[:, t0:t1])
+        A, E, sig = A[:, None, None], E[:, None, None], sig[:, None, None]
+        if linear:
+            Yh = Kc @ tr(W1)
+            G = 2.0 * (Yh - Vc)
+            if want_y:
+                y[:, t0:t1] = Qc @ tr(W1)
+            gc = tr(G * c[..., None]) @ Kc
+            gd = tr(G * dd[..., None]) @ Kc
+            W1, S1 = A * W1 + sig * S1 - gc, E * S1 - gd
+            continue
+        Z = Kc @ tr(W1)
+        s, Ak = _silu_parts(Z)
+        Yh = Ak @ tr(W2)
+        G = 2.0 * (Yh - Vc)
+        Dl = (G @ W2) * (s * (1.0 + Z * (1.0 - s)))
+        if want_y:
+            _, Aq = _silu_parts(Qc @ tr(W1))
+            y[:, t0:t1] = Aq @ tr(W2)
+        g2c = tr(G * c[..., None]) @ Ak
+        g2d = tr(G * dd[..., None]) @ Ak
+        g1c = tr(Dl * c[..., None]) @ Kc
+        g1d = tr(Dl * dd[..., None]) @ Kc
+        W2, S2 = A * W2 + sig * S2 - g2c, E * S2 - g2d
+        W1, S1 = A * W1 + sig * S1 - g1c, E * S1 - g1d
+    st = {"W1": W1, "S1": S1}
+    if not linear:
+        st.update(W2=W2, S2=S2)
+    return y, st
