@@ -1,0 +1,133 @@
+/*
+ * titans_mem.h -- C ABI of the Titans neural long-term memory library (sm_100a).
+ *
+ * The library computes the chunk-wise forward pass of the neural long-term
+ * memory described in "Titans: Learning to Memorize at Test Time" (pages: the
+ * mer.dev walk-through, sec. 3.1-3.2; the lowest.today German summary,
+ * "Gedaechtnisaktualisierungsmechanismus"; the hotdry blog, sec. 3.1):
+ *
+ *   memory      linear  M(x) = W x                 (walk-through sec. 3.1 "Memory Architecture")
+ *               MLP     M(x) = W2 silu(W1 x)       (blog sec. 3.1; SiLU per sec. 4.4)
+ *   loss        l_t = || M(k_t) - v_t ||_2^2       (sec. 3.1 "Objective")
+ *   momentum    S_t = eta_t S_{t-1} - theta_t grad l_t      (sec. 3.1 "Surprise Metric")
+ *   forgetting  M_t = (1 - alpha_t) M_{t-1} + S_t           (sec. 3.1 "Forgetting Mechanism")
+ *   chunking    every token of a chunk of b tokens takes its gradient at the
+ *               weights the chunk started with (sec. 3.2, t' = t - mod(t, b))
+ *   retrieval   y_t = M*(q_t), a forward pass with no update, using the same
+ *               chunk-start weights (sec. 3.1 "Retrieving a Memory")
+ *
+ * One "unit" is one (batch, head) pair; units are independent.
+ *
+ * Conventions for every call:
+ *  - Tensors are DEVICE pointers, row-major, contiguous, owned by the caller;
+ *    the library never frees or retains them. k, q, v, y and the state are
+ *    16-byte aligned; the gates alpha, eta, theta 4-byte aligned.
+ *  - Calls are asynchronous on the caller's CUDA stream (passed as void*, a
+ *    cudaStream_t; NULL = the legacy default stream).
+ *  - Argument checks happen before any launch and return TITANS_EINVAL or
+ *    TITANS_EUNSUPPORTED with a message in titans_last_error_string(); a
+ *    launch failure returns TITANS_ECUDA. Faults a kernel detects itself
+ *    (a wait that ran out of time) are recorded in a device status word that
+ *    titans_mem_sync_status() reads and clears (TITANS_EDEVICE).
+ *  - The calls allocate no device memory; titans_mem_init allocates the
+ *    handle's workspace and status word once.
+ *  - k and q are expected l2-normalised by the caller (sec. 4.4); the library
+ *    does not normalise.
+ */
+#ifndef TITANS_MEM_H
+#define TITANS_MEM_H
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    TITANS_OK = 0,
+    TITANS_EINVAL = 1,        /* bad argument: null/misaligned pointer, bad size */
+    TITANS_EUNSUPPORTED = 2,  /* valid but not supported (dimension, chunk length) */
+    TITANS_ECUDA = 3,         /* a CUDA runtime call or launch failed */
+    TITANS_EDEVICE = 4        /* the device status word reported a fault (timeout) */
+} titans_status_t;
+
+typedef enum {
+    TITANS_BF16 = 0,  /* k, q, v, y bf16; tensor-core arithmetic with fp32 accumulate; fp32 state */
+    TITANS_FP32 = 1   /* k, q, v, y fp32; CUDA-core fp32 arithmetic; fp32 state (reference mode) */
+} titans_mode_t;
+
+/* flags */
+#define TITANS_FLAG_CUDA_CORES 1u  /* run the CUDA-core chunk kernel even where the tensor-core one applies */
+
+typedef struct {
+    int d;             /* key/value width: 64 or 128 */
+    int d_hidden;      /* MLP hidden width h (4*d); 0 = linear memory */
+    int chunk;         /* largest chunk length the handle will be asked for, 1..128 */
+    titans_mode_t mode;
+    int B, H;          /* batch and heads: B*H units */
+    unsigned flags;    /* TITANS_FLAG_* */
+} titans_mem_config;
+
+typedef struct titans_mem *titans_mem_t;
+
+/* Kernel a call would run (titans_mem_path). */
+typedef enum {
+    TITANS_PATH_TC_MLP64 = 1,     /* tcgen05 bf16 chunk kernel, d=64, h=256, chunk<=64 */
+    TITANS_PATH_CUDA_CORES = 2,   /* CUDA-core fp32 chunk kernel (any supported shape) */
+    TITANS_PATH_STEP_CLUSTER = 3  /* single-token decode, thread-block-cluster kernel (MLP) */
+} titans_path_t;
+
+/* Validates the configuration and allocates the handle, its device status word and
+ * (for the CUDA-core path) its workspace on the current device.
+ * Returns TITANS_EINVAL for a null pointer or a non-positive size,
+ * TITANS_EUNSUPPORTED for d not in {64, 128}, d_hidden not in {0, 4d} or chunk
+ * outside 1..128, TITANS_ECUDA if an allocation fails. */
+titans_status_t titans_mem_init(const titans_mem_config *cfg, titans_mem_t *out);
+
+/* Frees the handle and its device memory. Must not race with work in flight. */
+titans_status_t titans_mem_destroy(titans_mem_t m);
+
+/*
+ * Chunk-wise forward over T tokens of every unit (update + retrieve).
+ *   k, q, v     [B, H, T, d]  bf16 (TITANS_BF16) or fp32 (TITANS_FP32)
+ *   alpha, eta, theta [B, H, T] fp32; alpha in [0, 1], eta, theta >= 0
+ *   MLP state:  W1, S1 [B, H, h, d], W2, S2 [B, H, d, h] fp32;
+ *   linear:     W1 = W, S1 = S [B, H, d, d] fp32, W2 = S2 = NULL
+ *               (column convention M(k) = W k, W is [d_out, d_in]).
+ *   The state is read at entry and overwritten with the state after token T-1.
+ *   y           [B, H, T, d] same dtype as k: y_t = M(q_t) with the weights at the
+ *               start of t's chunk.
+ *   chunk       1..cfg->chunk; a last chunk shorter than `chunk` follows the same rules.
+ * T >= 1 and T * d < 2^31 per unit.
+ */
+titans_status_t titans_mem_forward(titans_mem_t m, const void *k, const void *q, const void *v,
+                                   const float *alpha, const float *eta, const float *theta,
+                                   long T, int chunk, float *W1, float *W2, float *S1, float *S2,
+                                   void *y, void *stream);
+
+/*
+ * One decode step per unit with chunk = 1 semantics: y = M(q; W_{t-1}), then the
+ * update with the gradient at W_{t-1}.
+ *   k, q, v [B, H, d] (dtype of the mode); alpha, eta, theta [B, H] fp32;
+ *   state as in titans_mem_forward, updated in place; y [B, H, d].
+ */
+titans_status_t titans_mem_step(titans_mem_t m, const void *k, const void *q, const void *v,
+                                const float *alpha, const float *eta, const float *theta,
+                                float *W1, float *W2, float *S1, float *S2, void *y, void *stream);
+
+/* Kernel that titans_mem_forward (step = 0) or titans_mem_step (step = 1) would run with
+ * this chunk length; negative on an unsupported combination. */
+int titans_mem_path(titans_mem_t m, int chunk, int step);
+
+/* Synchronises the stream, then reads and clears the handle's device status word.
+ * TITANS_OK if no kernel reported a fault since the last call, else TITANS_EDEVICE. */
+titans_status_t titans_mem_sync_status(titans_mem_t m, void *stream);
+
+/* Thread-local message for the last non-OK status returned on this thread. */
+const char *titans_last_error_string(void);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+int titans_mem_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* TITANS_MEM_H */

@@ -1,0 +1,57 @@
+"""CPU-only checks of the C ABI: the library loads, exports every symbol the header
+declares, and rejects bad configurations before touching CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from titans_long_term_b200 import mem
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "titans_mem.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(titans_[a-z_]+)\s*\(", src)))
+
+
+def test_header_declares_the_binding_surface():
+    assert declared_functions() == sorted(mem.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol():
+    L = mem.lib()
+    for name in declared_functions():
+        assert hasattr(L, name), name
+    assert L.titans_mem_version() == 100
+
+
+@pytest.mark.parametrize("d,h,chunk,mode,B,H,status", [
+    (96, 0, 16, mem.FP32, 1, 1, mem.EUNSUPPORTED),
+    (64, 128, 16, mem.FP32, 1, 1, mem.EUNSUPPORTED),
+    (64, 256, 0, mem.BF16, 1, 1, mem.EUNSUPPORTED),
+    (64, 256, 129, mem.BF16, 1, 1, mem.EUNSUPPORTED),
+    (64, 256, 64, mem.BF16, 0, 1, mem.EINVAL),
+    (64, 256, 64, mem.BF16, 1, -2, mem.EINVAL),
+    (64, 256, 64, 7, 1, 1, mem.EINVAL),
+])
+def test_init_rejects_bad_configs(d, h, chunk, mode, B, H, status):
+    cfg = mem.Config(d, h, chunk, mode, B, H, 0)
+    out = ctypes.c_void_p()
+    assert mem.lib().titans_mem_init(ctypes.byref(cfg), ctypes.byref(out)) == status
+    assert out.value is None
+    assert mem.lib().titans_last_error_string().decode()
+
+
+def test_null_arguments():
+    L = mem.lib()
+    assert L.titans_mem_init(None, None) == mem.EINVAL
+    assert L.titans_mem_destroy(None) == mem.EINVAL
+    assert L.titans_mem_sync_status(None, None) == mem.EINVAL
+    assert L.titans_mem_path(None, 64, 0) == -1
+    rc = L.titans_mem_forward(None, None, None, None, None, None, None, 16, 16, None, None, None, None, None, None)
+    assert rc == mem.EINVAL
+    rc = L.titans_mem_step(None, None, None, None, None, None, None, None, None, None, None, None, None)
+    assert rc == mem.EINVAL

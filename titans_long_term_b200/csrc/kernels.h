@@ -1,0 +1,32 @@
+// Host-side launch interface shared by the library's .cu files (not part of the C ABI).
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstddef>
+
+namespace titans {
+
+struct ForwardArgs {
+    int d, h;          // h = 0: linear memory
+    long units, T;
+    int chunk;
+    bool bf16;         // k, q, v, y dtype
+    const void *k, *q, *v;
+    const float *alpha, *eta, *theta;
+    float *W1, *W2, *S1, *S2;
+    void* y;
+    float* ws;         // CUDA-core path workspace
+    size_t ws_per_unit;
+    unsigned* status;  // device status word
+};
+
+size_t cuda_cores_ws_floats(int d, int h, int n);
+cudaError_t launch_chunk_cuda_cores(const ForwardArgs& a, cudaStream_t st);
+cudaError_t launch_step_cluster(const ForwardArgs& a, cudaStream_t st);
+// Tensor-core chunk kernel (d = 64, h = 256, chunk <= 64, bf16). The tensor maps
+// describe k, q, v as [units][T][64] bf16 with a {64, chunk, 1} box and 128-byte swizzle.
+cudaError_t launch_chunk_tc_mlp64(const ForwardArgs& a, const CUtensorMap& tk, const CUtensorMap& tq,
+                                  const CUtensorMap& tv, cudaStream_t st);
+size_t chunk_tc_mlp64_smem_bytes();
+
+}  // namespace titans

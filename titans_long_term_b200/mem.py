@@ -1,0 +1,151 @@
+"""Python binding of the C ABI in include/titans_mem.h (argument marshalling only).
+
+Every computation runs in the CUDA library ``libtitans_mem.so`` built in-tree by
+``titans_long_term_b200/build.py``; if the library is missing this module raises
+instead of falling back to anything else. PyTorch supplies device memory and the
+current CUDA stream.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Dict, Optional
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libtitans_mem.so")
+
+OK, EINVAL, EUNSUPPORTED, ECUDA, EDEVICE = 0, 1, 2, 3, 4
+BF16, FP32 = 0, 1
+FLAG_CUDA_CORES = 1
+PATH_TC_MLP64, PATH_CUDA_CORES, PATH_STEP_CLUSTER = 1, 2, 3
+
+EXPORTED = ["titans_mem_init", "titans_mem_destroy", "titans_mem_forward", "titans_mem_step",
+            "titans_mem_path", "titans_mem_sync_status", "titans_last_error_string", "titans_mem_version"]
+
+
+class TitansError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"titans status {status}: {msg}")
+        self.status = status
+
+
+class Config(ctypes.Structure):
+    _fields_ = [("d", ctypes.c_int), ("d_hidden", ctypes.c_int), ("chunk", ctypes.c_int),
+                ("mode", ctypes.c_int), ("B", ctypes.c_int), ("H", ctypes.c_int), ("flags", ctypes.c_uint)]
+
+
+_lib = None
+
+
+def lib():
+    """Load the library (raises if it was not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: run `python -m titans_long_term_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i, l = ctypes.c_void_p, ctypes.c_int, ctypes.c_long
+        L.titans_mem_init.argtypes = [ctypes.POINTER(Config), ctypes.POINTER(vp)]
+        L.titans_mem_destroy.argtypes = [vp]
+        L.titans_mem_forward.argtypes = [vp, vp, vp, vp, vp, vp, vp, l, i, vp, vp, vp, vp, vp, vp]
+        L.titans_mem_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+        L.titans_mem_path.argtypes = [vp, i, i]
+        L.titans_mem_sync_status.argtypes = [vp, vp]
+        L.titans_last_error_string.restype = ctypes.c_char_p
+        for f in ("titans_mem_init", "titans_mem_destroy", "titans_mem_forward", "titans_mem_step",
+                  "titans_mem_path", "titans_mem_sync_status", "titans_mem_version"):
+            getattr(L, f).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _check(status: int):
+    if status != OK:
+        raise TitansError(status, lib().titans_last_error_string().decode())
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+class Memory:
+    """A configured memory: B*H independent units of a linear (d_hidden = 0) or
+    2-layer SiLU MLP memory (d_hidden = 4d)."""
+
+    def __init__(self, d: int, d_hidden: int, chunk: int, mode: str, B: int, H: int, cuda_cores: bool = False):
+        self.d, self.h, self.chunk, self.B, self.H = d, d_hidden, chunk, B, H
+        self.mode = mode
+        self.dtype = torch.bfloat16 if mode == "bf16" else torch.float32
+        cfg = Config(d, d_hidden, chunk, BF16 if mode == "bf16" else FP32, B, H,
+                     FLAG_CUDA_CORES if cuda_cores else 0)
+        h = ctypes.c_void_p()
+        _check(lib().titans_mem_init(ctypes.byref(cfg), ctypes.byref(h)))
+        self._h = h
+
+    def close(self):
+        if getattr(self, "_h", None):
+            lib().titans_mem_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def path(self, chunk: Optional[int] = None, step: bool = False) -> int:
+        return lib().titans_mem_path(self._h, chunk or self.chunk, int(step))
+
+    def _check_tensors(self, toks, gates, state, y, lead):
+        for n, t in list(toks.items()) + [("y", y)]:
+            if t.dtype != self.dtype or not t.is_cuda or not t.is_contiguous() or tuple(t.shape) != lead + (self.d,):
+                raise ValueError(f"{n}: expected contiguous CUDA {self.dtype} of shape {lead + (self.d,)}")
+        for n, t in gates.items():
+            if t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous() or tuple(t.shape) != lead:
+                raise ValueError(f"{n}: expected contiguous CUDA float32 of shape {lead}")
+        for n, t in state.items():
+            if t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous():
+                raise ValueError(f"{n}: expected contiguous CUDA float32")
+
+    def forward(self, k, q, v, alpha, eta, theta, state: Dict[str, torch.Tensor], chunk: Optional[int] = None,
+                y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        """k, q, v [B, H, T, d]; gates [B, H, T]; state W1, S1 (+ W2, S2) updated in place; returns y."""
+        T = k.shape[-2]
+        if y is None:
+            y = torch.empty_like(k)
+        self._check_tensors({"k": k, "q": q, "v": v}, {"alpha": alpha, "eta": eta, "theta": theta}, state, y,
+                            (self.B, self.H, T))
+        _check(lib().titans_mem_forward(self._h, _ptr(k), _ptr(q), _ptr(v), _ptr(alpha), _ptr(eta), _ptr(theta),
+                                        T, chunk or self.chunk, _ptr(state["W1"]), _ptr(state.get("W2")),
+                                        _ptr(state["S1"]), _ptr(state.get("S2")), _ptr(y), _stream(stream)))
+        return y
+
+    def step(self, k, q, v, alpha, eta, theta, state: Dict[str, torch.Tensor], y: Optional[torch.Tensor] = None,
+             stream=None) -> torch.Tensor:
+        """One decode token per unit: k, q, v [B, H, d]; gates [B, H]; state updated in place; returns y."""
+        if y is None:
+            y = torch.empty_like(k)
+        self._check_tensors({"k": k, "q": q, "v": v}, {"alpha": alpha, "eta": eta, "theta": theta}, state, y,
+                            (self.B, self.H))
+        _check(lib().titans_mem_step(self._h, _ptr(k), _ptr(q), _ptr(v), _ptr(alpha), _ptr(eta), _ptr(theta),
+                                     _ptr(state["W1"]), _ptr(state.get("W2")), _ptr(state["S1"]),
+                                     _ptr(state.get("S2")), _ptr(y), _stream(stream)))
+        return y
+
+    def sync_status(self, stream=None):
+        _check(lib().titans_mem_sync_status(self._h, _stream(stream)))
+
+
+def new_state(B: int, H: int, d: int, d_hidden: int, device="cuda") -> Dict[str, torch.Tensor]:
+    if d_hidden == 0:
+        z = torch.zeros(B, H, d, d, device=device)
+        return {"W1": z, "S1": z.clone()}
+    return {"W1": torch.zeros(B, H, d_hidden, d, device=device), "W2": torch.zeros(B, H, d, d_hidden, device=device),
+            "S1": torch.zeros(B, H, d_hidden, d, device=device), "S2": torch.zeros(B, H, d, d_hidden, device=device)}
