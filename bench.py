@@ -1,0 +1,369 @@
+"""Benchmark of the Titans memory's chunk-wise update + retrieve on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+
+One step = one titans_mem_forward over the whole workload: every (batch, head) unit
+runs all its chunks (update + retrieve) in one persistent kernel launch. The default
+workload is the 760M-class layer shape: MLP memory 64 -> 256 -> 64, B=8, H=16,
+T=4096, chunk 64. Inputs are seeded synthetic data (titans_long_term_b200.synth),
+resident in HBM before the timed region. Units are independent, so under torchrun
+every rank runs its own B*H units (weak scaling, no data-path collective); the
+elapsed time is the max over ranks.
+
+Prints one JSON line (rank 0). ``--impl reference`` times the fp64 CPU oracle (the
+reference arm for this method) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, HERE)
+
+from titans_long_term_b200 import mem, synth  # noqa: E402
+
+METRIC = "memory tokens/sec (update+retrieve) per B200; % bf16 tensor-core peak"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(HERE, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return PEAKS_FALLBACK, "fallback"
+
+
+def flops_per_head_token(w) -> float:
+    """Algorithmic FLOPs: MLP 18 d h (key forward 4dh, backprop to the hidden units 2dh, four
+    weighted outer-product sums 8dh, query retrieval 4dh); linear 8 d^2."""
+    return 18.0 * w.d * w.h if w.h else 8.0 * w.d * w.d
+
+
+def stream_bytes_per_head_token(w) -> float:
+    """k, q, v in, y out (input dtype) + three fp32 gates."""
+    e = 2 if w.dtype == "bf16" else 4
+    return 4 * w.d * e + 12
+
+
+def state_bytes_per_unit(w) -> float:
+    """W and S read once and written once per call (fp32)."""
+    n = 2 * w.d * w.h if w.h else w.d * w.d
+    return 4 * 2 * n * 4
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples (every 100 ms) bracketing the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.t_start = self.t_stop = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100",
+                 "-i", str(self.gpu)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self._reader = threading.Thread(target=self._read, daemon=True)
+        self._reader.start()
+        time.sleep(0.3)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def mark_start(self):
+        self.t_start = time.time()
+
+    def mark_stop(self):
+        self.t_stop = time.time()
+
+    def stop(self):
+        if self.proc:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        for ts, line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            rows.append((ts, parts))
+        inside = [p for ts, p in rows if self.t_start and self.t_stop and self.t_start - 0.1 <= ts <= self.t_stop + 0.1]
+        use = inside or [p for _, p in rows]
+        if not use:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no nvidia-smi samples"], "samples": 0}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(p[1]) for p in use if num(p[1]) is not None]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for p in use:
+            for name, val in zip(names, p[5:9]):
+                if val.strip().lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": num(use[0][2]),
+                "reasons": sorted(reasons), "samples": len(use), "samples_in_timed_region": len(inside),
+                "power_w_max": max((num(p[3]) or 0.0) for p in use)}
+
+
+# ---------------------------------------------------------------- oracle (CPU baseline / reference arm)
+
+def oracle_sample(w, core_seconds: float = 15.0, units_cap: int = 0):
+    """Time the fp64 oracle (token loop, OpenMP over units, all host cores) on a bounded
+    sample of the workload: the first U units x the first T tokens, sized from a short
+    calibration run to about `core_seconds` of CPU work."""
+    import oracle
+    cores = oracle.threads()
+    cal = synth.make_inputs(w, units=range(min(w.units, cores)), T=min(w.T, 2 * w.chunk))
+    st = {n: cal[n] for n in cal if n[0] in "WS"}
+    t = time.perf_counter()
+    oracle.forward(*(cal[n] for n in ("k", "q", "v", "alpha", "eta", "theta")), st, w.chunk)
+    rate = cal["k"].shape[0] * cal["k"].shape[1] / max(time.perf_counter() - t, 1e-6)  # head-tokens/s
+    want = rate * core_seconds / cores  # head-tokens for the target wall time
+    units = min(w.units, units_cap or w.units, max(1, cores))
+    T = int(min(w.T, max(w.chunk, (want / units) // w.chunk * w.chunk)))
+    while units < min(w.units, units_cap or w.units) and units * T < want and T == w.T:
+        units = min(w.units, units * 2)
+    inp = synth.make_inputs(w, units=range(units), T=T)
+    st = {n: inp[n] for n in inp if n[0] in "WS"}
+    t = time.perf_counter()
+    oracle.forward(*(inp[n] for n in ("k", "q", "v", "alpha", "eta", "theta")), st, w.chunk)
+    dt = time.perf_counter() - t
+    return {"value": units * T / w.H / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{units} units x {T} tokens of {w.name} (fp64 token loop), {dt:.2f} s wall",
+            "seconds": dt}
+
+
+def reference_arm(args, w, rank, world):
+    """The reference arm: the oracle as it stands, on this host's cores, one bounded sample per
+    step (sized so that warm-up + steps take about two minutes), rank 0 only."""
+    if rank != 0:
+        return
+    import oracle
+    per_step = 120.0 * oracle.threads() / max(1, args.steps + args.warmup)
+    per_step = min(per_step, 30.0 * oracle.threads())
+    for _ in range(args.warmup):
+        oracle_sample(w, core_seconds=per_step / 4)
+    vals, base = [], None
+    for _ in range(args.steps):
+        base = oracle_sample(w, core_seconds=per_step)
+        vals.append(base["value"])
+    value = statistics.median(vals)
+    base["value"] = value
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * w.B * w.T / value, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+            "impl": "reference",
+            "config": {"workload": w.name, "memory": f"MLP {w.d}-{w.h}-{w.d} SiLU" if w.h else f"linear {w.d}",
+                       "B": w.B, "H": w.H, "T": w.T, "chunk": w.chunk, "units": w.units},
+            "cpu_baseline": base,
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- our arm
+
+def our_arm(args, w, rank, world, local_rank):
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    # This rank's units: a contiguous block of a (world * B) x H batch, so every rank runs distinct data.
+    units = list(range(rank * w.units, (rank + 1) * w.units))
+    inp = synth.make_inputs(w, units=units)
+    toks = {n: inp[n].reshape(w.B, w.H, w.T, w.d).to(dev) for n in ("k", "q", "v")}
+    gates = {n: inp[n].reshape(w.B, w.H, w.T).to(dev) for n in ("alpha", "eta", "theta")}
+    state0 = {n: inp[n].reshape(w.B, w.H, *inp[n].shape[1:]).to(dev) for n in inp if n[0] in "WS"}
+    state = {n: t.clone() for n, t in state0.items()}
+    y = torch.empty_like(toks["k"])
+    m = mem.Memory(w.d, w.h, w.chunk, w.dtype, w.B, w.H)
+    path = m.path()
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        m.forward(toks["k"], toks["q"], toks["v"], gates["alpha"], gates["eta"], gates["theta"], state, y=y)
+
+    for _ in range(args.warmup):
+        step()
+    m.sync_status()
+    if world > 1:
+        torch.distributed.barrier()
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    phys = vis.split(",")[local_rank] if vis else str(local_rank)
+    clocks = ClockSampler(int(phys) if phys.isdigit() else local_rank)
+    if rank == 0:
+        clocks.start()
+    # Device-timed region: K launches, one event pair per launch on the launching stream.
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    clocks.mark_start()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(args.steps):
+        evs[i][0].record(stream)
+        step()
+        evs[i][1].record(stream)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks.mark_stop()
+    if world > 1:
+        torch.distributed.barrier()
+    m.sync_status()
+    elapsed_ms = t0.elapsed_time(t1)
+    launch_ms = [a.elapsed_time(b) for a, b in evs]
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+
+    # End-to-end through the public API from pinned host memory: H2D of the step's inputs,
+    # the forward, D2H of the step's result y.
+    host = {n: inp[n].reshape(t_.shape).pin_memory() for n, t_ in list(toks.items()) + list(gates.items())}
+    y_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+    h2d = sum(t_.numel() * t_.element_size() for t_ in host.values())
+    d2h = y_host.numel() * y_host.element_size()
+    e_steps = max(3, min(args.steps, 20))
+
+    def e2e_step():
+        for n, t_ in toks.items():
+            t_.copy_(host[n], non_blocking=True)
+        for n, t_ in gates.items():
+            t_.copy_(host[n], non_blocking=True)
+        step()
+        y_host.copy_(y, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(e_steps):
+        e2e_step()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = a.elapsed_time(b) / e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    m.sync_status()
+    if rank == 0:
+        clocks.stop()
+    if rank != 0:
+        return
+
+    ms = elapsed_ms / args.steps
+    tokens = world * w.B * w.T
+    value = tokens / (ms / 1e3)
+    peaks, which = load_peaks()
+    avg_launch = statistics.mean(launch_ms)
+    flops = flops_per_head_token(w) * w.units * w.T
+    achieved = flops / (avg_launch / 1e3) / 1e12
+    peak = peaks["bf16_tflops"]
+    algo_bytes = stream_bytes_per_head_token(w) * w.units * w.T + state_bytes_per_unit(w) * w.units
+    traffic = None
+    prof = os.path.join(HERE, "profiles", "traffic.json")
+    if os.path.exists(prof):
+        tr = json.load(open(prof)).get(w.name)
+        if tr and tr.get("kernel_sha") == kernel_sha():
+            traffic = tr["bytes_per_launch"]
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "fp32",
+        "data": "synthetic (seeded; k, v, q projections of one x_t)",
+        "config": {"workload": w.name,
+                   "memory": f"MLP {w.d}-{w.h}-{w.d} SiLU" if w.h else f"linear {w.d}x{w.d}",
+                   "B": w.B, "H": w.H, "T": w.T, "chunk": w.chunk, "units_per_gpu": w.units,
+                   "kernel": {1: "tcgen05 chunk kernel", 2: "CUDA-core chunk kernel"}.get(path, str(path)),
+                   "l2": "inputs larger than L2 (k, q, v, y, state = %.0f MB per step)" % (algo_bytes / 1e6)},
+        "head_tokens_per_s": value * w.H,
+        "pct_bf16_peak": 100.0 * achieved / peak,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": traffic,
+                     "peak_source": f"bf16_tflops ({which})", "kernel": "chunk_fwd_tc_mlp64",
+                     "flops_per_launch": flops, "avg_launch_ms": avg_launch,
+                     "frac_of_sustained": achieved / peaks.get("bf16_tflops_sustained", peak),
+                     "algorithmic_bytes_per_launch": algo_bytes,
+                     "hbm_gbs_at_algorithmic_bytes": algo_bytes / (avg_launch / 1e3) / 1e9},
+        "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": args.steps,
+        "clocks": clocks.summary(),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = oracle_sample(w)
+    print(json.dumps(line), flush=True)
+
+
+def kernel_sha() -> str:
+    import hashlib
+    p = os.path.join(HERE, "titans_long_term_b200", "csrc", "chunk_tc_mlp64.cu")
+    return hashlib.sha1(open(p, "rb").read()).hexdigest()[:12]
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="mlp-d64-b8h16-t4k", choices=list(synth.WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    w = synth.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        reference_arm(args, w, rank, world)
+        return
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        our_arm(args, w, rank, world, local_rank)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

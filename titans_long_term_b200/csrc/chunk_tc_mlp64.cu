@@ -6,22 +6,28 @@
 // weights, so the chunk's momentum / forgetting recurrence folds into
 //   W <- A W + sigma S - sum_j c_j g_j,   S <- E S - sum_j d_j g_j
 // with per-token c_j, d_j and per-chunk A, E, sigma from a division-free suffix scan
-// of the gates. The sums of per-token outer products are two weighted GEMMs, so the
+// of the gates. The sums of per-token outer products are weighted GEMMs, so the
 // whole chunk is five dense contractions on tcgen05:
-//   Z^T   [h x 2n] = W1 [K;Q]^T          keys and queries through layer 1
-//   Y     [2n x d] = silu(Z) W2^T         keys' M(k) and queries' retrieval
-//   (GW2)^T [h x n] = W2^T G^T            backprop of G = 2 (M(k) - v) to the hidden units
-//   dW1   [h x d] = Delta^T diag(-c|-d) K,  Delta = (G W2) * silu'(Z)
-//   dW2^T [h x d] = A_K^T diag(-c|-d) G
-// Everything is laid out with the hidden unit on the TMEM lane, so each thread owns
-// one hidden row j of every state matrix:
+//   Z^T     [h x 2n] = W1 [K;Q]^T          keys and queries through layer 1
+//   Y       [2n x d] = silu(Z) W2^T         keys' M(k) and queries' retrieval
+//   (GW2)^T [h x n]  = W2^T G^T             backprop of G = 2 (M(k) - v) to the hidden units
+//   dW1     [h x d]  = Delta^T diag(-c|-d) K,  Delta = (G W2) * silu'(Z_K)
+//   dW2^T   [h x d]  = A_K^T diag(-c|-d) G
+// The hidden unit sits on the TMEM lane, so each thread of the epilogue warps owns one
+// hidden row j of every state matrix:
 //   - W1[j, :] and W2[:, j] (fp32) live in that thread's registers,
 //   - S1[j, :] and S2[:, j] (fp32) live in TMEM and are the accumulators of the
-//     d-weighted GEMMs (pre-scaled by E before the GEMM accumulates -sum d_j g_j),
-//   - the bf16 copies of W1 and W2^T that feed the MMAs are rewritten in shared
-//     memory once per chunk.
-// One CTA (8 warps, 1 per SM) per (batch, head) unit, persistent over the chunk loop;
-// K, Q, V tiles of chunk c+2 stream in by TMA while chunk c computes.
+//     d-weighted GEMMs (pre-scaled by E before the GEMMs accumulate -sum d_j g_j),
+//   - the bf16 copies of W1 and W2^T that feed the MMAs are rewritten in shared memory
+//     once per chunk.
+// Warp roles (12 warps, one CTA per SM, persistent over the chunk loop of one unit):
+//   - warps 0-3 own hidden rows 0..127 ("tile 0"), warps 4-7 rows 128..255 ("tile 1");
+//     the two tiles run their epilogues independently, so the tensor core works on one
+//     tile while the other tile's warps run theirs;
+//   - warp 8 issues TMA (K, Q, V tiles two chunks ahead) and every MMA (lane 0), and
+//     computes the next chunk's gate scan and scaled key tiles; warps 9-11 only complete
+//     its warpgroup, which hands its registers to the epilogue warpgroups (setmaxnreg).
+// Hand-offs go through mbarriers only; every wait is bounded.
 #include <cuda_bf16.h>
 #include <cstdint>
 
@@ -31,7 +37,13 @@
 namespace titans {
 
 namespace tc {
-constexpr int kThreads = 256;
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 384;  // 3 warpgroups: tile 0, tile 1, producer (warp 8 works, 9..11 idle)
+// Register split: launched at kRegsLaunch per thread, the producer warpgroup gives registers
+// back and the two epilogue warpgroups take them: 128 * kRegsProducer + 256 * kRegsEpilogue
+// must not exceed 384 * kRegsLaunch (the block's launch allocation).
+constexpr int kRegsLaunch = 168, kRegsProducer = 88, kRegsEpilogue = 208;
+static_assert(128 * kRegsProducer + 256 * kRegsEpilogue <= 384 * kRegsLaunch, "register split");
 constexpr int kD = 64, kH = 256, kN = 64;
 // Shared-memory map (byte offsets from a 1024-aligned base). Every tile is
 // [rows][64] bf16 with the 128-byte swizzle: 128 B per row, 1024-B atoms of 8 rows.
@@ -48,15 +60,27 @@ constexpr uint32_t GC = G + 8192;      // -c_t G[t, :]       B of dW2^T (MN-majo
 constexpr uint32_t GD = GC + 8192;     // -d_t G[t, :]
 constexpr uint32_t KC = GD + 8192;     // -c_t K[t, :]       B of dW1 (MN-major)
 constexpr uint32_t KD = KC + 8192;     // -d_t K[t, :]
-constexpr uint32_t ALPHA = KD + 8192;  // 64 floats each
-constexpr uint32_t ETA = ALPHA + 256;
-constexpr uint32_t THETA = ETA + 256;
-constexpr uint32_t CC = THETA + 256;
-constexpr uint32_t DD = CC + 256;
-constexpr uint32_t SCAL = DD + 256;    // A, E, sigma
-constexpr uint32_t BAR = SCAL + 16;    // tma[0], tma[1], mma: 3 x u64
-constexpr uint32_t TPTR = BAR + 24;    // TMEM base address
-constexpr uint32_t FLAG = TPTR + 4;    // abort flag
+constexpr uint32_t GATES = KD + 8192;  // staging for the scan: alpha, eta, theta [3][64] floats
+constexpr uint32_t CC = GATES + 768;   // c_j  [2 parities][64]
+constexpr uint32_t DD = CC + 512;      // d_j  [2][64]
+constexpr uint32_t SCAL = DD + 512;    // A, E, sigma [2][4]
+constexpr uint32_t BAR = SCAL + 32;    // mbarriers, 8 B each
+enum Bar {
+    B_TMA0, B_TMA1,      // K, Q, V tiles landed (buffer 0 / 1)
+    B_Z0, B_Z1,          // Z^T of tile t done
+    B_A0, B_A1,          // tile t wrote its silu rows (and silu' into TMEM)
+    B_Y,                 // Y done
+    B_G,                 // G tiles written, Y read (all epilogue threads)
+    B_S0, B_S1,          // tile t's momentum pre-pass done
+    B_GW0, B_GW1,        // (GW2)^T and the S2^T accumulation of tile t done
+    B_D0, B_D1,          // tile t wrote Delta^T rows
+    B_DW0, B_DW1,        // weighted weight GEMMs of tile t done
+    B_W0, B_W1,          // tile t rewrote its bf16 weight rows (and read dW_c)
+    B_SC0, B_SC1,        // gate scan of a chunk with parity 0 / 1 published
+    kNumBars
+};
+constexpr uint32_t TPTR = BAR + 8 * kNumBars;  // TMEM base address
+constexpr uint32_t FLAG = TPTR + 4;            // abort flag
 constexpr uint32_t END = FLAG + 4;
 constexpr size_t kSmemBytes = END + 1024;  // + alignment slack
 // TMEM columns: [0, 256) working region, [256, 512) momentum S.
@@ -76,7 +100,6 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
           "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
         : "r"(taddr));
 }
-
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
@@ -85,14 +108,18 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
         "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
         : "memory");
 }
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
 
-// Writes a 64-element fp32 row as bf16 into row `row` of a swizzled [rows][64] tile.
-__device__ __forceinline__ void store_row_bf16(uint32_t tile, int row, const float (&w)[64]) {
+// Writes 16 fp32 values as bf16 into columns [16 blk, 16 blk + 16) of row `row` of a
+// swizzled [rows][64] tile (two 16-byte chunks).
+__device__ __forceinline__ void store16_bf16(uint32_t tile, int row, int blk, const float* x) {
 #pragma unroll
-    for (int ch = 0; ch < 8; ++ch) {
-        const uint32_t a = tile + (uint32_t)row * 128u + ((uint32_t)(ch ^ (row & 7)) << 4);
-        st_shared_v4(a, pack_bf16x2(w[8 * ch + 0], w[8 * ch + 1]), pack_bf16x2(w[8 * ch + 2], w[8 * ch + 3]),
-                     pack_bf16x2(w[8 * ch + 4], w[8 * ch + 5]), pack_bf16x2(w[8 * ch + 6], w[8 * ch + 7]));
+    for (int ch = 0; ch < 2; ++ch) {
+        const uint32_t a = tile + (uint32_t)row * 128u + ((uint32_t)((2 * blk + ch) ^ (row & 7)) << 4);
+        st_shared_v4(a, pack_bf16x2(x[8 * ch + 0], x[8 * ch + 1]), pack_bf16x2(x[8 * ch + 2], x[8 * ch + 3]),
+                     pack_bf16x2(x[8 * ch + 4], x[8 * ch + 5]), pack_bf16x2(x[8 * ch + 6], x[8 * ch + 7]));
     }
 }
 
@@ -151,7 +178,13 @@ __device__ __forceinline__ void gate_scan(int n, const float* sa, const float* s
     }
 }
 
-__device__ __forceinline__ float sigmoidf_fast(float z) { return __fdividef(1.f, 1.f + __expf(-z)); }
+// tanh via the hardware approximation (one MUFU op, relative error about 2^-11, below the
+// bf16 rounding the activations get next).
+__device__ __forceinline__ float tanh_approx(float x) {
+    float y;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
 
 __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ,
@@ -162,31 +195,30 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sb = smem_u32(sm);
-    float* s_alpha = reinterpret_cast<float*>(sm + ALPHA);
-    float* s_eta = reinterpret_cast<float*>(sm + ETA);
-    float* s_theta = reinterpret_cast<float*>(sm + THETA);
-    float* s_c = reinterpret_cast<float*>(sm + CC);
-    float* s_d = reinterpret_cast<float*>(sm + DD);
-    float* s_scal = reinterpret_cast<float*>(sm + SCAL);
-    uint64_t* bar_tma = reinterpret_cast<uint64_t*>(sm + BAR);
-    uint64_t* bar_mma = bar_tma + 2;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + BAR);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + FLAG);
+    float* s_cc = reinterpret_cast<float*>(sm + CC);
+    float* s_dd = reinterpret_cast<float*>(sm + DD);
+    float* s_scal = reinterpret_cast<float*>(sm + SCAL);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int quad = warp & 3, half = warp >> 2;
-    const int hrow = half * 128 + quad * 32 + lane;  // hidden row owned by this thread
-    const uint32_t lane_off = uint32_t(quad * 32) << 16;
     const long u = blockIdx.x;
+    const int nchunks = (int)((T + chunk - 1) / chunk);
 
     if (tid == 0) {
-        mbar_init(&bar_tma[0], 1);
-        mbar_init(&bar_tma[1], 1);
-        mbar_init(bar_mma, 1);
+        for (int b = 0; b < kNumBars; ++b) {
+            uint32_t cnt = 1;
+            if (b == B_A0 || b == B_A1 || b == B_S0 || b == B_S1 || b == B_D0 || b == B_D1 || b == B_W0 ||
+                b == B_W1)
+                cnt = 128;
+            else if (b == B_G)
+                cnt = 256;
+            else if (b == B_SC0 || b == B_SC1)
+                cnt = 32;
+            mbar_init(&bars[b], cnt);
+        }
         fence_mbar_init();
         *abort_flag = 0;
-        prefetch_tmap(&tmK);
-        prefetch_tmap(&tmQ);
-        prefetch_tmap(&tmV);
     }
     if (warp == 0) {
         tmem_alloc(reinterpret_cast<uint32_t*>(sm + TPTR), kTmemCols);
@@ -194,231 +226,321 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
     }
     // Token tiles start at zero: rows beyond the chunk length are never written by TMA.
     for (uint32_t o = tid * 16; o < 49152; o += kThreads * 16) st_shared_v4(sb + KQ0 + o, 0u, 0u, 0u, 0u);
-
-    // State of this thread's hidden row.
-    float w1[64], w2[64];
-    {
-        const float4* p = reinterpret_cast<const float4*>(W1g + (u * kH + hrow) * kD);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const float4 x = p[i];
-            w1[4 * i] = x.x;
-            w1[4 * i + 1] = x.y;
-            w1[4 * i + 2] = x.z;
-            w1[4 * i + 3] = x.w;
-        }
-        const float* q2 = W2g + u * kD * kH + hrow;
-#pragma unroll
-        for (int i = 0; i < 64; ++i) w2[i] = q2[(size_t)i * kH];
-    }
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sm + TPTR);
-    const uint32_t t_work = tmem + lane_off + half * 128;        // this warp's working columns
-    const uint32_t t_s = tmem + lane_off + 256 + half * 128;     // S1 at +0, S2^T at +64
-    {
-        const float* p1 = S1g + (u * kH + hrow) * kD;
-        const float* p2 = S2g + u * kD * kH + hrow;
-#pragma unroll
-        for (int hh = 0; hh < 4; ++hh) {
-            uint32_t r[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(p1[16 * hh + i]);
-            tmem_st16(t_s + 16 * hh, r);
-#pragma unroll
-            for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(p2[(size_t)(16 * hh + i) * kH]);
-            tmem_st16(t_s + 64 + 16 * hh, r);
-        }
-    }
-    store_row_bf16(sb + W1, hrow, w1);
-    store_row_bf16(sb + W2T, hrow, w2);
-    tmem_wait_st();
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
 
-    const int nchunks = (int)((T + chunk - 1) / chunk);
-    const uint32_t tx_bytes = 3u * (uint32_t)chunk * 128u;
-    uint32_t tma_issued[2] = {0, 0}, tma_done[2] = {0, 0};  // used by thread 0 only
-    auto issue_tma = [&](int c, int b) {
-        const uint32_t kq = b ? KQ1 : KQ0, vv = b ? V1 : V0;
-        mbar_arrive_expect_tx(&bar_tma[b], tx_bytes);
-        tma_load_3d(sm + kq, &tmK, &bar_tma[b], 0, c * chunk, (int)u);
-        tma_load_3d(sm + kq + 8192, &tmQ, &bar_tma[b], 0, c * chunk, (int)u);
-        tma_load_3d(sm + vv, &tmV, &bar_tma[b], 0, c * chunk, (int)u);
-        ++tma_issued[b];
-    };
-    if (tid == 0) {
-        issue_tma(0, 0);
-        if (nchunks > 1) issue_tma(1, 1);
-    }
-    uint32_t mma_phase = 0;
-    bool mma_pending = false;  // thread 0: a commit not yet waited for
-    auto wait_mma = [&]() {
-        if (!mbar_wait(bar_mma, mma_phase)) {
-            atomicOr(status, kStatusTimeoutMma);
-            *abort_flag = 1;
-        } else if (tid == 0) {
-            mma_pending = false;
-        }
-        mma_phase ^= 1u;
-        tc_fence_after();
+    // Bounded wait; on a timeout records the fault, raises the abort flag and returns false.
+    auto wait = [&](int b, uint32_t parity) -> bool {
+        if (mbar_wait(&bars[b], parity)) return true;
+        atomicOr(status, b <= B_TMA1 ? kStatusTimeoutTma : kStatusTimeoutMma);
+        *abort_flag = 1;
+        return false;
     };
 
-    const uint32_t idZ = idesc_bf16_f32(128, 128, 0, 0);
-    const uint32_t idY = idesc_bf16_f32(128, 64, 1, 1);
-    const uint32_t idG = idesc_bf16_f32(128, 64, 0, 0);
-    const uint32_t idW = idesc_bf16_f32(128, 64, 0, 1);
-
-    for (int c = 0; c < nchunks; ++c) {
-        const int buf = c & 1;
-        const uint32_t KQb = buf ? KQ1 : KQ0, Vb = buf ? V1 : V0;
-        const long t0 = (long)c * chunk;
-        const int n = (int)min((long)chunk, T - t0);
-
-        // (A) gates; K, Q tiles landed -> Z^T = W1 [K;Q]^T
-        if (tid < kN) {
-            const long g = u * T + t0 + tid;
-            s_alpha[tid] = tid < n ? alpha[g] : 0.f;
-            s_eta[tid] = tid < n ? eta[g] : 1.f;
-            s_theta[tid] = tid < n ? theta[g] : 0.f;
-        }
-        // Every thread waits on the tile barrier itself: the K and V tiles are read below
-        // with ordinary shared-memory loads as well as by the MMAs.
-        const bool landed = mbar_wait(&bar_tma[buf], (uint32_t)(c >> 1) & 1u);
-        if (!landed) {
-            atomicOr(status, kStatusTimeoutTma);
-            *abort_flag = 1;
-        }
-        if (tid == 0) {
-            if (landed) {
-                ++tma_done[buf];
-                tc_fence_after();
+    if (warp >= kEpiWarps) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsProducer));
+    }
+    if (warp > kEpiWarps) {
+        // warps 9..11: nothing to do
+    } else if (warp == kEpiWarps) {
+        // =========================== issuer warp: TMA, MMAs, gate scans, scaled key tiles
+        const uint32_t idZ = idesc_bf16_f32(128, 128, 0, 0);
+        const uint32_t idY = idesc_bf16_f32(128, 64, 1, 1);
+        const uint32_t idG = idesc_bf16_f32(128, 64, 0, 0);
+        const uint32_t idW = idesc_bf16_f32(128, 64, 0, 1);
+        const uint32_t tx_bytes = 3u * (uint32_t)chunk * 128u;
+        uint32_t tma_issued = 0, tma_waited = 0;  // counts per buffer packed: bits [0,16) buf 0, [16,32) buf 1
+        auto issue_tma = [&](int c) {
+            const int b = c & 1;
+            const uint32_t kq = b ? KQ1 : KQ0, vv = b ? V1 : V0;
+            mbar_arrive_expect_tx(&bars[B_TMA0 + b], tx_bytes);
+            tma_load_3d(sm + kq, &tmK, &bars[B_TMA0 + b], 0, c * chunk, (int)u);
+            tma_load_3d(sm + kq + 8192, &tmQ, &bars[B_TMA0 + b], 0, c * chunk, (int)u);
+            tma_load_3d(sm + vv, &tmV, &bars[B_TMA0 + b], 0, c * chunk, (int)u);
+            tma_issued += b ? 0x10000u : 1u;
+        };
+        // Gates of chunk c travel in registers (lane l holds tokens l and l + 32) one chunk ahead.
+        float ga[2], ge[2], gt[2];
+        auto load_gates = [&](int c) {
+            const long t0 = (long)c * chunk;
+            const long n = c < nchunks ? min((long)chunk, T - t0) : 0;
 #pragma unroll
-                for (int t = 0; t < 2; ++t)
+            for (int i = 0; i < 2; ++i) {
+                const int j = lane + 32 * i;
+                const bool ok = j < n;
+                const long g = u * T + t0 + j;
+                ga[i] = ok ? __ldg(alpha + g) : 0.f;
+                ge[i] = ok ? __ldg(eta + g) : 1.f;
+                gt[i] = ok ? __ldg(theta + g) : 0.f;
+            }
+        };
+        float* sg = reinterpret_cast<float*>(sm + GATES);
+        auto scan = [&](int c) {  // gates of chunk c are in registers
+            const long t0 = (long)c * chunk;
+            const int n = (int)min((long)chunk, T - t0);
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                sg[lane + 32 * i] = ga[i];
+                sg[64 + lane + 32 * i] = ge[i];
+                sg[128 + lane + 32 * i] = gt[i];
+            }
+            __syncwarp();
+            const int p = c & 1;
+            gate_scan(n, sg, sg + 64, sg + 128, s_cc + 64 * p, s_dd + 64 * p, s_scal + 4 * p, lane);
+            __syncwarp();
+            mbar_arrive(&bars[B_SC0 + p]);
+        };
+        if (lane == 0) {
+            prefetch_tmap(&tmK);
+            prefetch_tmap(&tmQ);
+            prefetch_tmap(&tmV);
+            issue_tma(0);
+            if (nchunks > 1) issue_tma(1);
+        }
+        load_gates(0);
+        scan(0);
+        load_gates(1);
+
+        for (int c = 0; c < nchunks; ++c) {
+            const int b = c & 1, p = c & 1;
+            const uint32_t ph = (uint32_t)c & 1u;
+            const uint32_t KQb = b ? KQ1 : KQ0;
+            bool ok = wait(B_TMA0 + b, (uint32_t)(c >> 1) & 1u);
+            if (ok) tma_waited += b ? 0x10000u : 1u;
+            // Z^T of tile t once tile t has rewritten its weight rows (after chunk c-1).
+            for (int t = 0; t < 2 && ok; ++t) {
+                ok = wait(B_W0 + t, ph);
+                if (ok && lane == 0) {
+                    tc_fence_after();
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks)
                         umma_bf16(tmem + t * 128, sdesc_sw128(sb + W1 + t * 16384 + ks * 32, 16, 1024),
                                   sdesc_sw128(sb + KQb + ks * 32, 16, 1024), idZ, ks > 0);
-                umma_commit(bar_mma);
-                mma_pending = true;
+                    umma_commit(&bars[B_Z0 + t]);
+                }
+            }
+            if (!ok || *abort_flag) break;
+            // Scaled key tiles of this chunk (the previous chunk's weight GEMMs, which read them,
+            // completed before tile 1 signalled B_W1 above).
+            {
+                const float* cc = s_cc + 64 * p;
+                const float* dd = s_dd + 64 * p;
+#pragma unroll 4
+                for (int i = 0; i < 16; ++i) {
+                    const uint32_t off = (uint32_t)(lane + 32 * i) * 16u;
+                    const int row = (lane + 32 * i) >> 3;
+                    const uint4 kv = ld_shared_v4(sb + KQb + off);
+                    const float cr = -cc[row], dr = -dd[row];
+                    const uint32_t in[4] = {kv.x, kv.y, kv.z, kv.w};
+                    uint32_t oc[4], od[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 f = unpack_bf16x2(in[e]);
+                        oc[e] = pack_bf16x2(cr * f.x, cr * f.y);
+                        od[e] = pack_bf16x2(dr * f.x, dr * f.y);
+                    }
+                    st_shared_v4(sb + KC + off, oc[0], oc[1], oc[2], oc[3]);
+                    st_shared_v4(sb + KD + off, od[0], od[1], od[2], od[3]);
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+            }
+            // Next chunk's gate scan (its gates are already in registers), then prefetch the one after.
+            if (c + 1 < nchunks) {
+                scan(c + 1);
+                load_gates(c + 2);
+            }
+            // Y = A W2^T: the K dimension (hidden units) in two halves, one per tile.
+            for (int t = 0; t < 2 && ok; ++t) {
+                ok = wait(B_A0 + t, ph);
+                if (ok && lane == 0) {
+                    tc_fence_after();
+#pragma unroll
+                    for (int ks = 8 * t; ks < 8 * t + 8; ++ks)
+                        umma_bf16(tmem + 64, sdesc_sw128(sb + AT0 + ks * 2048, AT1 - AT0, 1024),
+                                  sdesc_sw128(sb + W2T + ks * 2048, 8192, 1024), idY, ks > 0);
+                    if (t == 1) umma_commit(&bars[B_Y]);
+                }
+            }
+            if (!ok) break;
+            // G tiles written: the K, Q, V buffer of this chunk is free -> chunk c + 2.
+            ok = wait(B_G, ph);
+            if (!ok) break;
+            if (lane == 0 && c + 2 < nchunks) issue_tma(c + 2);
+            // (GW2)^T = W2^T G^T and S2^T += A_K^T diag(-d) G, per tile once its S is pre-scaled.
+            for (int t = 0; t < 2 && ok; ++t) {
+                ok = wait(B_S0 + t, ph);
+                if (ok && lane == 0) {
+                    tc_fence_after();
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        umma_bf16(tmem + t * 128 + 64, sdesc_sw128(sb + W2T + t * 16384 + ks * 32, 16, 1024),
+                                  sdesc_sw128(sb + G + ks * 32, 16, 1024), idG, ks > 0);
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        umma_bf16(tmem + 256 + t * 128 + 64, sdesc_sw128(sb + AT0 + t * 16384 + ks * 32, 16, 1024),
+                                  sdesc_sw128(sb + GD + ks * 2048, 8192, 1024), idW, 1);
+                    umma_commit(&bars[B_GW0 + t]);
+                }
+            }
+            if (!ok) break;
+            // dW1_c -> cols 128t, S1 += Delta^T diag(-d) K, dW2^T_c -> cols 128t+64, per tile.
+            for (int t = 0; t < 2 && ok; ++t) {
+                ok = wait(B_D0 + t, ph);
+                if (ok && lane == 0) {
+                    tc_fence_after();
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks) {
+                        const uint64_t dA = sdesc_sw128(sb + AT1 + t * 16384 + ks * 32, 16, 1024);
+                        const uint64_t aA = sdesc_sw128(sb + AT0 + t * 16384 + ks * 32, 16, 1024);
+                        umma_bf16(tmem + t * 128, dA, sdesc_sw128(sb + KC + ks * 2048, 8192, 1024), idW, ks > 0);
+                        umma_bf16(tmem + 256 + t * 128, dA, sdesc_sw128(sb + KD + ks * 2048, 8192, 1024), idW, 1);
+                        umma_bf16(tmem + t * 128 + 64, aA, sdesc_sw128(sb + GC + ks * 2048, 8192, 1024), idW,
+                                  ks > 0);
+                    }
+                    umma_commit(&bars[B_DW0 + t]);
+                }
+            }
+            if (!ok) break;
+            __syncwarp();
+        }
+        __syncwarp();
+        // Drain: after an abort, copies may still be in flight into shared memory.
+        if (lane == 0) {
+            for (int b = 0; b < 2; ++b) {
+                uint32_t iss = (tma_issued >> (16 * b)) & 0xFFFFu, don = (tma_waited >> (16 * b)) & 0xFFFFu;
+                while (don < iss) {
+                    if (!mbar_wait(&bars[B_TMA0 + b], don & 1u)) break;
+                    ++don;
+                }
             }
         }
-        __syncthreads();
-        if (*abort_flag) break;
-
-        // (B) gate scan
-        if (warp == 0) gate_scan(n, s_alpha, s_eta, s_theta, s_c, s_d, s_scal, lane);
-        __syncthreads();
-
-        // (C) momentum pre-pass: W <- A W + sigma S, S <- E S (the d-GEMM then adds -sum d_j g_j);
-        //     scaled key tiles -c_t K[t], -d_t K[t]
+    } else {
+        // =========================== epilogue warps: one hidden row per thread
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsEpilogue));
+        const int quad = warp & 3, tile = warp >> 2;
+        const int hrow = tile * 128 + quad * 32 + lane;
+        const uint32_t lane_off = uint32_t(quad * 32) << 16;
+        const uint32_t t_work = tmem + lane_off + tile * 128;     // this tile's working columns
+        const uint32_t t_s = tmem + lane_off + 256 + tile * 128;  // S1 at +0, S2^T at +64
+        float w1[64], w2[64];
         {
-            const float An = s_scal[0], En = s_scal[1], sig = s_scal[2];
+            const float4* p = reinterpret_cast<const float4*>(W1g + (u * kH + hrow) * kD);
 #pragma unroll
-            for (int hh = 0; hh < 4; ++hh) {
+            for (int i = 0; i < 16; ++i) {
+                const float4 x = p[i];
+                w1[4 * i] = x.x;
+                w1[4 * i + 1] = x.y;
+                w1[4 * i + 2] = x.z;
+                w1[4 * i + 3] = x.w;
+            }
+            const float* q2 = W2g + u * kD * kH + hrow;
+#pragma unroll
+            for (int i = 0; i < 64; ++i) w2[i] = q2[(size_t)i * kH];
+            const float* p1 = S1g + (u * kH + hrow) * kD;
+            const float* p2 = S2g + u * kD * kH + hrow;
+#pragma unroll
+            for (int blk = 0; blk < 4; ++blk) {
                 uint32_t r[16];
-                tmem_ld16(t_s + 16 * hh, r);
-                tmem_wait_ld();
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const float s = __uint_as_float(r[i]);
-                    w1[16 * hh + i] = An * w1[16 * hh + i] + sig * s;
-                    r[i] = __float_as_uint(En * s);
-                }
-                tmem_st16(t_s + 16 * hh, r);
+                for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(p1[16 * blk + i]);
+                tmem_st16(t_s + 16 * blk, r);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(p2[(size_t)(16 * blk + i) * kH]);
+                tmem_st16(t_s + 64 + 16 * blk, r);
             }
 #pragma unroll
-            for (int hh = 0; hh < 4; ++hh) {
-                uint32_t r[16];
-                tmem_ld16(t_s + 64 + 16 * hh, r);
-                tmem_wait_ld();
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const float s = __uint_as_float(r[i]);
-                    w2[16 * hh + i] = An * w2[16 * hh + i] + sig * s;
-                    r[i] = __float_as_uint(En * s);
-                }
-                tmem_st16(t_s + 64 + 16 * hh, r);
-            }
-            for (int qc = tid; qc < 512; qc += kThreads) {  // 16-byte chunks of the K tile
-                const uint32_t off = (uint32_t)qc * 16u;
-                const int row = qc >> 3;
-                const uint4 kv = ld_shared_v4(sb + KQb + off);
-                const float cr = -s_c[row], dr = -s_d[row];
-                const uint32_t in[4] = {kv.x, kv.y, kv.z, kv.w};
-                uint32_t oc[4], od[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float2 f = unpack_bf16x2(in[e]);
-                    oc[e] = pack_bf16x2(cr * f.x, cr * f.y);
-                    od[e] = pack_bf16x2(dr * f.x, dr * f.y);
-                }
-                st_shared_v4(sb + KC + off, oc[0], oc[1], oc[2], oc[3]);
-                st_shared_v4(sb + KD + off, od[0], od[1], od[2], od[3]);
+            for (int blk = 0; blk < 4; ++blk) {
+                store16_bf16(sb + W1, hrow, blk, w1 + 16 * blk);
+                store16_bf16(sb + W2T, hrow, blk, w2 + 16 * blk);
             }
             tmem_wait_st();
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(&bars[B_W0 + tile]);  // completion 0: the weights of "chunk -1"
         }
-        wait_mma();  // Z^T ready
 
-        // (D) A = silu(Z): keys -> AT0 (and silu'(Z_K) back into TMEM), queries -> AT1
-#pragma unroll
-        for (int cb = 0; cb < 8; ++cb) {  // 16-column blocks: 0..3 keys, 4..7 queries
-            uint32_t r[16];
-            tmem_ld16(t_work + 16 * cb, r);
-            tmem_wait_ld();
-            uint32_t pk[8];
-#pragma unroll
-            for (int i = 0; i < 16; i += 2) {
-                const float z0 = __uint_as_float(r[i]), z1 = __uint_as_float(r[i + 1]);
-                const float s0 = sigmoidf_fast(z0), s1 = sigmoidf_fast(z1);
-                pk[i / 2] = pack_bf16x2(z0 * s0, z1 * s1);
-                r[i] = __float_as_uint(s0 * (1.f + z0 * (1.f - s0)));
-                r[i + 1] = __float_as_uint(s1 * (1.f + z1 * (1.f - s1)));
-            }
-            const uint32_t tile = (cb < 4 ? AT0 : AT1), ch0 = (cb & 3) * 2;
-#pragma unroll
-            for (int ch = 0; ch < 2; ++ch) {
-                const uint32_t addr = sb + tile + (uint32_t)hrow * 128u + ((uint32_t)((ch0 + ch) ^ (hrow & 7)) << 4);
-                st_shared_v4(addr, pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
-            }
-            if (cb < 4) tmem_st16(t_work + 16 * cb, r);
-        }
-        tmem_wait_st();
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (*abort_flag) break;
+        for (int c = 0; c < nchunks; ++c) {
+            const int p = c & 1;
+            const uint32_t ph = (uint32_t)c & 1u;
+            const long t0 = (long)c * chunk;
+            const int n = (int)min((long)chunk, T - t0);
 
-        // (E) Y = A W2^T for keys (rows 0..63) and queries (rows 64..127) -> TMEM cols 64..127
-        if (tid == 0) {
+            // (1) momentum pre-pass: W <- A W + sigma S, S <- E S (the d-GEMMs then add -sum d_j g_j)
+            if (!wait(B_SC0 + p, (uint32_t)(c >> 1) & 1u)) break;
+            {
+                const float An = s_scal[4 * p], En = s_scal[4 * p + 1], sig = s_scal[4 * p + 2];
+#pragma unroll
+                for (int blk = 0; blk < 4; ++blk) {
+                    uint32_t r1[16], r2[16];
+                    tmem_ld16(t_s + 16 * blk, r1);
+                    tmem_ld16(t_s + 64 + 16 * blk, r2);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const float s1 = __uint_as_float(r1[i]), s2 = __uint_as_float(r2[i]);
+                        w1[16 * blk + i] = fmaf(An, w1[16 * blk + i], sig * s1);
+                        w2[16 * blk + i] = fmaf(An, w2[16 * blk + i], sig * s2);
+                        r1[i] = __float_as_uint(En * s1);
+                        r2[i] = __float_as_uint(En * s2);
+                    }
+                    tmem_st16(t_s + 16 * blk, r1);
+                    tmem_st16(t_s + 64 + 16 * blk, r2);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(&bars[B_S0 + tile]);
+            }
+
+            // (2) A = silu(Z): keys -> AT0 (and silu'(Z_K) into TMEM), queries -> AT1
+            if (!wait(B_Z0 + tile, ph)) break;
             tc_fence_after();
 #pragma unroll
-            for (int ks = 0; ks < 16; ++ks)
-                umma_bf16(tmem + 64, sdesc_sw128(sb + AT0 + ks * 2048, AT1 - AT0, 1024),
-                          sdesc_sw128(sb + W2T + ks * 2048, 8192, 1024), idY, ks > 0);
-            umma_commit(bar_mma);
-            mma_pending = true;
-        }
-        wait_mma();
-
-        // (F) keys: G = 2 (M(k) - v) and its scaled copies; queries: y
-        {
-            const int row = quad * 32 + lane;  // TMEM lane = token row of Y
+            for (int blk = 0; blk < 4; ++blk) {  // keys and queries, 16-column blocks
+                uint32_t rk[16], rq[16];
+                tmem_ld16(t_work + 16 * blk, rk);
+                tmem_ld16(t_work + 64 + 16 * blk, rq);
+                tmem_wait_ld();
+                float ak[16], aq[16];
 #pragma unroll
-            for (int hb = 0; hb < 2; ++hb) {
-                const int col0 = half * 32 + 16 * hb;
-                uint32_t r[16];
-                tmem_ld16(tmem + lane_off + 64 + col0, r);
+                for (int i = 0; i < 16; ++i) {
+                    // silu(z) = h (1 + tanh h), silu'(z) = (1 + tanh h + h (1 - tanh^2 h)) / 2, h = z / 2
+                    const float hk = 0.5f * __uint_as_float(rk[i]);
+                    const float tk = tanh_approx(hk);
+                    ak[i] = fmaf(hk, tk, hk);
+                    rk[i] = __float_as_uint(fmaf(0.5f, tk + fmaf(-hk * tk, tk, hk), 0.5f));
+                    const float hq = 0.5f * __uint_as_float(rq[i]);
+                    aq[i] = fmaf(hq, tanh_approx(hq), hq);
+                }
+                store16_bf16(sb + AT0, hrow, blk, ak);
+                store16_bf16(sb + AT1, hrow, blk, aq);
+                tmem_st16(t_work + 16 * blk, rk);
+            }
+            tmem_wait_st();
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(&bars[B_A0 + tile]);
+
+            // (3) G = 2 (M(k) - v) and its scaled copies (keys), y (queries). Token row = TMEM
+            //     lane (quadrant quad), this warp's 32 of the 64 columns: [32 tile, 32 tile + 32).
+            if (!wait(B_Y, ph)) break;
+            if (!wait(B_TMA0 + (c & 1), (uint32_t)(c >> 1) & 1u)) break;  // the V tile, read below
+            tc_fence_after();
+            {
+                const int row = quad * 32 + lane;
+                const uint32_t Vb = (c & 1) ? V1 : V0;
+                uint32_t r[32];
+                tmem_ld16(tmem + lane_off + 64 + 32 * tile, *reinterpret_cast<uint32_t(*)[16]>(r));
+                tmem_ld16(tmem + lane_off + 64 + 32 * tile + 16, *reinterpret_cast<uint32_t(*)[16]>(r + 16));
                 tmem_wait_ld();
                 if (row < kN) {
-                    const float cr = -s_c[row], dr = -s_d[row];
+                    const float cr = -s_cc[64 * p + row], dr = -s_dd[64 * p + row];
 #pragma unroll
-                    for (int ch = 0; ch < 2; ++ch) {
-                        const uint32_t off = sw128_off((uint32_t)row, (uint32_t)(col0 + 8 * ch));
+                    for (int ch = 0; ch < 4; ++ch) {
+                        const uint32_t off = sw128_off((uint32_t)row, (uint32_t)(32 * tile + 8 * ch));
                         const uint4 vv = ld_shared_v4(sb + Vb + off);
                         const uint32_t vin[4] = {vv.x, vv.y, vv.z, vv.w};
                         uint32_t og[4], oc[4], od[4];
@@ -436,9 +558,9 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
                         st_shared_v4(sb + GD + off, od[0], od[1], od[2], od[3]);
                     }
                 } else if (row - kN < n) {
-                    uint4* dst = reinterpret_cast<uint4*>(yg + ((u * T + t0 + (row - kN)) * kD + col0));
+                    uint4* dst = reinterpret_cast<uint4*>(yg + ((u * T + t0 + (row - kN)) * kD + 32 * tile));
 #pragma unroll
-                    for (int ch = 0; ch < 2; ++ch) {
+                    for (int ch = 0; ch < 4; ++ch) {
                         uint4 o;
                         o.x = pack_bf16x2(__uint_as_float(r[8 * ch]), __uint_as_float(r[8 * ch + 1]));
                         o.y = pack_bf16x2(__uint_as_float(r[8 * ch + 2]), __uint_as_float(r[8 * ch + 3]));
@@ -448,129 +570,75 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
                     }
                 }
             }
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (*abort_flag) break;
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(&bars[B_G]);
 
-        // (G) (GW2)^T = W2^T G^T -> tile t cols 128t+64..; S2^T += A_K^T diag(-d) G
-        if (tid == 0) {
+            // (4) Delta^T = (GW2)^T * silu'(Z_K)^T -> AT1 rows (the queries' tile was consumed by Y)
+            if (!wait(B_GW0 + tile, ph)) break;
             tc_fence_after();
 #pragma unroll
-            for (int t = 0; t < 2; ++t)
+            for (int blk = 0; blk < 4; ++blk) {
+                uint32_t g[16], sp[16];
+                tmem_ld16(t_work + 64 + 16 * blk, g);
+                tmem_ld16(t_work + 16 * blk, sp);
+                tmem_wait_ld();
+                float x[16];
 #pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    umma_bf16(tmem + t * 128 + 64, sdesc_sw128(sb + W2T + t * 16384 + ks * 32, 16, 1024),
-                              sdesc_sw128(sb + G + ks * 32, 16, 1024), idG, ks > 0);
-#pragma unroll
-            for (int t = 0; t < 2; ++t)
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    umma_bf16(tmem + 256 + t * 128 + 64, sdesc_sw128(sb + AT0 + t * 16384 + ks * 32, 16, 1024),
-                              sdesc_sw128(sb + GD + ks * 2048, 8192, 1024), idW, 1);
-            umma_commit(bar_mma);
-            mma_pending = true;
-        }
-        wait_mma();
-
-        // (H) Delta^T = (GW2)^T * silu'(Z_K)^T -> AT1 (the queries' tile is no longer needed)
-#pragma unroll
-        for (int cb = 0; cb < 4; ++cb) {
-            uint32_t g[16], s[16];
-            tmem_ld16(t_work + 64 + 16 * cb, g);
-            tmem_ld16(t_work + 16 * cb, s);
-            tmem_wait_ld();
-#pragma unroll
-            for (int ch = 0; ch < 2; ++ch) {
-                const uint32_t addr =
-                    sb + AT1 + (uint32_t)hrow * 128u + ((uint32_t)((2 * cb + ch) ^ (hrow & 7)) << 4);
-                float x[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) x[e] = __uint_as_float(g[8 * ch + e]) * __uint_as_float(s[8 * ch + e]);
-                st_shared_v4(addr, pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
-                             pack_bf16x2(x[6], x[7]));
+                for (int i = 0; i < 16; ++i) x[i] = __uint_as_float(g[i]) * __uint_as_float(sp[i]);
+                store16_bf16(sb + AT1, hrow, blk, x);
             }
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (*abort_flag) break;
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(&bars[B_D0 + tile]);
 
-        // (I) dW1_c' -> cols 128t, S1 += Delta^T diag(-d) K, dW2^T_c' -> cols 128t+64; prefetch chunk c+2
-        if (tid == 0) {
+            // (5) W <- (A W + sigma S) - sum_j c_j g_j; rewrite the bf16 operand rows
+            if (!wait(B_DW0 + tile, ph)) break;
             tc_fence_after();
 #pragma unroll
-            for (int t = 0; t < 2; ++t)
+            for (int blk = 0; blk < 4; ++blk) {
+                uint32_t r1[16], r2[16];
+                tmem_ld16(t_work + 16 * blk, r1);
+                tmem_ld16(t_work + 64 + 16 * blk, r2);
+                tmem_wait_ld();
 #pragma unroll
-                for (int ks = 0; ks < 4; ++ks) {
-                    const uint64_t dA = sdesc_sw128(sb + AT1 + t * 16384 + ks * 32, 16, 1024);
-                    const uint64_t aA = sdesc_sw128(sb + AT0 + t * 16384 + ks * 32, 16, 1024);
-                    umma_bf16(tmem + t * 128, dA, sdesc_sw128(sb + KC + ks * 2048, 8192, 1024), idW, ks > 0);
-                    umma_bf16(tmem + 256 + t * 128, dA, sdesc_sw128(sb + KD + ks * 2048, 8192, 1024), idW, 1);
-                    umma_bf16(tmem + t * 128 + 64, aA, sdesc_sw128(sb + GC + ks * 2048, 8192, 1024), idW, ks > 0);
+                for (int i = 0; i < 16; ++i) {
+                    w1[16 * blk + i] += __uint_as_float(r1[i]);
+                    w2[16 * blk + i] += __uint_as_float(r2[i]);
                 }
-            umma_commit(bar_mma);
-            mma_pending = true;
-            if (c + 2 < nchunks) issue_tma(c + 2, buf);
+                store16_bf16(sb + W1, hrow, blk, w1 + 16 * blk);
+                store16_bf16(sb + W2T, hrow, blk, w2 + 16 * blk);
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(&bars[B_W0 + tile]);
         }
-        wait_mma();
 
-        // (J) W <- (A W + sigma S) - sum_j c_j g_j; refresh the bf16 operand copies
+        // Final state of this hidden row (every MMA of the last chunk has completed).
+        {
+            float4* p = reinterpret_cast<float4*>(W1g + (u * kH + hrow) * kD);
 #pragma unroll
-        for (int cb = 0; cb < 4; ++cb) {
-            uint32_t r1[16], r2[16];
-            tmem_ld16(t_work + 16 * cb, r1);
-            tmem_ld16(t_work + 64 + 16 * cb, r2);
-            tmem_wait_ld();
+            for (int i = 0; i < 16; ++i) p[i] = make_float4(w1[4 * i], w1[4 * i + 1], w1[4 * i + 2], w1[4 * i + 3]);
+            float* q2 = W2g + u * kD * kH + hrow;
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                w1[16 * cb + i] += __uint_as_float(r1[i]);
-                w2[16 * cb + i] += __uint_as_float(r2[i]);
+            for (int i = 0; i < 64; ++i) q2[(size_t)i * kH] = w2[i];
+            float* p1 = S1g + (u * kH + hrow) * kD;
+            float* p2 = S2g + u * kD * kH + hrow;
+#pragma unroll
+            for (int blk = 0; blk < 4; ++blk) {
+                uint32_t r[16];
+                tmem_ld16(t_s + 16 * blk, r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 16; ++i) p1[16 * blk + i] = __uint_as_float(r[i]);
+                tmem_ld16(t_s + 64 + 16 * blk, r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 16; ++i) p2[(size_t)(16 * blk + i) * kH] = __uint_as_float(r[i]);
             }
         }
-        store_row_bf16(sb + W1, hrow, w1);
-        store_row_bf16(sb + W2T, hrow, w2);
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (*abort_flag) break;
     }
 
-    // Drain (only after an abort can copies or MMAs still be in flight), then write the state.
-    if (tid == 0) {
-        for (int b = 0; b < 2; ++b)
-            while (tma_done[b] < tma_issued[b]) {
-                if (!mbar_wait(&bar_tma[b], tma_done[b] & 1u)) break;
-                ++tma_done[b];
-            }
-        if (mma_pending) mbar_wait(bar_mma, mma_phase);
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    {
-        float4* p = reinterpret_cast<float4*>(W1g + (u * kH + hrow) * kD);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) p[i] = make_float4(w1[4 * i], w1[4 * i + 1], w1[4 * i + 2], w1[4 * i + 3]);
-        float* q2 = W2g + u * kD * kH + hrow;
-#pragma unroll
-        for (int i = 0; i < 64; ++i) q2[(size_t)i * kH] = w2[i];
-        float* p1 = S1g + (u * kH + hrow) * kD;
-        float* p2 = S2g + u * kD * kH + hrow;
-#pragma unroll
-        for (int hh = 0; hh < 4; ++hh) {
-            uint32_t r[16];
-            tmem_ld16(t_s + 16 * hh, r);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 16; ++i) p1[16 * hh + i] = __uint_as_float(r[i]);
-            tmem_ld16(t_s + 64 + 16 * hh, r);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 16; ++i) p2[(size_t)(16 * hh + i) * kH] = __uint_as_float(r[i]);
-        }
-    }
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
