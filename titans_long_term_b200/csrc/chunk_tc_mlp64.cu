@@ -24,9 +24,14 @@
 //   - warps 0-3 own hidden rows 0..127 ("tile 0"), warps 4-7 rows 128..255 ("tile 1");
 //     the two tiles run their epilogues independently, so the tensor core works on one
 //     tile while the other tile's warps run theirs;
-//   - warp 8 issues TMA (K, Q, V tiles two chunks ahead) and every MMA (lane 0), and
-//     computes the next chunk's gate scan and scaled key tiles; warps 9-11 only complete
-//     its warpgroup, which hands its registers to the epilogue warpgroups (setmaxnreg).
+//   - warps 8 and 9 issue the MMAs of tile 0 and tile 1 (one elected lane each: a single
+//     thread issues a tcgen05.mma only every ~80 cycles, two issuers double the rate);
+//     Y is split into the two tiles' partial sums over their hidden units, so the two
+//     issuers never need to be ordered; warp 8 also issues the TMA loads (K, Q, V two
+//     chunks ahead);
+//   - warp 10 prefetches the gates, runs the gate scan a chunk ahead and writes the scaled
+//     key tiles; warp 11 only completes the producer warpgroup, which hands registers to
+//     the epilogue warpgroups (setmaxnreg).
 // Hand-offs go through mbarriers only; every wait is bounded.
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -69,7 +74,7 @@ enum Bar {
     B_TMA0, B_TMA1,      // K, Q, V tiles landed (buffer 0 / 1)
     B_Z0, B_Z1,          // Z^T of tile t done
     B_A0, B_A1,          // tile t wrote its silu rows (and silu' into TMEM)
-    B_Y,                 // Y done
+    B_Y0, B_Y1,          // partial Y of tile t (sum over its hidden units) done
     B_G,                 // G tiles written, Y read (all epilogue threads)
     B_S0, B_S1,          // tile t's momentum pre-pass done
     B_GW0, B_GW1,        // (GW2)^T and the S2^T accumulation of tile t done
@@ -77,6 +82,7 @@ enum Bar {
     B_DW0, B_DW1,        // weighted weight GEMMs of tile t done
     B_W0, B_W1,          // tile t rewrote its bf16 weight rows (and read dW_c)
     B_SC0, B_SC1,        // gate scan of a chunk with parity 0 / 1 published
+    B_KC,                // scaled key tiles of the chunk written
     kNumBars
 };
 constexpr uint32_t TPTR = BAR + 8 * kNumBars;  // TMEM base address
@@ -86,7 +92,7 @@ constexpr size_t kSmemBytes = END + 1024;  // + alignment slack
 // TMEM columns: [0, 256) working region, [256, 512) momentum S.
 //   working, tile t (hidden rows 128t..128t+127) at column 128t:
 //     +0..63   Z_K^T, then silu'(Z_K)^T, then dW1_c
-//     +64..127 Z_Q^T, then (GW2)^T, then dW2^T_c     (tile 0's +64..127 also hosts Y)
+//     +64..127 Z_Q^T, then the partial Y of tile t, then (GW2)^T, then dW2^T_c
 //   S region, tile t at column 256 + 128t: +0..63 S1 rows, +64..127 S2^T rows.
 constexpr uint32_t kTmemCols = 512;
 }  // namespace tc
@@ -213,7 +219,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
                 cnt = 128;
             else if (b == B_G)
                 cnt = 256;
-            else if (b == B_SC0 || b == B_SC1)
+            else if (b == B_SC0 || b == B_SC1 || b == B_KC)
                 cnt = 32;
             mbar_init(&bars[b], cnt);
         }
@@ -243,27 +249,9 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
     if (warp >= kEpiWarps) {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsProducer));
     }
-    if (warp > kEpiWarps) {
-        // warps 9..11: nothing to do
-    } else if (warp == kEpiWarps) {
-        // =========================== issuer warp: TMA, MMAs, gate scans, scaled key tiles
-        const uint32_t idZ = idesc_bf16_f32(128, 128, 0, 0);
-        const uint32_t idY = idesc_bf16_f32(128, 64, 1, 1);
-        const uint32_t idG = idesc_bf16_f32(128, 64, 0, 0);
-        const uint32_t idW = idesc_bf16_f32(128, 64, 0, 1);
-        const uint32_t tx_bytes = 3u * (uint32_t)chunk * 128u;
-        uint32_t tma_issued = 0, tma_waited = 0;  // counts per buffer packed: bits [0,16) buf 0, [16,32) buf 1
-        auto issue_tma = [&](int c) {
-            const int b = c & 1;
-            const uint32_t kq = b ? KQ1 : KQ0, vv = b ? V1 : V0;
-            mbar_arrive_expect_tx(&bars[B_TMA0 + b], tx_bytes);
-            tma_load_3d(sm + kq, &tmK, &bars[B_TMA0 + b], 0, c * chunk, (int)u);
-            tma_load_3d(sm + kq + 8192, &tmQ, &bars[B_TMA0 + b], 0, c * chunk, (int)u);
-            tma_load_3d(sm + vv, &tmV, &bars[B_TMA0 + b], 0, c * chunk, (int)u);
-            tma_issued += b ? 0x10000u : 1u;
-        };
-        // Gates of chunk c travel in registers (lane l holds tokens l and l + 32) one chunk ahead.
-        float ga[2], ge[2], gt[2];
+    if (warp == kEpiWarps + 2) {
+        // =========================== scan warp: gates, gate scans, scaled key tiles
+        float ga[2], ge[2], gt[2];  // gates of one chunk, lane l holds tokens l and l + 32
         auto load_gates = [&](int c) {
             const long t0 = (long)c * chunk;
             const long n = c < nchunks ? min((long)chunk, T - t0) : 0;
@@ -293,38 +281,16 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
             __syncwarp();
             mbar_arrive(&bars[B_SC0 + p]);
         };
-        if (lane == 0) {
-            prefetch_tmap(&tmK);
-            prefetch_tmap(&tmQ);
-            prefetch_tmap(&tmV);
-            issue_tma(0);
-            if (nchunks > 1) issue_tma(1);
-        }
         load_gates(0);
         scan(0);
         load_gates(1);
-
         for (int c = 0; c < nchunks; ++c) {
-            const int b = c & 1, p = c & 1;
-            const uint32_t ph = (uint32_t)c & 1u;
-            const uint32_t KQb = b ? KQ1 : KQ0;
-            bool ok = wait(B_TMA0 + b, (uint32_t)(c >> 1) & 1u);
-            if (ok) tma_waited += b ? 0x10000u : 1u;
-            // Z^T of tile t once tile t has rewritten its weight rows (after chunk c-1).
-            for (int t = 0; t < 2 && ok; ++t) {
-                ok = wait(B_W0 + t, ph);
-                if (ok && lane == 0) {
-                    tc_fence_after();
-#pragma unroll
-                    for (int ks = 0; ks < 4; ++ks)
-                        umma_bf16(tmem + t * 128, sdesc_sw128(sb + W1 + t * 16384 + ks * 32, 16, 1024),
-                                  sdesc_sw128(sb + KQb + ks * 32, 16, 1024), idZ, ks > 0);
-                    umma_commit(&bars[B_Z0 + t]);
-                }
-            }
-            if (!ok || *abort_flag) break;
-            // Scaled key tiles of this chunk (the previous chunk's weight GEMMs, which read them,
-            // completed before tile 1 signalled B_W1 above).
+            const int p = c & 1;
+            const uint32_t KQb = (c & 1) ? KQ1 : KQ0;
+            if (!wait(B_TMA0 + (c & 1), (uint32_t)(c >> 1) & 1u)) break;
+            // The previous chunk's weight GEMMs of both tiles (which read the scaled key tiles;
+            // every reader of the other scan buffer finished before them) have completed.
+            if (c > 0 && (!wait(B_DW0, (uint32_t)(c - 1) & 1u) || !wait(B_DW1, (uint32_t)(c - 1) & 1u))) break;
             {
                 const float* cc = s_cc + 64 * p;
                 const float* dd = s_dd + 64 * p;
@@ -346,70 +312,115 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
                     st_shared_v4(sb + KD + off, od[0], od[1], od[2], od[3]);
                 }
                 fence_proxy_async_smem();
-                __syncwarp();
+                mbar_arrive(&bars[B_KC]);
             }
-            // Next chunk's gate scan (its gates are already in registers), then prefetch the one after.
             if (c + 1 < nchunks) {
                 scan(c + 1);
                 load_gates(c + 2);
             }
-            // Y = A W2^T: the K dimension (hidden units) in two halves, one per tile.
-            for (int t = 0; t < 2 && ok; ++t) {
-                ok = wait(B_A0 + t, ph);
-                if (ok && lane == 0) {
-                    tc_fence_after();
-#pragma unroll
-                    for (int ks = 8 * t; ks < 8 * t + 8; ++ks)
-                        umma_bf16(tmem + 64, sdesc_sw128(sb + AT0 + ks * 2048, AT1 - AT0, 1024),
-                                  sdesc_sw128(sb + W2T + ks * 2048, 8192, 1024), idY, ks > 0);
-                    if (t == 1) umma_commit(&bars[B_Y]);
-                }
+        }
+    } else if (warp > kEpiWarps + 1) {
+        // warp 11: nothing to do
+    } else if (warp >= kEpiWarps) {
+        // =========================== issuer warps: warp 8 + t issues tile t's MMAs (warp 8 also TMA)
+        const int t = warp - kEpiWarps;
+        const uint32_t idZ = idesc_bf16_f32(128, 128, 0, 0);
+        const uint32_t idY = idesc_bf16_f32(128, 64, 1, 1);
+        const uint32_t idG = idesc_bf16_f32(128, 64, 0, 0);
+        const uint32_t idW = idesc_bf16_f32(128, 64, 0, 1);
+        const uint32_t tx_bytes = 3u * (uint32_t)chunk * 128u;
+        // Descriptor bases at offset 0 of shared memory; a tile at byte offset X is base + X / 16
+        // (the start-address field is the low 14 bits and every address stays below 256 KB).
+        const uint64_t dK = sdesc_sw128(sb, 16, 1024);            // K-major, 8-row groups 1024 B apart
+        const uint64_t dMN32 = sdesc_sw128(sb, AT1 - AT0, 1024);  // MN-major, 64-element blocks 32 KB apart
+        const uint64_t dMN8 = sdesc_sw128(sb, 8192, 1024);        // MN-major, single 64-element block
+#define DSC(base, off) ((base) + (uint64_t)((off) >> 4))
+        uint32_t tma_issued = 0, tma_waited = 0;  // counts per buffer packed: bits [0,16) buf 0, [16,32) buf 1
+        auto issue_tma = [&](int c) {
+            const int b = c & 1;
+            const uint32_t kq = b ? KQ1 : KQ0, vv = b ? V1 : V0;
+            mbar_arrive_expect_tx(&bars[B_TMA0 + b], tx_bytes);
+            tma_load_3d(sm + kq, &tmK, &bars[B_TMA0 + b], 0, c * chunk, (int)u);
+            tma_load_3d(sm + kq + 8192, &tmQ, &bars[B_TMA0 + b], 0, c * chunk, (int)u);
+            tma_load_3d(sm + vv, &tmV, &bars[B_TMA0 + b], 0, c * chunk, (int)u);
+            tma_issued += b ? 0x10000u : 1u;
+        };
+        if (t == 0 && lane == 0) {
+            prefetch_tmap(&tmK);
+            prefetch_tmap(&tmQ);
+            prefetch_tmap(&tmV);
+            issue_tma(0);
+            if (nchunks > 1) issue_tma(1);
+        }
+        for (int c = 0; c < nchunks; ++c) {
+            const int b = c & 1;
+            const uint32_t ph = (uint32_t)c & 1u;
+            const uint32_t KQb = b ? KQ1 : KQ0;
+            bool ok = wait(B_TMA0 + b, (uint32_t)(c >> 1) & 1u);
+            if (ok) tma_waited += b ? 0x10000u : 1u;
+            // Z^T of tile t once tile t has rewritten its weight rows (after chunk c-1).
+            if (ok) ok = wait(B_W0 + t, ph);
+            if (ok && lane == 0) {
+                tc_fence_after();
+#pragma unroll 1
+                for (int ks = 0; ks < 4; ++ks)
+                    umma_bf16(tmem + t * 128, DSC(dK, W1 + t * 16384 + ks * 32), DSC(dK, KQb + ks * 32), idZ, ks > 0);
+                umma_commit(&bars[B_Z0 + t]);
+            }
+            if (!ok || *abort_flag) break;
+            // Partial Y of tile t: its 128 hidden units are K-steps 8t .. 8t+7 of A W2^T.
+            ok = wait(B_A0 + t, ph);
+            if (ok && lane == 0) {
+                tc_fence_after();
+#pragma unroll 1
+                for (int j = 0; j < 8; ++j)
+                    umma_bf16(tmem + t * 128 + 64, DSC(dMN32, AT0 + (8 * t + j) * 2048),
+                              DSC(dMN8, W2T + (8 * t + j) * 2048), idY, j > 0);
+                umma_commit(&bars[B_Y0 + t]);
             }
             if (!ok) break;
-            // G tiles written: the K, Q, V buffer of this chunk is free -> chunk c + 2.
-            ok = wait(B_G, ph);
+            ok = wait(B_G, ph);  // G tiles written, both partial Y read
             if (!ok) break;
-            if (lane == 0 && c + 2 < nchunks) issue_tma(c + 2);
-            // (GW2)^T = W2^T G^T and S2^T += A_K^T diag(-d) G, per tile once its S is pre-scaled.
-            for (int t = 0; t < 2 && ok; ++t) {
-                ok = wait(B_S0 + t, ph);
-                if (ok && lane == 0) {
-                    tc_fence_after();
-#pragma unroll
-                    for (int ks = 0; ks < 4; ++ks)
-                        umma_bf16(tmem + t * 128 + 64, sdesc_sw128(sb + W2T + t * 16384 + ks * 32, 16, 1024),
-                                  sdesc_sw128(sb + G + ks * 32, 16, 1024), idG, ks > 0);
-#pragma unroll
-                    for (int ks = 0; ks < 4; ++ks)
-                        umma_bf16(tmem + 256 + t * 128 + 64, sdesc_sw128(sb + AT0 + t * 16384 + ks * 32, 16, 1024),
-                                  sdesc_sw128(sb + GD + ks * 2048, 8192, 1024), idW, 1);
-                    umma_commit(&bars[B_GW0 + t]);
-                }
+            // (GW2)^T = W2^T G^T and S2^T += A_K^T diag(-d) G once tile t's S is pre-scaled.
+            ok = wait(B_S0 + t, ph);
+            if (ok && lane == 0) {
+                tc_fence_after();
+#pragma unroll 1
+                for (int ks = 0; ks < 4; ++ks)
+                    umma_bf16(tmem + t * 128 + 64, DSC(dK, W2T + t * 16384 + ks * 32), DSC(dK, G + ks * 32), idG,
+                              ks > 0);
+#pragma unroll 1
+                for (int ks = 0; ks < 4; ++ks)
+                    umma_bf16(tmem + 256 + t * 128 + 64, DSC(dK, AT0 + t * 16384 + ks * 32), DSC(dMN8, GD + ks * 2048),
+                              idW, 1);
+                umma_commit(&bars[B_GW0 + t]);
             }
             if (!ok) break;
-            // dW1_c -> cols 128t, S1 += Delta^T diag(-d) K, dW2^T_c -> cols 128t+64, per tile.
-            for (int t = 0; t < 2 && ok; ++t) {
-                ok = wait(B_D0 + t, ph);
-                if (ok && lane == 0) {
-                    tc_fence_after();
-#pragma unroll
-                    for (int ks = 0; ks < 4; ++ks) {
-                        const uint64_t dA = sdesc_sw128(sb + AT1 + t * 16384 + ks * 32, 16, 1024);
-                        const uint64_t aA = sdesc_sw128(sb + AT0 + t * 16384 + ks * 32, 16, 1024);
-                        umma_bf16(tmem + t * 128, dA, sdesc_sw128(sb + KC + ks * 2048, 8192, 1024), idW, ks > 0);
-                        umma_bf16(tmem + 256 + t * 128, dA, sdesc_sw128(sb + KD + ks * 2048, 8192, 1024), idW, 1);
-                        umma_bf16(tmem + t * 128 + 64, aA, sdesc_sw128(sb + GC + ks * 2048, 8192, 1024), idW,
-                                  ks > 0);
-                    }
-                    umma_commit(&bars[B_DW0 + t]);
+            // Scaled key tiles written: with the G tiles written before, every reader of this
+            // chunk's K, Q, V buffer is done -> chunk c + 2.
+            ok = wait(B_KC, ph);
+            if (ok && t == 0 && lane == 0 && c + 2 < nchunks) issue_tma(c + 2);
+            // dW1_c -> cols 128t, S1 += Delta^T diag(-d) K, dW2^T_c -> cols 128t+64.
+            if (ok) ok = wait(B_D0 + t, ph);
+            if (ok && lane == 0) {
+                tc_fence_after();
+#pragma unroll 1
+                for (int ks = 0; ks < 4; ++ks) {
+                    const uint64_t dA = DSC(dK, AT1 + t * 16384 + ks * 32);
+                    const uint64_t aA = DSC(dK, AT0 + t * 16384 + ks * 32);
+                    umma_bf16(tmem + t * 128, dA, DSC(dMN8, KC + ks * 2048), idW, ks > 0);
+                    umma_bf16(tmem + 256 + t * 128, dA, DSC(dMN8, KD + ks * 2048), idW, 1);
+                    umma_bf16(tmem + t * 128 + 64, aA, DSC(dMN8, GC + ks * 2048), idW, ks > 0);
                 }
+                umma_commit(&bars[B_DW0 + t]);
             }
             if (!ok) break;
             __syncwarp();
         }
+#undef DSC
         __syncwarp();
         // Drain: after an abort, copies may still be in flight into shared memory.
-        if (lane == 0) {
+        if (t == 0 && lane == 0) {
             for (int b = 0; b < 2; ++b) {
                 uint32_t iss = (tma_issued >> (16 * b)) & 0xFFFFu, don = (tma_waited >> (16 * b)) & 0xFFFFu;
                 while (don < iss) {
@@ -504,20 +515,27 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
                 tmem_ld16(t_work + 16 * blk, rk);
                 tmem_ld16(t_work + 64 + 16 * blk, rq);
                 tmem_wait_ld();
-                float ak[16], aq[16];
+                uint32_t pk[8], pq[8];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
+                for (int i = 0; i < 16; i += 2) {
                     // silu(z) = h (1 + tanh h), silu'(z) = (1 + tanh h + h (1 - tanh^2 h)) / 2, h = z / 2
-                    const float hk = 0.5f * __uint_as_float(rk[i]);
-                    const float tk = tanh_approx(hk);
-                    ak[i] = fmaf(hk, tk, hk);
-                    rk[i] = __float_as_uint(fmaf(0.5f, tk + fmaf(-hk * tk, tk, hk), 0.5f));
-                    const float hq = 0.5f * __uint_as_float(rq[i]);
-                    aq[i] = fmaf(hq, tanh_approx(hq), hq);
+                    const float h0 = 0.5f * __uint_as_float(rk[i]), h1 = 0.5f * __uint_as_float(rk[i + 1]);
+                    const float t0_ = tanh_approx(h0), t1_ = tanh_approx(h1);
+                    pk[i / 2] = pack_bf16x2(fmaf(h0, t0_, h0), fmaf(h1, t1_, h1));
+                    rk[i] = __float_as_uint(fmaf(0.5f, t0_ + fmaf(-h0 * t0_, t0_, h0), 0.5f));
+                    rk[i + 1] = __float_as_uint(fmaf(0.5f, t1_ + fmaf(-h1 * t1_, t1_, h1), 0.5f));
+                    const float g0 = 0.5f * __uint_as_float(rq[i]), g1 = 0.5f * __uint_as_float(rq[i + 1]);
+                    pq[i / 2] = pack_bf16x2(fmaf(g0, tanh_approx(g0), g0), fmaf(g1, tanh_approx(g1), g1));
                 }
-                store16_bf16(sb + AT0, hrow, blk, ak);
-                store16_bf16(sb + AT1, hrow, blk, aq);
                 tmem_st16(t_work + 16 * blk, rk);
+#pragma unroll
+                for (int ch = 0; ch < 2; ++ch) {
+                    const uint32_t sw = (uint32_t)((2 * blk + ch) ^ (hrow & 7)) << 4;
+                    st_shared_v4(sb + AT0 + (uint32_t)hrow * 128u + sw, pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2],
+                                 pk[4 * ch + 3]);
+                    st_shared_v4(sb + AT1 + (uint32_t)hrow * 128u + sw, pq[4 * ch], pq[4 * ch + 1], pq[4 * ch + 2],
+                                 pq[4 * ch + 3]);
+                }
             }
             tmem_wait_st();
             fence_proxy_async_smem();
@@ -526,47 +544,54 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
 
             // (3) G = 2 (M(k) - v) and its scaled copies (keys), y (queries). Token row = TMEM
             //     lane (quadrant quad), this warp's 32 of the 64 columns: [32 tile, 32 tile + 32).
-            if (!wait(B_Y, ph)) break;
+            if (!wait(B_Y0, ph) || !wait(B_Y1, ph)) break;
             if (!wait(B_TMA0 + (c & 1), (uint32_t)(c >> 1) & 1u)) break;  // the V tile, read below
             tc_fence_after();
             {
                 const int row = quad * 32 + lane;
                 const uint32_t Vb = (c & 1) ? V1 : V0;
-                uint32_t r[32];
-                tmem_ld16(tmem + lane_off + 64 + 32 * tile, *reinterpret_cast<uint32_t(*)[16]>(r));
-                tmem_ld16(tmem + lane_off + 64 + 32 * tile + 16, *reinterpret_cast<uint32_t(*)[16]>(r + 16));
-                tmem_wait_ld();
-                if (row < kN) {
-                    const float cr = -s_cc[64 * p + row], dr = -s_dd[64 * p + row];
+                const bool key = row < kN, query = !key && row - kN < n;
+                const float cr = key ? -s_cc[64 * p + row] : 0.f, dr = key ? -s_dd[64 * p + row] : 0.f;
+#pragma unroll 1
+                for (int hb = 0; hb < 2; ++hb) {
+                    const int col0 = 32 * tile + 16 * hb;
+                    uint32_t r[16], r2[16];
+                    tmem_ld16(tmem + lane_off + 64 + col0, r);         // tile 0's partial Y
+                    tmem_ld16(tmem + lane_off + 128 + 64 + col0, r2);  // tile 1's partial Y
+                    tmem_wait_ld();
 #pragma unroll
-                    for (int ch = 0; ch < 4; ++ch) {
-                        const uint32_t off = sw128_off((uint32_t)row, (uint32_t)(32 * tile + 8 * ch));
-                        const uint4 vv = ld_shared_v4(sb + Vb + off);
-                        const uint32_t vin[4] = {vv.x, vv.y, vv.z, vv.w};
-                        uint32_t og[4], oc[4], od[4];
+                    for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) + __uint_as_float(r2[i]));
+                    if (key) {
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float2 vf = unpack_bf16x2(vin[e]);
-                            const float g0 = 2.f * (__uint_as_float(r[8 * ch + 2 * e]) - vf.x);
-                            const float g1 = 2.f * (__uint_as_float(r[8 * ch + 2 * e + 1]) - vf.y);
-                            og[e] = pack_bf16x2(g0, g1);
-                            oc[e] = pack_bf16x2(cr * g0, cr * g1);
-                            od[e] = pack_bf16x2(dr * g0, dr * g1);
+                        for (int ch = 0; ch < 2; ++ch) {
+                            const uint32_t off = sw128_off((uint32_t)row, (uint32_t)(col0 + 8 * ch));
+                            const uint4 vv = ld_shared_v4(sb + Vb + off);
+                            const uint32_t vin[4] = {vv.x, vv.y, vv.z, vv.w};
+                            uint32_t og[4], oc[4], od[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const float2 vf = unpack_bf16x2(vin[e]);
+                                const float g0 = 2.f * (__uint_as_float(r[8 * ch + 2 * e]) - vf.x);
+                                const float g1 = 2.f * (__uint_as_float(r[8 * ch + 2 * e + 1]) - vf.y);
+                                og[e] = pack_bf16x2(g0, g1);
+                                oc[e] = pack_bf16x2(cr * g0, cr * g1);
+                                od[e] = pack_bf16x2(dr * g0, dr * g1);
+                            }
+                            st_shared_v4(sb + G + off, og[0], og[1], og[2], og[3]);
+                            st_shared_v4(sb + GC + off, oc[0], oc[1], oc[2], oc[3]);
+                            st_shared_v4(sb + GD + off, od[0], od[1], od[2], od[3]);
                         }
-                        st_shared_v4(sb + G + off, og[0], og[1], og[2], og[3]);
-                        st_shared_v4(sb + GC + off, oc[0], oc[1], oc[2], oc[3]);
-                        st_shared_v4(sb + GD + off, od[0], od[1], od[2], od[3]);
-                    }
-                } else if (row - kN < n) {
-                    uint4* dst = reinterpret_cast<uint4*>(yg + ((u * T + t0 + (row - kN)) * kD + 32 * tile));
+                    } else if (query) {
+                        uint4* dst = reinterpret_cast<uint4*>(yg + ((u * T + t0 + (row - kN)) * kD + col0));
 #pragma unroll
-                    for (int ch = 0; ch < 4; ++ch) {
-                        uint4 o;
-                        o.x = pack_bf16x2(__uint_as_float(r[8 * ch]), __uint_as_float(r[8 * ch + 1]));
-                        o.y = pack_bf16x2(__uint_as_float(r[8 * ch + 2]), __uint_as_float(r[8 * ch + 3]));
-                        o.z = pack_bf16x2(__uint_as_float(r[8 * ch + 4]), __uint_as_float(r[8 * ch + 5]));
-                        o.w = pack_bf16x2(__uint_as_float(r[8 * ch + 6]), __uint_as_float(r[8 * ch + 7]));
-                        dst[ch] = o;
+                        for (int ch = 0; ch < 2; ++ch) {
+                            uint4 o;
+                            o.x = pack_bf16x2(__uint_as_float(r[8 * ch]), __uint_as_float(r[8 * ch + 1]));
+                            o.y = pack_bf16x2(__uint_as_float(r[8 * ch + 2]), __uint_as_float(r[8 * ch + 3]));
+                            o.z = pack_bf16x2(__uint_as_float(r[8 * ch + 4]), __uint_as_float(r[8 * ch + 5]));
+                            o.w = pack_bf16x2(__uint_as_float(r[8 * ch + 6]), __uint_as_float(r[8 * ch + 7]));
+                            dst[ch] = o;
+                        }
                     }
                 }
             }
