@@ -113,6 +113,31 @@ titans_status_t titans_mem_step(titans_mem_t m, const void *k, const void *q, co
                                 const float *alpha, const float *eta, const float *theta,
                                 float *W1, float *W2, float *S1, float *S2, void *y, void *stream);
 
+/*
+ * Chunk-wise forward that allocates no device memory, for callers that cannot call
+ * cudaMalloc: code inside someone else's stream capture, under an allocator that owns all
+ * device memory, on a path that must not synchronize the device, or a plug-in that must
+ * not leave allocations behind (titans_mem_init allocates, so those callers cannot hold a
+ * handle). The pages on the method have no counterpart: this is a deployment variant.
+ *
+ * Same arguments and semantics as titans_mem_forward, with the configuration passed
+ * directly (cfg->flags is ignored); it always runs the CUDA-core (fp32 arithmetic) chunk
+ * kernel. Its scratch is a fixed 16 MiB device array inside the library, held by every GPU
+ * that loads the library until the process exits:
+ *  - the first call on a device looks up the array there; make it before any stream
+ *    capture meant to contain later calls;
+ *  - every call shares the array, so calls that overlap on a GPU race: serialize them;
+ *  - nothing in the array needs clearing between calls;
+ *  - a call needing more than the array holds -- B*H units x (4*chunk*h + chunk*d floats
+ *    for the MLP memory, chunk*d for the linear one, each rounded up to 64 floats) -- returns
+ *    TITANS_EUNSUPPORTED with a message in titans_last_error_string().
+ * No device status word: the kernel has no waits to time out.
+ */
+titans_status_t titans_mem_forward_noalloc(const titans_mem_config *cfg, const void *k, const void *q,
+                                           const void *v, const float *alpha, const float *eta,
+                                           const float *theta, long T, int chunk, float *W1, float *W2,
+                                           float *S1, float *S2, void *y, void *stream);
+
 /* Kernel that titans_mem_forward (step = 0) or titans_mem_step (step = 1) would run with
  * this chunk length; negative on an unsupported combination. */
 int titans_mem_path(titans_mem_t m, int chunk, int step);

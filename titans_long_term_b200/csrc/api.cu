@@ -133,6 +133,11 @@ titans_status_t cuda_fail(cudaError_t e, const char* what) {
 
 }  // namespace
 
+namespace titans {
+// Lets the library's other entry points report through titans_last_error_string().
+void set_last_error(const std::string& msg) { g_err = msg; }
+}  // namespace titans
+
 extern "C" {
 
 int titans_mem_version(void) { return 100; }

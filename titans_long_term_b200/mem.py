@@ -22,7 +22,8 @@ FLAG_CUDA_CORES = 1
 PATH_TC_MLP64, PATH_CUDA_CORES, PATH_STEP_CLUSTER = 1, 2, 3
 
 EXPORTED = ["titans_mem_init", "titans_mem_destroy", "titans_mem_forward", "titans_mem_step",
-            "titans_mem_path", "titans_mem_sync_status", "titans_last_error_string", "titans_mem_version"]
+            "titans_mem_path", "titans_mem_sync_status", "titans_last_error_string", "titans_mem_version",
+            "titans_mem_forward_noalloc"]
 
 
 class TitansError(RuntimeError):
@@ -52,10 +53,12 @@ def lib():
         L.titans_mem_forward.argtypes = [vp, vp, vp, vp, vp, vp, vp, l, i, vp, vp, vp, vp, vp, vp]
         L.titans_mem_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
         L.titans_mem_path.argtypes = [vp, i, i]
+        L.titans_mem_forward_noalloc.argtypes = [ctypes.POINTER(Config), vp, vp, vp, vp, vp, vp, l, i, vp, vp, vp,
+                                                 vp, vp, vp]
         L.titans_mem_sync_status.argtypes = [vp, vp]
         L.titans_last_error_string.restype = ctypes.c_char_p
         for f in ("titans_mem_init", "titans_mem_destroy", "titans_mem_forward", "titans_mem_step",
-                  "titans_mem_path", "titans_mem_sync_status", "titans_mem_version"):
+                  "titans_mem_path", "titans_mem_sync_status", "titans_mem_version", "titans_mem_forward_noalloc"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -149,3 +152,19 @@ def new_state(B: int, H: int, d: int, d_hidden: int, device="cuda") -> Dict[str,
         return {"W1": z, "S1": z.clone()}
     return {"W1": torch.zeros(B, H, d_hidden, d, device=device), "W2": torch.zeros(B, H, d, d_hidden, device=device),
             "S1": torch.zeros(B, H, d_hidden, d, device=device), "S2": torch.zeros(B, H, d, d_hidden, device=device)}
+
+
+def forward_noalloc(k, q, v, alpha, eta, theta, state: Dict[str, torch.Tensor], chunk: int, mode: str,
+                    y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """titans_mem_forward_noalloc: the CUDA-core chunk forward with the library's fixed scratch
+    array (no device allocation by the library). k, q, v [B, H, T, d]; gates [B, H, T]; state
+    updated in place; returns y. Calls that overlap on the GPU race on the shared scratch."""
+    B, H, T, d = k.shape
+    h = state["W1"].shape[-2] if "W2" in state else 0
+    if y is None:
+        y = torch.empty_like(k)
+    cfg = Config(d, h, chunk, BF16 if mode == "bf16" else FP32, B, H, 0)
+    _check(lib().titans_mem_forward_noalloc(ctypes.byref(cfg), _ptr(k), _ptr(q), _ptr(v), _ptr(alpha), _ptr(eta),
+                                            _ptr(theta), T, chunk, _ptr(state["W1"]), _ptr(state.get("W2")),
+                                            _ptr(state["S1"]), _ptr(state.get("S2")), _ptr(y), _stream(stream)))
+    return y
