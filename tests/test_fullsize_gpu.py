@@ -1,0 +1,147 @@
+"""Full-size parity of the five workloads against the oracle (GPU; slow).
+
+The 760M-class workload (MLP 64-256-64, B=8, H=16, T=4096, chunk 64) runs in exactly
+the launch configuration bench.py times and is compared on every unit. The long stream
+(T = 1,048,576) is compared on every unit for its first 65,536 tokens and on two sampled
+units for the whole stream (the oracle's chunk closed form, pinned to its token loop, is
+used where the token loop would take minutes). The wide memory (128-512-128) is compared
+on the whole prefill and on sampled decode units over 1024 steps that start from the
+oracle's own prefill state. fp32 reference mode is held to 1e-4 on the prefixes the
+library claims it for.
+"""
+import functools
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from parity import TOL, compare, gpu_inputs, run_gpu
+from titans_long_term_b200 import mem, synth
+
+pytestmark = [pytest.mark.gpu, pytest.mark.slow]
+
+
+def _oracle(inp, chunk, units=None, closed_form=True):
+    sel = slice(None) if units is None else list(units)
+    args = [inp[n][sel] for n in ("k", "q", "v", "alpha", "eta", "theta")]
+    st = {n: inp[n][sel] for n in inp if n[0] in "WS"}
+    f = oracle.forward_closed_form if closed_form else oracle.forward
+    return f(*args, st, chunk)
+
+
+@pytest.mark.parametrize("mode", ["bf16", "fp32"])
+def test_mlp_b2h4_t2k(mode):
+    w = synth.WORKLOADS["mlp-d64-b2h4-t2k"]
+    inp = synth.make_inputs(w, dtype=mode)
+    m = mem.Memory(w.d, w.h, w.chunk, mode, w.B, w.H)
+    gy, gst = run_gpu(m, inp, w.B, w.H, w.chunk)
+    ry, rst = _oracle(inp, w.chunk, closed_form=False)
+    compare(gy, gst, ry, rst, TOL[mode], what=f"b2h4 {mode}")
+
+
+@pytest.mark.parametrize("mode", ["bf16", "fp32"])
+def test_760m_class_layer(mode):
+    """B=8, H=16, T=4096, chunk 64: the benchmarked workload, every unit."""
+    w = synth.WORKLOADS["mlp-d64-b8h16-t4k"]
+    inp = synth.make_inputs(w, dtype=mode)
+    m = mem.Memory(w.d, w.h, w.chunk, mode, w.B, w.H)
+    if mode == "bf16":
+        assert m.path() == mem.PATH_TC_MLP64
+    gy, gst = run_gpu(m, inp, w.B, w.H, w.chunk)
+    ry, rst = _oracle(inp, w.chunk)
+    compare(gy, gst, ry, rst, TOL[mode], what=f"760M-class {mode}")
+
+
+@pytest.mark.parametrize("mode", ["bf16", "fp32"])
+def test_long_stream_prefix_every_unit(mode):
+    w = synth.WORKLOADS["mlp-d64-b1h16-t1m"]
+    inp = synth.make_inputs(w, T=65536, dtype=mode)
+    m = mem.Memory(w.d, w.h, w.chunk, mode, w.B, w.H)
+    gy, gst = run_gpu(m, inp, w.B, w.H, w.chunk)
+    ry, rst = _oracle(inp, w.chunk)
+    compare(gy, gst, ry, rst, TOL[mode], what=f"long stream 64K {mode}")
+
+
+# Final-state bar for the bf16 path over the full 1,048,576-token stream. The recurrence is
+# ill-conditioned over this horizon: the oracle itself moves its final W1 by 1.0e-2 when its
+# initial weights are perturbed once at bf16 scale (2^-9), and the bf16 path rounds its
+# operands in every one of the 16,384 chunks (measured gap 7.3e-2). The retrieval outputs y
+# keep the 2e-2 bar over the whole stream; the fp32 CUDA-core path keeps 1e-4 on everything.
+LONG_STREAM_BF16_STATE_TOL = 1e-1
+
+
+def test_long_stream_full_sampled_units():
+    """All 1,048,576 tokens on the GPU for the 16 units (tensor-core path); y at every token
+    (2e-2) and the final state (LONG_STREAM_BF16_STATE_TOL) of units 0 and 11 against the
+    oracle. The recall probes (every 4096th token repeats one key/value pair) are part of y."""
+    w = synth.WORKLOADS["mlp-d64-b1h16-t1m"]
+    inp = synth.make_inputs(w)
+    m = mem.Memory(w.d, w.h, w.chunk, "bf16", w.B, w.H)
+    gy, gst = run_gpu(m, inp, w.B, w.H, w.chunk)
+    units = [0, 11]
+    ry, rst = _oracle(inp, w.chunk, units=units)
+    compare(gy, {}, ry, {}, TOL["bf16"], units=units, what="long stream 1M y")
+    worst = compare(gy, gst, ry, rst, LONG_STREAM_BF16_STATE_TOL, units=units, what="long stream 1M state")
+    print("long stream 1M bf16 worst relative errors:", worst)
+    assert np.isfinite(gy).all()
+
+
+def test_long_stream_full_fp32_sampled_units():
+    """fp32 reference mode (CUDA-core kernel) over all 1,048,576 tokens: units 0 and 11, 1e-4."""
+    w = synth.WORKLOADS["mlp-d64-b1h16-t1m"]
+    inp = synth.make_inputs(w, dtype="fp32")
+    m = mem.Memory(w.d, w.h, w.chunk, "fp32", w.B, w.H)
+    gy, gst = run_gpu(m, inp, w.B, w.H, w.chunk)
+    units = [0, 11]
+    ry, rst = _oracle(inp, w.chunk, units=units)
+    worst = compare(gy, gst, ry, rst, TOL["fp32"], units=units, what="long stream 1M fp32")
+    print("long stream 1M fp32 worst relative errors:", worst)
+
+
+@functools.lru_cache(maxsize=2)
+def _wide_prefill(mode):
+    w = synth.WORKLOADS["mlp-d128-b4h8-t16k"]
+    inp = synth.make_inputs(w, dtype=mode)
+    ry, rst = _oracle(inp, w.chunk)
+    return w, inp, ry, rst
+
+
+@pytest.mark.parametrize("mode", ["bf16", "fp32"])
+def test_wide_memory_prefill(mode):
+    w, inp, ry, rst = _wide_prefill(mode)
+    m = mem.Memory(w.d, w.h, w.chunk, mode, w.B, w.H)
+    gy, gst = run_gpu(m, inp, w.B, w.H, w.chunk)
+    compare(gy, gst, ry, rst, TOL[mode], what=f"wide prefill {mode}")
+
+
+@pytest.mark.parametrize("mode,steps", [("bf16", 1024), ("fp32", 64)])
+def test_wide_memory_decode(mode, steps):
+    """256 x 8 decode units, each starting from the oracle's final prefill state of unit
+    (b // 64) * 8 + h; titans_mem_step for `steps` steps; 32 sampled units against the oracle
+    run with chunk = 1 over the same per-step inputs."""
+    w, inp, _, rst = _wide_prefill(mode)
+    src = synth.decode_state_rows(w)
+    n = w.decode_B * w.H
+    dev = "cuda"
+    state = {nm: torch.as_tensor(np.ascontiguousarray(x[src]), dtype=torch.float32).reshape(w.decode_B, w.H, *x.shape[1:]).to(dev)
+             for nm, x in rst.items()}
+    state0 = {nm: t.reshape(n, *t.shape[2:]).cpu().clone() for nm, t in state.items()}
+    m = mem.Memory(w.d, w.h, 1, mode, w.decode_B, w.H)
+    assert m.path(1, step=True) == mem.PATH_STEP_CLUSTER
+    sample = np.arange(3, n, n // 32)
+    ys, toks = [], []
+    for s in range(steps):
+        d = synth.decode_step_inputs(w, s, dtype=mode)
+        toks.append({k: v[sample] for k, v in d.items()})
+        g = {k: v.reshape(w.decode_B, w.H, *v.shape[1:]).to(dev) for k, v in d.items()}
+        y = m.step(g["k"], g["q"], g["v"], g["alpha"], g["eta"], g["theta"], state)
+        ys.append(y.reshape(n, -1)[torch.as_tensor(sample, device=dev)].float().cpu())
+    m.sync_status()
+    gy = torch.stack(ys, 1).numpy()
+    gst = {nm: t.reshape(n, *t.shape[2:])[torch.as_tensor(sample, device=dev)].cpu().numpy()
+           for nm, t in state.items()}
+    seq = {k: torch.stack([tk[k] for tk in toks], 1) for k in toks[0]}
+    ry, rs = oracle.forward(seq["k"], seq["q"], seq["v"], seq["alpha"], seq["eta"], seq["theta"],
+                            {nm: x[sample] for nm, x in state0.items()}, 1)
+    compare(gy, gst, ry, rs, TOL[mode], what=f"decode {mode} x{steps}")

@@ -44,6 +44,7 @@ result does not depend on which other units or ranges were asked for.
 from __future__ import annotations
 
 import dataclasses
+import functools
 from typing import Dict, Optional, Sequence
 
 import numpy as np
@@ -117,6 +118,7 @@ def _gate_ranges(w: Workload):
     return 0.002, 0.8, 0.99, 0.003
 
 
+@functools.lru_cache(maxsize=4096)
 def _projections(w: Workload, unit: int):
     g = _gen(w.seed, unit, 0x960)
     s = 1.0 / np.sqrt(w.d)
@@ -215,14 +217,28 @@ def make_inputs(w: Workload, units: Optional[Sequence[int]] = None, T: Optional[
 def decode_step_inputs(w: Workload, step: int, dtype: Optional[str] = None) -> Dict[str, torch.Tensor]:
     """Per-step decode inputs for decode_B x H units: k, q, v [decode_B*H, d]; gates [decode_B*H].
 
-    Decode unit u uses the projections of the prefill unit whose state it starts from."""
+    One generator per step draws x and the gates for every decode unit; decode unit u
+    projects its x with the projections of the prefill unit whose state it starts from."""
     dtype = w.dtype if dtype is None else dtype
+    n = w.decode_B * w.H
     src = decode_state_rows(w)
-    parts = [_draw(w, _gen(w.seed + 1000, step, u), 1, _projections(w, int(src[u])))
-             for u in range(w.decode_B * w.H)]
-    k, q, v, a, e, t = (torch.cat([p[i] for p in parts]) for i in range(6))
-    return {"k": _cast(k, dtype), "q": _cast(q, dtype), "v": _cast(v, dtype),
-            "alpha": a, "eta": e, "theta": t}
+    g = _gen(w.seed + 1000, step)
+    x = torch.randn(n, w.d, generator=g)
+    amax, elo, ehi, tmax = _gate_ranges(w)
+    a = torch.rand(n, generator=g) * amax
+    e = elo + torch.rand(n, generator=g) * (ehi - elo)
+    t = torch.rand(n, generator=g) * tmax
+    k = torch.empty(n, w.d)
+    q = torch.empty(n, w.d)
+    v = torch.empty(n, w.d)
+    for s_ in np.unique(src):
+        rows = torch.as_tensor(np.nonzero(src == s_)[0])
+        WK, WV, WQ = _projections(w, int(s_))
+        xs = x[rows]
+        k[rows] = _l2n(xs @ WK)
+        q[rows] = _l2n(xs @ WQ)
+        v[rows] = xs @ WV
+    return {"k": _cast(k, dtype), "q": _cast(q, dtype), "v": _cast(v, dtype), "alpha": a, "eta": e, "theta": t}
 
 
 def decode_state_rows(w: Workload) -> np.ndarray:
