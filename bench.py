@@ -192,13 +192,29 @@ def reference_arm(args, w, rank, world):
     print(json.dumps(line), flush=True)
 
 
+# ---------------------------------------------------------------- multi-rank helpers
+
+def rank_units(w, rank: int):
+    """Units of one rank: rank r runs units [r * B*H, (r + 1) * B*H) of a (world * B) x H batch, so
+    every rank processes its own data and per-GPU work stays fixed as ranks are added (weak scaling)."""
+    return list(range(rank * w.units, (rank + 1) * w.units))
+
+
+def max_over_ranks(value: float, device, world: int) -> float:
+    """Max of a per-rank duration over all ranks (the job is as slow as its slowest rank)."""
+    if world == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
 # ---------------------------------------------------------------- our arm
 
 def our_arm(args, w, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    # This rank's units: a contiguous block of a (world * B) x H batch, so every rank runs distinct data.
-    units = list(range(rank * w.units, (rank + 1) * w.units))
+    units = rank_units(w, rank)
     inp = synth.make_inputs(w, units=units)
     toks = {n: inp[n].reshape(w.B, w.H, w.T, w.d).to(dev) for n in ("k", "q", "v")}
     gates = {n: inp[n].reshape(w.B, w.H, w.T).to(dev) for n in ("alpha", "eta", "theta")}
@@ -241,12 +257,8 @@ def our_arm(args, w, rank, world, local_rank):
     if world > 1:
         torch.distributed.barrier()
     m.sync_status()
-    elapsed_ms = t0.elapsed_time(t1)
+    elapsed_ms = max_over_ranks(t0.elapsed_time(t1), dev, world)
     launch_ms = [a.elapsed_time(b) for a, b in evs]
-    if world > 1:
-        t = torch.tensor([elapsed_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
 
     # End-to-end through the public API from pinned host memory: H2D of the step's inputs,
     # the forward, D2H of the step's result y.
@@ -274,11 +286,7 @@ def our_arm(args, w, rank, world, local_rank):
         e2e_step()
     b.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = a.elapsed_time(b) / e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(a.elapsed_time(b) / e_steps, dev, world)
     m.sync_status()
     if rank == 0:
         clocks.stop()
@@ -329,6 +337,68 @@ def our_arm(args, w, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
+def decode_arm(args, w, rank, world, local_rank):
+    """One step = one titans_mem_step (single-token update + retrieve) for every decode unit
+    (decode_B x H), starting from seeded states; bound by HBM: each unit reads and writes its
+    four fp32 state matrices once per step."""
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    n = w.decode_B * w.H
+    src = synth.decode_state_rows(w)
+    st0 = synth.make_inputs(w, units=sorted(set(src.tolist())), T=1)
+    pos = {u: i for i, u in enumerate(sorted(set(src.tolist())))}
+    idx = torch.as_tensor([pos[int(u)] for u in src])
+    state = {nm: st0[nm][idx].reshape(w.decode_B, w.H, *st0[nm].shape[1:]).contiguous().to(dev)
+             for nm in st0 if nm[0] in "WS"}
+    K = max(args.steps, 1)
+    steps_in = [synth.decode_step_inputs(w, s) for s in range(min(K, 16))]
+    dev_in = [{k: v.reshape(w.decode_B, w.H, *v.shape[1:]).to(dev) for k, v in d.items()} for d in steps_in]
+    m = mem.Memory(w.d, w.h, 1, w.dtype, w.decode_B, w.H)
+    y = torch.empty_like(dev_in[0]["k"])
+
+    def step(i):
+        g = dev_in[i % len(dev_in)]
+        m.step(g["k"], g["q"], g["v"], g["alpha"], g["eta"], g["theta"], state, y=y)
+
+    for i in range(args.warmup):
+        step(i)
+    m.sync_status()
+    stream = torch.cuda.current_stream(dev)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    torch.cuda.synchronize(dev)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(K):
+        evs[i][0].record(stream)
+        step(i)
+        evs[i][1].record(stream)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    m.sync_status()
+    elapsed = max_over_ranks(t0.elapsed_time(t1), dev, world)
+    if rank != 0:
+        return
+    ms = elapsed / K
+    avg = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    peaks, which = load_peaks()
+    state_bytes = n * 2 * 4 * (2 * w.d * w.h) * 4 / 2  # read + write of W1, W2, S1, S2 (fp32)
+    io_bytes = n * (4 * w.d * (2 if w.dtype == "bf16" else 4) + 12)
+    gbs = (state_bytes + io_bytes) / (avg / 1e3) / 1e9
+    print(json.dumps({
+        "metric": "decode tokens/sec (single-token update+retrieve, every head) per B200",
+        "value": world * w.decode_B / (ms / 1e3), "unit": "tokens/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": w.dtype, "data": "synthetic (seeded)",
+        "config": {"workload": w.name + " decode", "decode_B": w.decode_B, "H": w.H, "units": n,
+                   "l2": "state larger than L2 (%.2f GB per step)" % (state_bytes / 1e9)},
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": gbs / peaks["hbm_gbs"], "traffic": None, "peak_source": f"hbm_gbs ({which})",
+                     "kernel": "step_mlp_cluster", "bytes_per_launch": state_bytes + io_bytes,
+                     "avg_launch_ms": avg},
+        "gpu_launches": K}), flush=True)
+
+
 def kernel_sha() -> str:
     import hashlib
     p = os.path.join(HERE, "titans_long_term_b200", "csrc", "chunk_tc_mlp64.cu")
@@ -343,6 +413,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="mlp-d64-b8h16-t4k", choices=list(synth.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--phase", choices=["forward", "decode"], default="forward",
+                    help="forward: the chunk-wise update + retrieve (default); decode: titans_mem_step")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -359,7 +431,10 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local_rank))
     try:
-        our_arm(args, w, rank, world, local_rank)
+        if args.phase == "decode":
+            decode_arm(args, w, rank, world, local_rank)
+        else:
+            our_arm(args, w, rank, world, local_rank)
     finally:
         if world > 1:
             torch.distributed.destroy_process_group()
