@@ -382,7 +382,7 @@ def decode_arm(args, w, rank, world, local_rank):
     ms = elapsed / K
     avg = statistics.mean(a.elapsed_time(b) for a, b in evs)
     peaks, which = load_peaks()
-    state_bytes = n * 2 * 4 * (2 * w.d * w.h) * 4 / 2  # read + write of W1, W2, S1, S2 (fp32)
+    state_bytes = n * 2 * (4 * w.d * w.h * 4)  # W1, W2, S1, S2 (fp32, d*h each): read once, written once
     io_bytes = n * (4 * w.d * (2 if w.dtype == "bf16" else 4) + 12)
     gbs = (state_bytes + io_bytes) / (avg / 1e3) / 1e9
     print(json.dumps({
@@ -415,6 +415,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--phase", choices=["forward", "decode"], default="forward",
                     help="forward: the chunk-wise update + retrieve (default); decode: titans_mem_step")
+    ap.add_argument("--decode-b", type=int, default=0, help="decode batch (default: the workload's, 256)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -422,6 +423,9 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     w = synth.WORKLOADS[args.workload]
+    if args.phase == "decode" and args.decode_b:
+        import dataclasses
+        w = dataclasses.replace(w, decode_B=args.decode_b)
     if args.impl == "reference":
         reference_arm(args, w, rank, world)
         return
