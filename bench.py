@@ -57,9 +57,9 @@ def stream_bytes_per_head_token(w) -> float:
 
 
 def state_bytes_per_unit(w) -> float:
-    """W and S read once and written once per call (fp32)."""
+    """W and S read once and written once per call (fp32): 4 x |W| x 4 B, |W| = |W1| + |W2|."""
     n = 2 * w.d * w.h if w.h else w.d * w.d
-    return 4 * 2 * n * 4
+    return 4 * n * 4
 
 
 # ---------------------------------------------------------------- clocks
