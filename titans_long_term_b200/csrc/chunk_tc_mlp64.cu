@@ -24,14 +24,15 @@
 //   - warps 0-3 own hidden rows 0..127 ("tile 0"), warps 4-7 rows 128..255 ("tile 1");
 //     the two tiles run their epilogues independently, so the tensor core works on one
 //     tile while the other tile's warps run theirs;
-//   - warps 8 and 9 issue the MMAs of tile 0 and tile 1 (one elected lane each: a single
-//     thread issues a tcgen05.mma only every ~80 cycles, two issuers double the rate);
-//     Y is split into the two tiles' partial sums over their hidden units, so the two
-//     issuers never need to be ordered; warp 8 also issues the TMA loads (K, Q, V two
-//     chunks ahead);
+//   - warps 8 and 9 issue tile 0's and tile 1's forward, backprop and W1-side MMAs (one
+//     elected lane each: a single thread issues a tcgen05.mma only every ~80-200 cycles,
+//     so more issuers shorten each MMA phase); Y is split into the two tiles' partial sums
+//     over their hidden units, so those issuers never need ordering; warp 8 also issues
+//     the TMA loads (K, Q, V two chunks ahead);
+//   - warp 11 issues both tiles' W2-side weight GEMMs (S2^T accumulation, dW2^T_c);
 //   - warp 10 prefetches the gates, runs the gate scan a chunk ahead and writes the scaled
-//     key tiles; warp 11 only completes the producer warpgroup, which hands registers to
-//     the epilogue warpgroups (setmaxnreg).
+//     key tiles. The producer warpgroup (warps 8-11) hands registers to the epilogue
+//     warpgroups (setmaxnreg).
 // Hand-offs go through mbarriers only; every wait is bounded.
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -79,7 +80,8 @@ enum Bar {
     B_S0, B_S1,          // tile t's momentum pre-pass done
     B_GW0, B_GW1,        // (GW2)^T and the S2^T accumulation of tile t done
     B_D0, B_D1,          // tile t wrote Delta^T rows
-    B_DW0, B_DW1,        // weighted weight GEMMs of tile t done
+    B_DW0, B_DW1,        // weighted W1 GEMMs of tile t done (dW1_c, S1 accumulation)
+    B_DX0, B_DX1,        // weighted W2 GEMMs of tile t done (S2^T accumulation, dW2^T_c)
     B_W0, B_W1,          // tile t rewrote its bf16 weight rows (and read dW_c)
     B_SC0, B_SC1,        // gate scan of a chunk with parity 0 / 1 published
     B_KC,                // scaled key tiles of the chunk written
@@ -319,8 +321,42 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
                 load_gates(c + 2);
             }
         }
-    } else if (warp > kEpiWarps + 1) {
-        // warp 11: nothing to do
+    } else if (warp == kEpiWarps + 3) {
+        // =========================== W2-side issuer: S2^T += A_K^T diag(-d) G, dW2^T_c = A_K^T diag(-c) G
+        const uint32_t idW = idesc_bf16_f32(128, 64, 0, 1);
+        const uint64_t dK = sdesc_sw128(sb, 16, 1024);
+        const uint64_t dMN8 = sdesc_sw128(sb, 8192, 1024);
+#define DSC(base, off) ((base) + (uint64_t)((off) >> 4))
+        for (int c = 0; c < nchunks; ++c) {
+            const uint32_t ph = (uint32_t)c & 1u;
+            bool ok = wait(B_G, ph);  // G and its scaled copies written
+            // S2^T accumulation of tile t once its S is pre-scaled.
+            for (int t = 0; t < 2 && ok; ++t) {
+                ok = wait(B_S0 + t, ph);
+                if (ok && lane == 0) {
+                    tc_fence_after();
+#pragma unroll 1
+                    for (int ks = 0; ks < 4; ++ks)
+                        umma_bf16(tmem + 256 + t * 128 + 64, DSC(dK, AT0 + t * 16384 + ks * 32),
+                                  DSC(dMN8, GD + ks * 2048), idW, 1);
+                }
+            }
+            // dW2^T_c of tile t into columns 128t+64 once the Delta epilogue has read (GW2)^T there.
+            for (int t = 0; t < 2 && ok; ++t) {
+                ok = wait(B_D0 + t, ph);
+                if (ok && lane == 0) {
+                    tc_fence_after();
+#pragma unroll 1
+                    for (int ks = 0; ks < 4; ++ks)
+                        umma_bf16(tmem + t * 128 + 64, DSC(dK, AT0 + t * 16384 + ks * 32),
+                                  DSC(dMN8, GC + ks * 2048), idW, ks > 0);
+                    umma_commit(&bars[B_DX0 + t]);
+                }
+            }
+            if (!ok) break;
+            __syncwarp();
+        }
+#undef DSC
     } else if (warp >= kEpiWarps) {
         // =========================== issuer warps: warp 8 + t issues tile t's MMAs (warp 8 also TMA)
         const int t = warp - kEpiWarps;
@@ -381,36 +417,28 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
             if (!ok) break;
             ok = wait(B_G, ph);  // G tiles written, both partial Y read
             if (!ok) break;
-            // (GW2)^T = W2^T G^T and S2^T += A_K^T diag(-d) G once tile t's S is pre-scaled.
-            ok = wait(B_S0 + t, ph);
-            if (ok && lane == 0) {
+            // (GW2)^T = W2^T G^T.
+            if (lane == 0) {
                 tc_fence_after();
 #pragma unroll 1
                 for (int ks = 0; ks < 4; ++ks)
                     umma_bf16(tmem + t * 128 + 64, DSC(dK, W2T + t * 16384 + ks * 32), DSC(dK, G + ks * 32), idG,
                               ks > 0);
-#pragma unroll 1
-                for (int ks = 0; ks < 4; ++ks)
-                    umma_bf16(tmem + 256 + t * 128 + 64, DSC(dK, AT0 + t * 16384 + ks * 32), DSC(dMN8, GD + ks * 2048),
-                              idW, 1);
                 umma_commit(&bars[B_GW0 + t]);
             }
-            if (!ok) break;
             // Scaled key tiles written: with the G tiles written before, every reader of this
             // chunk's K, Q, V buffer is done -> chunk c + 2.
             ok = wait(B_KC, ph);
             if (ok && t == 0 && lane == 0 && c + 2 < nchunks) issue_tma(c + 2);
-            // dW1_c -> cols 128t, S1 += Delta^T diag(-d) K, dW2^T_c -> cols 128t+64.
-            if (ok) ok = wait(B_D0 + t, ph);
+            // dW1_c -> cols 128t and S1 += Delta^T diag(-d) K once S is pre-scaled and Delta^T written.
+            if (ok) ok = wait(B_S0 + t, ph) && wait(B_D0 + t, ph);
             if (ok && lane == 0) {
                 tc_fence_after();
 #pragma unroll 1
                 for (int ks = 0; ks < 4; ++ks) {
                     const uint64_t dA = DSC(dK, AT1 + t * 16384 + ks * 32);
-                    const uint64_t aA = DSC(dK, AT0 + t * 16384 + ks * 32);
                     umma_bf16(tmem + t * 128, dA, DSC(dMN8, KC + ks * 2048), idW, ks > 0);
                     umma_bf16(tmem + 256 + t * 128, dA, DSC(dMN8, KD + ks * 2048), idW, 1);
-                    umma_bf16(tmem + t * 128 + 64, aA, DSC(dMN8, GC + ks * 2048), idW, ks > 0);
                 }
                 umma_commit(&bars[B_DW0 + t]);
             }
@@ -618,7 +646,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
             mbar_arrive(&bars[B_D0 + tile]);
 
             // (5) W <- (A W + sigma S) - sum_j c_j g_j; rewrite the bf16 operand rows
-            if (!wait(B_DW0 + tile, ph)) break;
+            if (!wait(B_DW0 + tile, ph) || !wait(B_DX0 + tile, ph)) break;
             tc_fence_after();
 #pragma unroll
             for (int blk = 0; blk < 4; ++blk) {
