@@ -411,7 +411,8 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="mlp-d64-b8h16-t4k", choices=list(synth.WORKLOADS))
+    ap.add_argument("--workload", default=None, choices=list(synth.WORKLOADS),
+                    help="default: mlp-d64-b8h16-t4k for --phase forward, mlp-d128-b4h8-t16k for decode")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--phase", choices=["forward", "decode"], default="forward",
                     help="forward: the chunk-wise update + retrieve (default); decode: titans_mem_step")
@@ -422,7 +423,11 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.workload is None:
+        args.workload = "mlp-d128-b4h8-t16k" if args.phase == "decode" else "mlp-d64-b8h16-t4k"
     w = synth.WORKLOADS[args.workload]
+    if args.phase == "decode" and not (w.decode_B or args.decode_b):
+        ap.error(f"workload {w.name} has no decode batch: pass --decode-b")
     if args.phase == "decode" and args.decode_b:
         import dataclasses
         w = dataclasses.replace(w, decode_B=args.decode_b)

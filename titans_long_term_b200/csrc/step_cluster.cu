@@ -6,7 +6,11 @@
 // thread-block cluster per unit splits the hidden width into 64-row slices (C = h / 64
 // CTAs): each CTA keeps its slice of W1 (64 x d) and W2 (d x 64) in registers, computes
 // its partial M(k) and M(q), and the partials are summed across the cluster through
-// distributed shared memory. Every state element crosses HBM exactly twice (read, write).
+// distributed shared memory. The momentum slices S1, S2 are not needed before the update,
+// so they stream into shared memory (cp.async) while the forward runs; that keeps the
+// registers under 128 per thread and two CTAs resident per SM, so one CTA's loads overlap
+// the other's arithmetic and cluster exchange. Every state element crosses HBM exactly
+// twice (read, write).
 #include <cooperative_groups.h>
 #include <cuda_bf16.h>
 
@@ -22,8 +26,23 @@ __device__ __forceinline__ float ld1(const __nv_bfloat16* p) { return __bfloat16
 constexpr int kStepThreads = 256;
 constexpr int kSlice = 64;  // hidden rows per CTA
 
+// Dynamic shared memory of one CTA: the S1 slice [64][D] and S2 slice [D][64] (fp32).
+template <int D>
+constexpr size_t step_smem_bytes() {
+    return (size_t)2 * kSlice * D * sizeof(float);
+}
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)),
+                 "l"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;" ::: "memory");
+}
+
 template <int D, typename Tin>
-__global__ void __launch_bounds__(kStepThreads) step_mlp_cluster(
+__global__ void __launch_bounds__(kStepThreads, 2) step_mlp_cluster(
     const Tin* __restrict__ k, const Tin* __restrict__ q, const Tin* __restrict__ v,
     const float* __restrict__ alpha, const float* __restrict__ eta, const float* __restrict__ theta,
     float* __restrict__ W1, float* __restrict__ W2, float* __restrict__ S1, float* __restrict__ S2,
@@ -37,6 +56,9 @@ __global__ void __launch_bounds__(kStepThreads) step_mlp_cluster(
     __shared__ float zk[kSlice], zq[kSlice], ak[kSlice], aq[kSlice], sp[kSlice], dl[kSlice];
     __shared__ float part[2][D];
     __shared__ float red[8][kSlice];
+    extern __shared__ float4 step_dyn[];
+    float* sS1 = reinterpret_cast<float*>(step_dyn);  // [kSlice][D]
+    float* sS2 = sS1 + kSlice * D;                    // [D][kSlice]
 
     cg::cluster_group cluster = cg::this_cluster();
     const int r = (int)cluster.block_rank();
@@ -49,24 +71,31 @@ __global__ void __launch_bounds__(kStepThreads) step_mlp_cluster(
     const float* W2u = W2 + u * D * H;
     const float* S2u = S2 + u * D * H;
 
-    // Issue every state load first; the arithmetic below waits on them.
-    float w1[R1][MC], s1[R1][MC], w2[R2][2], s2[R2][2];
+    // Issue every state load first: S1 and S2 slices into shared memory (16-byte pieces),
+    // W1 and W2 slices into registers; the arithmetic below waits on them.
+    {
+        const float* src1 = S1u + (size_t)j0 * D;  // contiguous [kSlice][D]
+#pragma unroll
+        for (int m = 0; m < kSlice * D / 4 / kStepThreads; ++m) {
+            const int id = tid + kStepThreads * m;
+            cp_async16(sS1 + 4 * id, src1 + 4 * id);
+        }
+#pragma unroll
+        for (int m = 0; m < D * kSlice / 4 / kStepThreads; ++m) {
+            const int id = tid + kStepThreads * m, row = id / (kSlice / 4), q4 = id % (kSlice / 4);
+            cp_async16(sS2 + row * kSlice + 4 * q4, S2u + (size_t)row * H + j0 + 4 * q4);
+        }
+    }
+    float w1[R1][MC], w2[R2][2];
 #pragma unroll
     for (int i = 0; i < R1; ++i)
 #pragma unroll
-        for (int c = 0; c < MC; ++c) {
-            const size_t o = (size_t)(j0 + warp * R1 + i) * D + lane + 32 * c;
-            w1[i][c] = __ldcs(W1u + o);
-            s1[i][c] = __ldcs(S1u + o);
-        }
+        for (int c = 0; c < MC; ++c)
+            w1[i][c] = __ldcs(W1u + (size_t)(j0 + warp * R1 + i) * D + lane + 32 * c);
 #pragma unroll
     for (int i = 0; i < R2; ++i)
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-            const size_t o = (size_t)(warp + 8 * i) * H + j0 + lane + 32 * c;
-            w2[i][c] = __ldcs(W2u + o);
-            s2[i][c] = __ldcs(S2u + o);
-        }
+        for (int c = 0; c < 2; ++c) w2[i][c] = __ldcs(W2u + (size_t)(warp + 8 * i) * H + j0 + lane + 32 * c);
     for (int i = tid; i < D; i += kStepThreads) {
         sk[i] = ld1(k + u * D + i);
         sq[i] = ld1(q + u * D + i);
@@ -152,6 +181,7 @@ __global__ void __launch_bounds__(kStepThreads) step_mlp_cluster(
         for (int w = 0; w < 8; ++w) b += red[w][tid];
         dl[tid] = b * sp[tid];
     }
+    cp_async_wait_all();
     __syncthreads();
     float* W1w = W1 + u * H * D;
     float* S1w = S1 + u * H * D;
@@ -163,7 +193,7 @@ __global__ void __launch_bounds__(kStepThreads) step_mlp_cluster(
         for (int c = 0; c < MC; ++c) {
             const int jl = warp * R1 + i, m = lane + 32 * c;
             const size_t o = (size_t)(j0 + jl) * D + m;
-            const float s = et * s1[i][c] - th * (dl[jl] * sk[m]);
+            const float s = et * sS1[jl * D + m] - th * (dl[jl] * sk[m]);
             __stcs(S1w + o, s);
             __stcs(W1w + o, (1.f - al) * w1[i][c] + s);
         }
@@ -173,7 +203,7 @@ __global__ void __launch_bounds__(kStepThreads) step_mlp_cluster(
         for (int c = 0; c < 2; ++c) {
             const int row = warp + 8 * i, jj = lane + 32 * c;
             const size_t o = (size_t)row * H + j0 + jj;
-            const float s = et * s2[i][c] - th * (sG[row] * ak[jj]);
+            const float s = et * sS2[row * kSlice + jj] - th * (sG[row] * ak[jj]);
             __stcs(S2w + o, s);
             __stcs(W2w + o, (1.f - al) * w2[i][c] + s);
         }
@@ -183,10 +213,17 @@ __global__ void __launch_bounds__(kStepThreads) step_mlp_cluster(
 template <int D, typename Tin>
 static cudaError_t launch_step(const ForwardArgs& a, cudaStream_t st) {
     constexpr int C = 4 * D / kSlice;
+    static bool attr_set = false;  // per process; the attribute is per function, not per device
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(step_mlp_cluster<D, Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)step_smem_bytes<D>());
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(a.units * C));
     cfg.blockDim = dim3(kStepThreads);
-    cfg.dynamicSmemBytes = 0;
+    cfg.dynamicSmemBytes = step_smem_bytes<D>();
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
