@@ -17,7 +17,9 @@
 // hidden row j of every state matrix:
 //   - W1[j, :] and W2[:, j] (fp32) live in that thread's registers,
 //   - S1[j, :] and S2[:, j] (fp32) live in TMEM and are the accumulators of the
-//     d-weighted GEMMs (pre-scaled by E before the GEMMs accumulate -sum d_j g_j),
+//     d-weighted GEMMs (scaled by E before the GEMMs accumulate -sum d_j g_j; the four
+//     producer warps do that pass, one TMEM lane quadrant each, while the epilogue warps
+//     run the SiLU),
 //   - the bf16 copies of W1 and W2^T that feed the MMAs are rewritten in shared memory
 //     once per chunk.
 // Warp roles (12 warps, one CTA per SM, persistent over the chunk loop of one unit):
@@ -85,6 +87,7 @@ enum Bar {
     B_W0, B_W1,          // tile t rewrote its bf16 weight rows (and read dW_c)
     B_SC0, B_SC1,        // gate scan of a chunk with parity 0 / 1 published
     B_KC,                // scaled key tiles of the chunk written
+    B_RS,                // the four producer warps scaled S <- E S for the chunk
     kNumBars
 };
 constexpr uint32_t TPTR = BAR + 8 * kNumBars;  // TMEM base address
@@ -223,6 +226,8 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
                 cnt = 256;
             else if (b == B_SC0 || b == B_SC1 || b == B_KC)
                 cnt = 32;
+            else if (b == B_RS)
+                cnt = 4;
             mbar_init(&bars[b], cnt);
         }
         fence_mbar_init();
@@ -251,6 +256,31 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
     if (warp >= kEpiWarps) {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsProducer));
     }
+    // Momentum decay of chunk c, S <- E S, run by each producer warp on the S columns of both
+    // tiles in its TMEM lane quadrant, after both tiles' pre-passes have read S (B_S); this
+    // chunk's S accumulation waits for all four (B_RS). Returns false on a timeout.
+    auto rescale_s = [&](int c) -> bool {
+        const int p = c & 1;
+        if (!wait(B_SC0 + p, (uint32_t)(c >> 1) & 1u)) return false;
+        if (!wait(B_S0, (uint32_t)c & 1u) || !wait(B_S1, (uint32_t)c & 1u)) return false;
+        tc_fence_after();
+        const float En = s_scal[4 * p + 1];
+        const uint32_t tq = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + 256;
+#pragma unroll 1
+        for (int col = 0; col < 256; col += 16) {
+            uint32_t r[16];
+            tmem_ld16(tq + col, r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(En * __uint_as_float(r[i]));
+            tmem_st16(tq + col, r);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[B_RS]);
+        return true;
+    };
     if (warp == kEpiWarps + 2) {
         // =========================== scan warp: gates, gate scans, scaled key tiles
         float ga[2], ge[2], gt[2];  // gates of one chunk, lane l holds tokens l and l + 32
@@ -316,6 +346,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
                 fence_proxy_async_smem();
                 mbar_arrive(&bars[B_KC]);
             }
+            if (!rescale_s(c)) break;
             if (c + 1 < nchunks) {
                 scan(c + 1);
                 load_gates(c + 2);
@@ -329,10 +360,11 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
 #define DSC(base, off) ((base) + (uint64_t)((off) >> 4))
         for (int c = 0; c < nchunks; ++c) {
             const uint32_t ph = (uint32_t)c & 1u;
-            bool ok = wait(B_G, ph);  // G and its scaled copies written
-            // S2^T accumulation of tile t once its S is pre-scaled.
+            bool ok = rescale_s(c);
+            ok = ok && wait(B_G, ph);  // G and its scaled copies written
+            // S2^T accumulation of tile t once S is scaled by E (B_RS).
+            ok = ok && wait(B_RS, ph);
             for (int t = 0; t < 2 && ok; ++t) {
-                ok = wait(B_S0 + t, ph);
                 if (ok && lane == 0) {
                     tc_fence_after();
 #pragma unroll 1
@@ -404,6 +436,8 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
                 umma_commit(&bars[B_Z0 + t]);
             }
             if (!ok || *abort_flag) break;
+            __syncwarp();
+            if (!rescale_s(c)) break;
             // Partial Y of tile t: its 128 hidden units are K-steps 8t .. 8t+7 of A W2^T.
             ok = wait(B_A0 + t, ph);
             if (ok && lane == 0) {
@@ -431,7 +465,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
             ok = wait(B_KC, ph);
             if (ok && t == 0 && lane == 0 && c + 2 < nchunks) issue_tma(c + 2);
             // dW1_c -> cols 128t and S1 += Delta^T diag(-d) K once S is pre-scaled and Delta^T written.
-            if (ok) ok = wait(B_S0 + t, ph) && wait(B_D0 + t, ph);
+            if (ok) ok = wait(B_RS, ph) && wait(B_D0 + t, ph);
             if (ok && lane == 0) {
                 tc_fence_after();
 #pragma unroll 1
@@ -508,10 +542,11 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
             const long t0 = (long)c * chunk;
             const int n = (int)min((long)chunk, T - t0);
 
-            // (1) momentum pre-pass: W <- A W + sigma S, S <- E S (the d-GEMMs then add -sum d_j g_j)
+            // (1) momentum pre-pass: W <- A W + sigma S (reads S only; the producer warps then
+            //     scale S <- E S, and the d-GEMMs add -sum d_j g_j)
             if (!wait(B_SC0 + p, (uint32_t)(c >> 1) & 1u)) break;
             {
-                const float An = s_scal[4 * p], En = s_scal[4 * p + 1], sig = s_scal[4 * p + 2];
+                const float An = s_scal[4 * p], sig = s_scal[4 * p + 2];
 #pragma unroll
                 for (int blk = 0; blk < 4; ++blk) {
                     uint32_t r1[16], r2[16];
@@ -520,16 +555,10 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
                     tmem_wait_ld();
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
-                        const float s1 = __uint_as_float(r1[i]), s2 = __uint_as_float(r2[i]);
-                        w1[16 * blk + i] = fmaf(An, w1[16 * blk + i], sig * s1);
-                        w2[16 * blk + i] = fmaf(An, w2[16 * blk + i], sig * s2);
-                        r1[i] = __float_as_uint(En * s1);
-                        r2[i] = __float_as_uint(En * s2);
+                        w1[16 * blk + i] = fmaf(An, w1[16 * blk + i], sig * __uint_as_float(r1[i]));
+                        w2[16 * blk + i] = fmaf(An, w2[16 * blk + i], sig * __uint_as_float(r2[i]));
                     }
-                    tmem_st16(t_s + 16 * blk, r1);
-                    tmem_st16(t_s + 64 + 16 * blk, r2);
                 }
-                tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(&bars[B_S0 + tile]);
             }
