@@ -436,8 +436,6 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
                 umma_commit(&bars[B_Z0 + t]);
             }
             if (!ok || *abort_flag) break;
-            __syncwarp();
-            if (!rescale_s(c)) break;
             // Partial Y of tile t: its 128 hidden units are K-steps 8t .. 8t+7 of A W2^T.
             ok = wait(B_A0 + t, ph);
             if (ok && lane == 0) {
@@ -449,6 +447,8 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
                 umma_commit(&bars[B_Y0 + t]);
             }
             if (!ok) break;
+            __syncwarp();
+            if (!rescale_s(c)) break;
             ok = wait(B_G, ph);  // G tiles written, both partial Y read
             if (!ok) break;
             // (GW2)^T = W2^T G^T.
@@ -542,28 +542,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
             const long t0 = (long)c * chunk;
             const int n = (int)min((long)chunk, T - t0);
 
-            // (1) momentum pre-pass: W <- A W + sigma S (reads S only; the producer warps then
-            //     scale S <- E S, and the d-GEMMs add -sum d_j g_j)
-            if (!wait(B_SC0 + p, (uint32_t)(c >> 1) & 1u)) break;
-            {
-                const float An = s_scal[4 * p], sig = s_scal[4 * p + 2];
-#pragma unroll
-                for (int blk = 0; blk < 4; ++blk) {
-                    uint32_t r1[16], r2[16];
-                    tmem_ld16(t_s + 16 * blk, r1);
-                    tmem_ld16(t_s + 64 + 16 * blk, r2);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        w1[16 * blk + i] = fmaf(An, w1[16 * blk + i], sig * __uint_as_float(r1[i]));
-                        w2[16 * blk + i] = fmaf(An, w2[16 * blk + i], sig * __uint_as_float(r2[i]));
-                    }
-                }
-                tc_fence_before();
-                mbar_arrive(&bars[B_S0 + tile]);
-            }
-
-            // (2) A = silu(Z): keys -> AT0 (and silu'(Z_K) into TMEM), queries -> AT1
+            // (1) A = silu(Z): keys -> AT0 (and silu'(Z_K) into TMEM), queries -> AT1
             if (!wait(B_Z0 + tile, ph)) break;
             tc_fence_after();
 #pragma unroll
@@ -599,10 +578,31 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
             tc_fence_before();
             mbar_arrive(&bars[B_A0 + tile]);
 
+            // (2) momentum pre-pass while the tensor core runs Y: W <- A W + sigma S (reads S only;
+            //     the producer warps then scale S <- E S, and the d-GEMMs add -sum d_j g_j)
+            if (!wait(B_SC0 + p, (uint32_t)(c >> 1) & 1u)) break;
+            {
+                const float An = s_scal[4 * p], sig = s_scal[4 * p + 2];
+#pragma unroll
+                for (int blk = 0; blk < 4; ++blk) {
+                    uint32_t r1[16], r2[16];
+                    tmem_ld16(t_s + 16 * blk, r1);
+                    tmem_ld16(t_s + 64 + 16 * blk, r2);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        w1[16 * blk + i] = fmaf(An, w1[16 * blk + i], sig * __uint_as_float(r1[i]));
+                        w2[16 * blk + i] = fmaf(An, w2[16 * blk + i], sig * __uint_as_float(r2[i]));
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive(&bars[B_S0 + tile]);
+            }
+
             // (3) G = 2 (M(k) - v) and its scaled copies (keys), y (queries). Token row = TMEM
             //     lane (quadrant quad), this warp's 32 of the 64 columns: [32 tile, 32 tile + 32).
-            if (!wait(B_Y0, ph) || !wait(B_Y1, ph)) break;
             if (!wait(B_TMA0 + (c & 1), (uint32_t)(c >> 1) & 1u)) break;  // the V tile, read below
+            if (!wait(B_Y0, ph) || !wait(B_Y1, ph)) break;
             tc_fence_after();
             {
                 const int row = quad * 32 + lane;
