@@ -88,6 +88,7 @@ enum Bar {
     B_SC0, B_SC1,        // gate scan of a chunk with parity 0 / 1 published
     B_KC,                // scaled key tiles of the chunk written
     B_RS,                // the four producer warps scaled S <- E S for the chunk
+    B_SA0, B_SA1,        // S1 and S2^T accumulations of tile t done (a commit from each issuer)
     kNumBars
 };
 constexpr uint32_t TPTR = BAR + 8 * kNumBars;  // TMEM base address
@@ -228,6 +229,8 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
                 cnt = 32;
             else if (b == B_RS)
                 cnt = 4;
+            else if (b == B_SA0 || b == B_SA1)
+                cnt = 2;
             mbar_init(&bars[b], cnt);
         }
         fence_mbar_init();
@@ -320,9 +323,9 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
             const int p = c & 1;
             const uint32_t KQb = (c & 1) ? KQ1 : KQ0;
             if (!wait(B_TMA0 + (c & 1), (uint32_t)(c >> 1) & 1u)) break;
-            // The previous chunk's weight GEMMs of both tiles (which read the scaled key tiles;
-            // every reader of the other scan buffer finished before them) have completed.
-            if (c > 0 && (!wait(B_DW0, (uint32_t)(c - 1) & 1u) || !wait(B_DW1, (uint32_t)(c - 1) & 1u))) break;
+            // The previous chunk's S1 accumulations of both tiles (the last readers of the scaled
+            // key tiles; every reader of the other scan buffer finished before them) have completed.
+            if (c > 0 && (!wait(B_SA0, (uint32_t)(c - 1) & 1u) || !wait(B_SA1, (uint32_t)(c - 1) & 1u))) break;
             {
                 const float* cc = s_cc + 64 * p;
                 const float* dd = s_dd + 64 * p;
@@ -362,17 +365,6 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
             const uint32_t ph = (uint32_t)c & 1u;
             bool ok = rescale_s(c);
             ok = ok && wait(B_G, ph);  // G and its scaled copies written
-            // S2^T accumulation of tile t once S is scaled by E (B_RS).
-            ok = ok && wait(B_RS, ph);
-            for (int t = 0; t < 2 && ok; ++t) {
-                if (ok && lane == 0) {
-                    tc_fence_after();
-#pragma unroll 1
-                    for (int ks = 0; ks < 4; ++ks)
-                        umma_bf16(tmem + 256 + t * 128 + 64, DSC(dK, AT0 + t * 16384 + ks * 32),
-                                  DSC(dMN8, GD + ks * 2048), idW, 1);
-                }
-            }
             // dW2^T_c of tile t into columns 128t+64 once the Delta epilogue has read (GW2)^T there.
             for (int t = 0; t < 2 && ok; ++t) {
                 ok = wait(B_D0 + t, ph);
@@ -383,6 +375,20 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
                         umma_bf16(tmem + t * 128 + 64, DSC(dK, AT0 + t * 16384 + ks * 32),
                                   DSC(dMN8, GC + ks * 2048), idW, ks > 0);
                     umma_commit(&bars[B_DX0 + t]);
+                }
+            }
+            // S2^T accumulation of tile t (S already scaled by E, B_RS): off the weight-update
+            // path, it runs while the epilogue rewrites the weights; the next chunk's SiLU
+            // (which overwrites A_K) waits for B_SA.
+            ok = ok && wait(B_RS, ph);
+            for (int t = 0; t < 2 && ok; ++t) {
+                if (lane == 0) {
+                    tc_fence_after();
+#pragma unroll 1
+                    for (int ks = 0; ks < 4; ++ks)
+                        umma_bf16(tmem + 256 + t * 128 + 64, DSC(dK, AT0 + t * 16384 + ks * 32),
+                                  DSC(dMN8, GD + ks * 2048), idW, 1);
+                    umma_commit(&bars[B_SA0 + t]);
                 }
             }
             if (!ok) break;
@@ -469,12 +475,16 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
             if (ok && lane == 0) {
                 tc_fence_after();
 #pragma unroll 1
-                for (int ks = 0; ks < 4; ++ks) {
-                    const uint64_t dA = DSC(dK, AT1 + t * 16384 + ks * 32);
-                    umma_bf16(tmem + t * 128, dA, DSC(dMN8, KC + ks * 2048), idW, ks > 0);
-                    umma_bf16(tmem + 256 + t * 128, dA, DSC(dMN8, KD + ks * 2048), idW, 1);
-                }
+                for (int ks = 0; ks < 4; ++ks)
+                    umma_bf16(tmem + t * 128, DSC(dK, AT1 + t * 16384 + ks * 32), DSC(dMN8, KC + ks * 2048), idW,
+                              ks > 0);
                 umma_commit(&bars[B_DW0 + t]);
+                // S1 accumulation after the weight GEMM: the weight update waits for dW1_c only.
+#pragma unroll 1
+                for (int ks = 0; ks < 4; ++ks)
+                    umma_bf16(tmem + 256 + t * 128, DSC(dK, AT1 + t * 16384 + ks * 32), DSC(dMN8, KD + ks * 2048),
+                              idW, 1);
+                umma_commit(&bars[B_SA0 + t]);
             }
             if (!ok) break;
             __syncwarp();
@@ -544,6 +554,8 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
 
             // (1) A = silu(Z): keys -> AT0 (and silu'(Z_K) into TMEM), queries -> AT1
             if (!wait(B_Z0 + tile, ph)) break;
+            // The previous chunk's S accumulations read this tile's A_K and Delta^T rows.
+            if (c > 0 && !wait(B_SA0 + tile, (uint32_t)(c - 1) & 1u)) break;
             tc_fence_after();
 #pragma unroll
             for (int blk = 0; blk < 4; ++blk) {  // keys and queries, 16-column blocks
@@ -696,7 +708,8 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
             mbar_arrive(&bars[B_W0 + tile]);
         }
 
-        // Final state of this hidden row (every MMA of the last chunk has completed).
+        // Final state of this hidden row, once the last chunk's S accumulations have completed.
+        if (nchunks > 0 && !*abort_flag) wait(B_SA0 + tile, (uint32_t)(nchunks - 1) & 1u);
         {
             float4* p = reinterpret_cast<float4*>(W1g + (u * kH + hrow) * kD);
 #pragma unroll
