@@ -618,19 +618,19 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
             tc_fence_after();
             {
                 const int row = quad * 32 + lane;
-                const uint32_t Vb = (c & 1) ? V1 : V0;
-                const bool key = row < kN, query = !key && row - kN < n;
-                const float cr = key ? -s_cc[64 * p + row] : 0.f, dr = key ? -s_dd[64 * p + row] : 0.f;
+                if (row < kN) {  // key row: G and its c- and d-scaled copies (bf16 tiles)
+                    const uint32_t Vb = (c & 1) ? V1 : V0;
+                    const float cr = -s_cc[64 * p + row], dr = -s_dd[64 * p + row];
 #pragma unroll 1
-                for (int hb = 0; hb < 2; ++hb) {
-                    const int col0 = 32 * tile + 16 * hb;
-                    uint32_t r[16], r2[16];
-                    tmem_ld16(tmem + lane_off + 64 + col0, r);         // tile 0's partial Y
-                    tmem_ld16(tmem + lane_off + 128 + 64 + col0, r2);  // tile 1's partial Y
-                    tmem_wait_ld();
+                    for (int hb = 0; hb < 2; ++hb) {
+                        const int col0 = 32 * tile + 16 * hb;
+                        uint32_t r[16], r2[16];
+                        tmem_ld16(tmem + lane_off + 64 + col0, r);         // tile 0's partial Y
+                        tmem_ld16(tmem + lane_off + 128 + 64 + col0, r2);  // tile 1's partial Y
+                        tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) + __uint_as_float(r2[i]));
-                    if (key) {
+                        for (int i = 0; i < 16; ++i)
+                            r[i] = __float_as_uint(__uint_as_float(r[i]) + __uint_as_float(r2[i]));
 #pragma unroll
                         for (int ch = 0; ch < 2; ++ch) {
                             const uint32_t off = sw128_off((uint32_t)row, (uint32_t)(col0 + 8 * ch));
@@ -650,23 +650,33 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
                             st_shared_v4(sb + GC + off, oc[0], oc[1], oc[2], oc[3]);
                             st_shared_v4(sb + GD + off, od[0], od[1], od[2], od[3]);
                         }
-                    } else if (query) {
-                        uint4* dst = reinterpret_cast<uint4*>(yg + ((u * T + t0 + (row - kN)) * kD + col0));
+                    }
+                    fence_proxy_async_smem();
+                    tc_fence_before();
+                    mbar_arrive(&bars[B_G]);
+                } else {  // query row: y, stored after the arrival (the TMEM reads are what GW waits for)
+                    uint32_t o[16];
 #pragma unroll
-                        for (int ch = 0; ch < 2; ++ch) {
-                            uint4 o;
-                            o.x = pack_bf16x2(__uint_as_float(r[8 * ch]), __uint_as_float(r[8 * ch + 1]));
-                            o.y = pack_bf16x2(__uint_as_float(r[8 * ch + 2]), __uint_as_float(r[8 * ch + 3]));
-                            o.z = pack_bf16x2(__uint_as_float(r[8 * ch + 4]), __uint_as_float(r[8 * ch + 5]));
-                            o.w = pack_bf16x2(__uint_as_float(r[8 * ch + 6]), __uint_as_float(r[8 * ch + 7]));
-                            dst[ch] = o;
-                        }
+                    for (int hb = 0; hb < 2; ++hb) {
+                        const int col0 = 32 * tile + 16 * hb;
+                        uint32_t r[16], r2[16];
+                        tmem_ld16(tmem + lane_off + 64 + col0, r);
+                        tmem_ld16(tmem + lane_off + 128 + 64 + col0, r2);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            o[8 * hb + i] = pack_bf16x2(__uint_as_float(r[2 * i]) + __uint_as_float(r2[2 * i]),
+                                                        __uint_as_float(r[2 * i + 1]) + __uint_as_float(r2[2 * i + 1]));
+                    }
+                    tc_fence_before();
+                    mbar_arrive(&bars[B_G]);
+                    if (row - kN < n) {
+                        uint4* dst = reinterpret_cast<uint4*>(yg + ((u * T + t0 + (row - kN)) * kD + 32 * tile));
+#pragma unroll
+                        for (int q4 = 0; q4 < 4; ++q4) dst[q4] = make_uint4(o[4 * q4], o[4 * q4 + 1], o[4 * q4 + 2], o[4 * q4 + 3]);
                     }
                 }
             }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            mbar_arrive(&bars[B_G]);
 
             // (4) Delta^T = (GW2)^T * silu'(Z_K)^T -> AT1 rows (the queries' tile was consumed by Y)
             if (!wait(B_GW0 + tile, ph)) break;
