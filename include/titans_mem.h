@@ -103,6 +103,41 @@ titans_status_t titans_mem_forward(titans_mem_t m, const void *k, const void *q,
                                    long T, int chunk, float *W1, float *W2, float *S1, float *S2,
                                    void *y, void *stream);
 
+/* Device buffers that titans_mem_forward_host stages through, each the size of the host
+ * array of the same name ([B, H, T, d] for k, q, v, y; [B, H, T] for the gates). The call
+ * overwrites them; their contents afterwards are unspecified (segment-major layout). */
+typedef struct {
+    void *k, *q, *v;
+    float *alpha, *eta, *theta;
+    void *y;
+} titans_device_buffers;
+
+/*
+ * titans_mem_forward with the token streams and y in HOST memory and the state on the
+ * device: T is cut into segments of t_seg tokens (a multiple of `chunk`; 0 picks about
+ * eight segments), and each segment's host-to-device copy, forward and device-to-host copy
+ * of y run on three streams, so the copies of one segment overlap the compute and copies of
+ * the others. Running a stream in segments gives exactly the result of one call over T (a
+ * segment boundary is a chunk boundary).
+ *   k, q, v, alpha, eta, theta, y: host arrays with titans_mem_forward's shapes and dtypes;
+ *     page-locked memory (cudaHostAlloc / cudaHostRegister) lets the copies overlap, pageable
+ *     memory is correct but serialises them. They must stay valid until `stream` completes.
+ *   W1, W2, S1, S2: device state as in titans_mem_forward.
+ *   dev: device scratch (see titans_device_buffers), 16-byte aligned like the device
+ *     arguments of titans_mem_forward.
+ * Asynchronous on `stream`: the copies start after the work already queued on it, and work
+ * queued on it afterwards starts after the last copy of y. The handle's two copy streams are
+ * created on first use; calls on one handle must not overlap.
+ * Returns TITANS_EINVAL for a null pointer, a misaligned device buffer or a t_seg that is
+ * not a multiple of chunk, TITANS_ECUDA if a copy or launch fails (earlier segments may
+ * then be queued already), and otherwise what titans_mem_forward returns per segment.
+ */
+titans_status_t titans_mem_forward_host(titans_mem_t m, const void *k, const void *q, const void *v,
+                                        const float *alpha, const float *eta, const float *theta,
+                                        long T, int chunk, float *W1, float *W2, float *S1, float *S2,
+                                        void *y, const titans_device_buffers *dev, long t_seg,
+                                        void *stream);
+
 /*
  * One decode step per unit with chunk = 1 semantics: y = M(q; W_{t-1}), then the
  * update with the gradient at W_{t-1}.

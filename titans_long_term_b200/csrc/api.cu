@@ -5,7 +5,9 @@
 
 #include <cstdint>
 #include <cstdio>
+#include <algorithm>
 #include <string>
+#include <vector>
 
 #include "../../include/titans_mem.h"
 #include "kernels.h"
@@ -16,6 +18,9 @@ struct titans_mem {
     unsigned* status;   // device status word
     float* ws;          // CUDA-core path workspace
     size_t ws_per_unit; // floats
+    // titans_mem_forward_host: copy streams and events, created on first use.
+    cudaStream_t s_in = nullptr, s_out = nullptr;
+    std::vector<cudaEvent_t> ev;  // [0] start, [1] done, then (copied in, computed) per segment
 };
 
 namespace {
@@ -176,6 +181,9 @@ titans_status_t titans_mem_init(const titans_mem_config* cfg, titans_mem_t* out)
 
 titans_status_t titans_mem_destroy(titans_mem_t m) {
     if (!m) return fail(TITANS_EINVAL, "handle is NULL");
+    for (cudaEvent_t e : m->ev) cudaEventDestroy(e);
+    if (m->s_in) cudaStreamDestroy(m->s_in);
+    if (m->s_out) cudaStreamDestroy(m->s_out);
     cudaFree(m->ws);
     cudaFree(m->status);
     delete m;
@@ -213,6 +221,83 @@ titans_status_t titans_mem_forward(titans_mem_t m, const void* k, const void* q,
         e = titans::launch_chunk_cuda_cores(a, st);
     }
     if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
+    return TITANS_OK;
+}
+
+titans_status_t titans_mem_forward_host(titans_mem_t m, const void* k, const void* q, const void* v,
+                                        const float* alpha, const float* eta, const float* theta, long T, int chunk,
+                                        float* W1, float* W2, float* S1, float* S2, void* y,
+                                        const titans_device_buffers* dev, long t_seg, void* stream) {
+    if (!m) return fail(TITANS_EINVAL, "handle is NULL");
+    if (!dev) return fail(TITANS_EINVAL, "dev is NULL");
+    const void* host[] = {k, q, v, alpha, eta, theta, y};
+    const char* names[] = {"k", "q", "v", "alpha", "eta", "theta", "y"};
+    for (int i = 0; i < 7; ++i)
+        if (!host[i]) return fail(TITANS_EINVAL, std::string(names[i]) + " is NULL");
+    titans_status_t s = check_ptrs(m, dev->k, dev->q, dev->v, dev->alpha, dev->eta, dev->theta, W1, W2, S1, S2,
+                                   dev->y);
+    if (s != TITANS_OK) return s;
+    if (T < 1) return fail(TITANS_EINVAL, "T must be >= 1");
+    if (chunk < 1 || chunk > m->cfg.chunk)
+        return fail(TITANS_EUNSUPPORTED, "chunk must be in 1..config.chunk");
+    if (t_seg < 0 || t_seg % chunk != 0) return fail(TITANS_EINVAL, "t_seg must be a non-negative multiple of chunk");
+    if (t_seg == 0) t_seg = ((T + 7) / 8 + chunk - 1) / chunk * chunk;
+    const long nseg = (T + t_seg - 1) / t_seg;
+    if (nseg > 4096) return fail(TITANS_EINVAL, "more than 4096 segments: raise t_seg");
+    int cur = -1;
+    cudaError_t e = cudaGetDevice(&cur);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (cur != m->device) return fail(TITANS_EINVAL, "the current device is not the handle's device");
+    if (!m->s_in) {
+        e = cudaStreamCreateWithFlags(&m->s_in, cudaStreamNonBlocking);
+        if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&m->s_out, cudaStreamNonBlocking);
+        if (e != cudaSuccess) return cuda_fail(e, "creating the copy streams");
+    }
+    while ((long)m->ev.size() < 2 + 2 * nseg) {
+        cudaEvent_t ev;
+        e = cudaEventCreateWithFlags(&ev, cudaEventDisableTiming);
+        if (e != cudaSuccess) return cuda_fail(e, "creating events");
+        m->ev.push_back(ev);
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const size_t es = m->cfg.mode == TITANS_BF16 ? 2 : 4;  // token element size
+    const size_t units = (size_t)m->cfg.B * m->cfg.H, d = (size_t)m->cfg.d;
+    const size_t row_h = (size_t)T * d * es;  // one unit's host stream of k, q, v or y
+    // Copies and forward of segment i: tokens [t0, t0 + tn) of every unit, packed on the
+    // device as [units][tn][...] at the offset of the segments before it.
+    e = cudaEventRecord(m->ev[0], st);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(m->s_in, m->ev[0], 0);
+    if (e != cudaSuccess) return cuda_fail(e, "ordering after the caller's stream");
+    for (long i = 0; i < nseg; ++i) {
+        const long t0 = i * t_seg, tn = std::min(t_seg, T - t0);
+        const size_t tok_off = units * (size_t)t0 * d * es, gate_off = units * (size_t)t0;
+        char* dk[3] = {static_cast<char*>(dev->k) + tok_off, static_cast<char*>(dev->q) + tok_off,
+                       static_cast<char*>(dev->v) + tok_off};
+        const char* hk[3] = {static_cast<const char*>(k), static_cast<const char*>(q), static_cast<const char*>(v)};
+        for (int j = 0; j < 3 && e == cudaSuccess; ++j)
+            e = cudaMemcpy2DAsync(dk[j], (size_t)tn * d * es, hk[j] + (size_t)t0 * d * es, row_h, (size_t)tn * d * es,
+                                  units, cudaMemcpyHostToDevice, m->s_in);
+        float* dg[3] = {dev->alpha + gate_off, dev->eta + gate_off, dev->theta + gate_off};
+        const float* hg[3] = {alpha, eta, theta};
+        for (int j = 0; j < 3 && e == cudaSuccess; ++j)
+            e = cudaMemcpy2DAsync(dg[j], (size_t)tn * 4, hg[j] + t0, (size_t)T * 4, (size_t)tn * 4, units,
+                                  cudaMemcpyHostToDevice, m->s_in);
+        if (e == cudaSuccess) e = cudaEventRecord(m->ev[2 + 2 * i], m->s_in);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(st, m->ev[2 + 2 * i], 0);
+        if (e != cudaSuccess) return cuda_fail(e, "copying a segment in");
+        char* dy = static_cast<char*>(dev->y) + tok_off;
+        s = titans_mem_forward(m, dk[0], dk[1], dk[2], dg[0], dg[1], dg[2], tn, chunk, W1, W2, S1, S2, dy, stream);
+        if (s != TITANS_OK) return s;
+        e = cudaEventRecord(m->ev[3 + 2 * i], st);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(m->s_out, m->ev[3 + 2 * i], 0);
+        if (e == cudaSuccess)
+            e = cudaMemcpy2DAsync(static_cast<char*>(y) + (size_t)t0 * d * es, row_h, dy, (size_t)tn * d * es,
+                                  (size_t)tn * d * es, units, cudaMemcpyDeviceToHost, m->s_out);
+        if (e != cudaSuccess) return cuda_fail(e, "copying a segment out");
+    }
+    e = cudaEventRecord(m->ev[1], m->s_out);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(st, m->ev[1], 0);
+    if (e != cudaSuccess) return cuda_fail(e, "ordering the caller's stream after the copies");
     return TITANS_OK;
 }
 

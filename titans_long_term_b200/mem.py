@@ -23,7 +23,7 @@ PATH_TC_MLP64, PATH_CUDA_CORES, PATH_STEP_CLUSTER = 1, 2, 3
 
 EXPORTED = ["titans_mem_init", "titans_mem_destroy", "titans_mem_forward", "titans_mem_step",
             "titans_mem_path", "titans_mem_sync_status", "titans_last_error_string", "titans_mem_version",
-            "titans_mem_forward_noalloc"]
+            "titans_mem_forward_noalloc", "titans_mem_forward_host"]
 
 
 class TitansError(RuntimeError):
@@ -35,6 +35,11 @@ class TitansError(RuntimeError):
 class Config(ctypes.Structure):
     _fields_ = [("d", ctypes.c_int), ("d_hidden", ctypes.c_int), ("chunk", ctypes.c_int),
                 ("mode", ctypes.c_int), ("B", ctypes.c_int), ("H", ctypes.c_int), ("flags", ctypes.c_uint)]
+
+
+class DeviceBuffers(ctypes.Structure):
+    _fields_ = [("k", ctypes.c_void_p), ("q", ctypes.c_void_p), ("v", ctypes.c_void_p), ("alpha", ctypes.c_void_p),
+                ("eta", ctypes.c_void_p), ("theta", ctypes.c_void_p), ("y", ctypes.c_void_p)]
 
 
 _lib = None
@@ -55,10 +60,13 @@ def lib():
         L.titans_mem_path.argtypes = [vp, i, i]
         L.titans_mem_forward_noalloc.argtypes = [ctypes.POINTER(Config), vp, vp, vp, vp, vp, vp, l, i, vp, vp, vp,
                                                  vp, vp, vp]
+        L.titans_mem_forward_host.argtypes = [vp, vp, vp, vp, vp, vp, vp, l, i, vp, vp, vp, vp, vp,
+                                              ctypes.POINTER(DeviceBuffers), l, vp]
         L.titans_mem_sync_status.argtypes = [vp, vp]
         L.titans_last_error_string.restype = ctypes.c_char_p
         for f in ("titans_mem_init", "titans_mem_destroy", "titans_mem_forward", "titans_mem_step",
-                  "titans_mem_path", "titans_mem_sync_status", "titans_mem_version", "titans_mem_forward_noalloc"):
+                  "titans_mem_path", "titans_mem_sync_status", "titans_mem_version", "titans_mem_forward_noalloc",
+                  "titans_mem_forward_host"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -128,6 +136,30 @@ class Memory:
         _check(lib().titans_mem_forward(self._h, _ptr(k), _ptr(q), _ptr(v), _ptr(alpha), _ptr(eta), _ptr(theta),
                                         T, chunk or self.chunk, _ptr(state["W1"]), _ptr(state.get("W2")),
                                         _ptr(state["S1"]), _ptr(state.get("S2")), _ptr(y), _stream(stream)))
+        return y
+
+    def forward_host(self, k, q, v, alpha, eta, theta, state: Dict[str, torch.Tensor], y: torch.Tensor,
+                     staging: Dict[str, torch.Tensor], chunk: Optional[int] = None, t_seg: int = 0,
+                     stream=None) -> torch.Tensor:
+        """titans_mem_forward_host: k, q, v [B, H, T, d] and gates [B, H, T] in host memory (pinned
+        for overlap), y [B, H, T, d] host output, state on the device (updated in place);
+        `staging` holds device tensors k, q, v, alpha, eta, theta, y of the same shapes (scratch).
+        Asynchronous on the stream: synchronize before reading y."""
+        T = k.shape[-2]
+        lead = (self.B, self.H, T)
+        for n, t in (("k", k), ("q", q), ("v", v), ("y", y)):
+            if t.is_cuda or t.dtype != self.dtype or not t.is_contiguous() or tuple(t.shape) != lead + (self.d,):
+                raise ValueError(f"{n}: expected contiguous host {self.dtype} of shape {lead + (self.d,)}")
+        for n, t in (("alpha", alpha), ("eta", eta), ("theta", theta)):
+            if t.is_cuda or t.dtype != torch.float32 or not t.is_contiguous() or tuple(t.shape) != lead:
+                raise ValueError(f"{n}: expected contiguous host float32 of shape {lead}")
+        self._check_tensors({n: staging[n] for n in ("k", "q", "v")},
+                            {n: staging[n] for n in ("alpha", "eta", "theta")}, state, staging["y"], lead)
+        dev = DeviceBuffers(*(staging[n].data_ptr() for n in ("k", "q", "v", "alpha", "eta", "theta", "y")))
+        _check(lib().titans_mem_forward_host(self._h, _ptr(k), _ptr(q), _ptr(v), _ptr(alpha), _ptr(eta),
+                                             _ptr(theta), T, chunk or self.chunk, _ptr(state["W1"]),
+                                             _ptr(state.get("W2")), _ptr(state["S1"]), _ptr(state.get("S2")),
+                                             _ptr(y), ctypes.byref(dev), t_seg, _stream(stream)))
         return y
 
     def step(self, k, q, v, alpha, eta, theta, state: Dict[str, torch.Tensor], y: Optional[torch.Tensor] = None,
