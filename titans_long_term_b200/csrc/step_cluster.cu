@@ -165,6 +165,9 @@ __global__ void __launch_bounds__(kStepThreads, 2) step_mlp_cluster(
                 y[u * D + i] = yq;
         }
     }
+    // This CTA is done reading the other slices' partials: arrive now, wait only before
+    // exiting, so no CTA holds its SM until the slowest one of the cluster has stored.
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
     __syncthreads();
     // Backprop through W2 for this slice's hidden units: per-lane partial over its rows.
 #pragma unroll
@@ -207,7 +210,7 @@ __global__ void __launch_bounds__(kStepThreads, 2) step_mlp_cluster(
             __stcs(S2w + o, s);
             __stcs(W2w + o, (1.f - al) * w2[i][c] + s);
         }
-    cluster.sync();  // no CTA leaves while another may still read its partials
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");  // no CTA leaves while another may still read its partials
 }
 
 template <int D, typename Tin>
