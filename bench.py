@@ -327,7 +327,7 @@ def our_arm(args, w, rank, world, local_rank):
                      "hbm_gbs_at_algorithmic_bytes": algo_bytes / (avg_launch / 1e3) / 1e9},
         "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
-                "api": "titans_mem_forward_host (pinned host buffers, ~8 overlapped segments)"},
+                "api": "titans_mem_forward_host (pinned host buffers, ~16 overlapped segments)"},
         "gpu_launches": args.steps,
         "clocks": clocks.summary(),
     }

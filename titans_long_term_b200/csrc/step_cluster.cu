@@ -23,7 +23,8 @@ namespace titans {
 __device__ __forceinline__ float ld1(const float* p) { return __ldg(p); }
 __device__ __forceinline__ float ld1(const __nv_bfloat16* p) { return __bfloat162float(*p); }
 
-constexpr int kStepThreads = 256;
+constexpr int kStepWarps = 8;
+constexpr int kStepThreads = 32 * kStepWarps;
 constexpr int kSlice = 64;  // hidden rows per CTA
 
 // Dynamic shared memory of one CTA: the S1 slice [64][D] and S2 slice [D][64] (fp32).
@@ -50,12 +51,12 @@ __global__ void __launch_bounds__(kStepThreads, 2) step_mlp_cluster(
     constexpr int H = 4 * D;
     constexpr int C = H / kSlice;        // CTAs per unit (cluster size)
     constexpr int MC = D / 32;           // W1 columns per lane
-    constexpr int R1 = kSlice / 8;       // W1 rows per warp
-    constexpr int R2 = D / 8;            // W2 rows per warp
+    constexpr int R1 = kSlice / kStepWarps;  // W1 rows per warp
+    constexpr int R2 = D / kStepWarps;       // W2 rows per warp
     __shared__ float sk[D], sq[D], sv[D], sG[D];
     __shared__ float zk[kSlice], zq[kSlice], ak[kSlice], aq[kSlice], sp[kSlice], dl[kSlice];
     __shared__ float part[2][D];
-    __shared__ float red[8][kSlice];
+    __shared__ float red[kStepWarps][kSlice];
     extern __shared__ float4 step_dyn[];
     float* sS1 = reinterpret_cast<float*>(step_dyn);  // [kSlice][D]
     float* sS2 = sS1 + kSlice * D;                    // [D][kSlice]
@@ -95,7 +96,7 @@ __global__ void __launch_bounds__(kStepThreads, 2) step_mlp_cluster(
 #pragma unroll
     for (int i = 0; i < R2; ++i)
 #pragma unroll
-        for (int c = 0; c < 2; ++c) w2[i][c] = __ldcs(W2u + (size_t)(warp + 8 * i) * H + j0 + lane + 32 * c);
+        for (int c = 0; c < 2; ++c) w2[i][c] = __ldcs(W2u + (size_t)(warp + kStepWarps * i) * H + j0 + lane + 32 * c);
     for (int i = tid; i < D; i += kStepThreads) {
         sk[i] = ld1(k + u * D + i);
         sq[i] = ld1(q + u * D + i);
@@ -143,8 +144,8 @@ __global__ void __launch_bounds__(kStepThreads, 2) step_mlp_cluster(
             b += __shfl_xor_sync(0xffffffffu, b, o);
         }
         if (lane == 0) {
-            part[0][warp + 8 * i] = a;
-            part[1][warp + 8 * i] = b;
+            part[0][warp + kStepWarps * i] = a;
+            part[1][warp + kStepWarps * i] = b;
         }
     }
     cluster.sync();
@@ -174,14 +175,14 @@ __global__ void __launch_bounds__(kStepThreads, 2) step_mlp_cluster(
     for (int c = 0; c < 2; ++c) {
         float acc = 0.f;
 #pragma unroll
-        for (int i = 0; i < R2; ++i) acc += w2[i][c] * sG[warp + 8 * i];
+        for (int i = 0; i < R2; ++i) acc += w2[i][c] * sG[warp + kStepWarps * i];
         red[warp][lane + 32 * c] = acc;
     }
     __syncthreads();
     if (tid < kSlice) {
         float b = 0.f;
 #pragma unroll
-        for (int w = 0; w < 8; ++w) b += red[w][tid];
+        for (int w = 0; w < kStepWarps; ++w) b += red[w][tid];
         dl[tid] = b * sp[tid];
     }
     cp_async_wait_all();
@@ -204,7 +205,7 @@ __global__ void __launch_bounds__(kStepThreads, 2) step_mlp_cluster(
     for (int i = 0; i < R2; ++i)
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
-            const int row = warp + 8 * i, jj = lane + 32 * c;
+            const int row = warp + kStepWarps * i, jj = lane + 32 * c;
             const size_t o = (size_t)row * H + j0 + jj;
             const float s = et * sS2[row * kSlice + jj] - th * (sG[row] * ak[jj]);
             __stcs(S2w + o, s);
