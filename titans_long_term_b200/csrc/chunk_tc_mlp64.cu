@@ -37,6 +37,7 @@
 //     warpgroups (setmaxnreg).
 // Hand-offs go through mbarriers only; every wait is bounded.
 #include <cuda_bf16.h>
+#include <atomic>
 #include <cstdint>
 
 #include "kernels.h"
@@ -756,12 +757,17 @@ size_t chunk_tc_mlp64_smem_bytes() { return tc::kSmemBytes; }
 
 cudaError_t launch_chunk_tc_mlp64(const ForwardArgs& a, const CUtensorMap& tk, const CUtensorMap& tq,
                                   const CUtensorMap& tv, cudaStream_t st) {
-    static bool attr_set = false;  // per process; the attribute is per function, not per device
-    if (!attr_set) {
+    // The shared-memory opt-in is per function and device: set it once per device.
+    static std::atomic<unsigned long long> attr_set{0};
+    int dev = 0;
+    cudaError_t e0 = cudaGetDevice(&dev);
+    if (e0 != cudaSuccess) return e0;
+    const unsigned long long bit = 1ull << (dev & 63);
+    if (!(attr_set.load() & bit)) {
         cudaError_t e = cudaFuncSetAttribute(chunk_fwd_tc_mlp64, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)tc::kSmemBytes);
         if (e != cudaSuccess) return e;
-        attr_set = true;
+        attr_set.fetch_or(bit);
     }
     chunk_fwd_tc_mlp64<<<(unsigned)a.units, tc::kThreads, tc::kSmemBytes, st>>>(
         tk, tq, tv, a.alpha, a.eta, a.theta, a.W1, a.W2, a.S1, a.S2, (__nv_bfloat16*)a.y, a.T, a.chunk, a.status);

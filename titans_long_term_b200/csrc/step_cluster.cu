@@ -14,6 +14,8 @@
 #include <cooperative_groups.h>
 #include <cuda_bf16.h>
 
+#include <atomic>
+
 #include "kernels.h"
 
 namespace cg = cooperative_groups;
@@ -217,12 +219,17 @@ __global__ void __launch_bounds__(kStepThreads, 2) step_mlp_cluster(
 template <int D, typename Tin>
 static cudaError_t launch_step(const ForwardArgs& a, cudaStream_t st) {
     constexpr int C = 4 * D / kSlice;
-    static bool attr_set = false;  // per process; the attribute is per function, not per device
-    if (!attr_set) {
+    // The shared-memory opt-in is per function and device: set it once per device.
+    static std::atomic<unsigned long long> attr_set{0};
+    int dev = 0;
+    cudaError_t e0 = cudaGetDevice(&dev);
+    if (e0 != cudaSuccess) return e0;
+    const unsigned long long bit = 1ull << (dev & 63);
+    if (!(attr_set.load() & bit)) {
         cudaError_t e = cudaFuncSetAttribute(step_mlp_cluster<D, Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)step_smem_bytes<D>());
         if (e != cudaSuccess) return e;
-        attr_set = true;
+        attr_set.fetch_or(bit);
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(a.units * C));
