@@ -335,7 +335,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
                     const uint32_t off = (uint32_t)(lane + 32 * i) * 16u;
                     const int row = (lane + 32 * i) >> 3;
                     const uint4 kv = ld_shared_v4(sb + KQb + off);
-                    const float cr = -cc[row], dr = -dd[row];
+                    const float cr = -0.5f * cc[row], dr = -0.5f * dd[row];  // W1, S1 are kept halved
                     const uint32_t in[4] = {kv.x, kv.y, kv.z, kv.w};
                     uint32_t oc[4], od[4];
 #pragma unroll
@@ -516,10 +516,10 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
                 const float4 x = p[i];
-                w1[4 * i] = x.x;
-                w1[4 * i + 1] = x.y;
-                w1[4 * i + 2] = x.z;
-                w1[4 * i + 3] = x.w;
+                w1[4 * i] = 0.5f * x.x;
+                w1[4 * i + 1] = 0.5f * x.y;
+                w1[4 * i + 2] = 0.5f * x.z;
+                w1[4 * i + 3] = 0.5f * x.w;
             }
             const float* q2 = W2g + u * kD * kH + hrow;
 #pragma unroll
@@ -530,7 +530,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
             for (int blk = 0; blk < 4; ++blk) {
                 uint32_t r[16];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(p1[16 * blk + i]);
+                for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(0.5f * p1[16 * blk + i]);
                 tmem_st16(t_s + 16 * blk, r);
 #pragma unroll
                 for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(p2[(size_t)(16 * blk + i) * kH]);
@@ -568,12 +568,14 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
 #pragma unroll
                 for (int i = 0; i < 16; i += 2) {
                     // silu(z) = h (1 + tanh h), silu'(z) = (1 + tanh h + h (1 - tanh^2 h)) / 2, h = z / 2
-                    const float h0 = 0.5f * __uint_as_float(rk[i]), h1 = 0.5f * __uint_as_float(rk[i + 1]);
+                    const float h0 = __uint_as_float(rk[i]), h1 = __uint_as_float(rk[i + 1]);
                     const float t0_ = tanh_approx(h0), t1_ = tanh_approx(h1);
-                    pk[i / 2] = pack_bf16x2(fmaf(h0, t0_, h0), fmaf(h1, t1_, h1));
-                    rk[i] = __float_as_uint(fmaf(0.5f, t0_ + fmaf(-h0 * t0_, t0_, h0), 0.5f));
-                    rk[i + 1] = __float_as_uint(fmaf(0.5f, t1_ + fmaf(-h1 * t1_, t1_, h1), 0.5f));
-                    const float g0 = 0.5f * __uint_as_float(rq[i]), g1 = 0.5f * __uint_as_float(rq[i + 1]);
+                    const float a0 = fmaf(h0, t0_, h0), a1 = fmaf(h1, t1_, h1);  // silu
+                    const float s0 = fmaf(0.5f, t0_, 0.5f), s1 = fmaf(0.5f, t1_, 0.5f);  // sigmoid
+                    pk[i / 2] = pack_bf16x2(a0, a1);
+                    rk[i] = __float_as_uint(fmaf(-a0, s0, a0 + s0));  // silu' = sigma + silu (1 - sigma)
+                    rk[i + 1] = __float_as_uint(fmaf(-a1, s1, a1 + s1));
+                    const float g0 = __uint_as_float(rq[i]), g1 = __uint_as_float(rq[i + 1]);
                     pq[i / 2] = pack_bf16x2(fmaf(g0, tanh_approx(g0), g0), fmaf(g1, tanh_approx(g1), g1));
                 }
                 tmem_st16(t_work + 16 * blk, rk);
@@ -724,7 +726,8 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
         {
             float4* p = reinterpret_cast<float4*>(W1g + (u * kH + hrow) * kD);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) p[i] = make_float4(w1[4 * i], w1[4 * i + 1], w1[4 * i + 2], w1[4 * i + 3]);
+            for (int i = 0; i < 16; ++i)
+                p[i] = make_float4(2.f * w1[4 * i], 2.f * w1[4 * i + 1], 2.f * w1[4 * i + 2], 2.f * w1[4 * i + 3]);
             float* q2 = W2g + u * kD * kH + hrow;
 #pragma unroll
             for (int i = 0; i < 64; ++i) q2[(size_t)i * kH] = w2[i];
@@ -736,7 +739,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
                 tmem_ld16(t_s + 16 * blk, r);
                 tmem_wait_ld();
 #pragma unroll
-                for (int i = 0; i < 16; ++i) p1[16 * blk + i] = __uint_as_float(r[i]);
+                for (int i = 0; i < 16; ++i) p1[16 * blk + i] = 2.f * __uint_as_float(r[i]);
                 tmem_ld16(t_s + 64 + 16 * blk, r);
                 tmem_wait_ld();
 #pragma unroll
