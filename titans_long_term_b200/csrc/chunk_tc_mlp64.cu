@@ -558,7 +558,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
             // The previous chunk's S accumulations read this tile's A_K and Delta^T rows.
             if (c > 0 && !wait(B_SA0 + tile, (uint32_t)(c - 1) & 1u)) break;
             tc_fence_after();
-#pragma unroll
+#pragma unroll 1
             for (int blk = 0; blk < 4; ++blk) {  // keys and queries, 16-column blocks
                 uint32_t rk[16], rq[16];
                 tmem_ld16(t_work + 16 * blk, rk);
@@ -684,7 +684,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
             // (4) Delta^T = (GW2)^T * silu'(Z_K)^T -> AT1 rows (the queries' tile was consumed by Y)
             if (!wait(B_GW0 + tile, ph)) break;
             tc_fence_after();
-#pragma unroll
+#pragma unroll 1
             for (int blk = 0; blk < 4; ++blk) {
                 uint32_t g[16], sp[16];
                 tmem_ld16(t_work + 64 + 16 * blk, g);
