@@ -399,9 +399,15 @@ def decode_arm(args, w, rank, world, local_rank):
 
 
 def kernel_sha() -> str:
+    """sha1 (first 12 hex digits) of the tensor-core kernel's source with `//` comments and
+    blank lines removed, so that the stored DRAM counters stay matched to the code across
+    comment-only edits and go stale on any code change."""
     import hashlib
+    import re
     p = os.path.join(HERE, "titans_long_term_b200", "csrc", "chunk_tc_mlp64.cu")
-    return hashlib.sha1(open(p, "rb").read()).hexdigest()[:12]
+    lines = [re.sub(r"\s*//.*$", "", ln).rstrip() for ln in open(p).read().splitlines()]
+    code = "\n".join(ln for ln in lines if ln)
+    return hashlib.sha1(code.encode()).hexdigest()[:12]
 
 
 def main():

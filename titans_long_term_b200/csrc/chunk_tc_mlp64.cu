@@ -15,23 +15,25 @@
 //   dW2^T   [h x d]  = A_K^T diag(-c|-d) G
 // The hidden unit sits on the TMEM lane, so each thread of the epilogue warps owns one
 // hidden row j of every state matrix:
-//   - W1[j, :] and W2[:, j] (fp32) live in that thread's registers,
-//   - S1[j, :] and S2[:, j] (fp32) live in TMEM and are the accumulators of the
-//     d-weighted GEMMs (scaled by E before the GEMMs accumulate -sum d_j g_j; the four
-//     producer warps do that pass, one TMEM lane quadrant each, while the epilogue warps
-//     run the SiLU),
+//   - W1[j, :] and W2[:, j] (fp32) live in that thread's registers (W1 at half scale, so
+//     the Z GEMM yields h = z/2, the argument of tanh in silu(z) = h (1 + tanh h)),
+//   - S1[j, :] (half scale) and S2[:, j] (fp32) live in TMEM and are the accumulators of
+//     the d-weighted GEMMs,
 //   - the bf16 copies of W1 and W2^T that feed the MMAs are rewritten in shared memory
 //     once per chunk.
+// Per chunk, on the epilogue warps: SiLU of Z (keys also silu'); the momentum pre-pass
+// W <- A W + sigma S (reads S only) while the tensor core computes Y; G and y; Delta;
+// W += dW_c and the bf16 rows. The decay S <- E S is done by the four producer warps, one
+// TMEM lane quadrant each; the d-weighted GEMMs (S accumulation) are issued after the
+// weight GEMMs, off the weight-update path.
 // Warp roles (12 warps, one CTA per SM, persistent over the chunk loop of one unit):
 //   - warps 0-3 own hidden rows 0..127 ("tile 0"), warps 4-7 rows 128..255 ("tile 1");
-//     the two tiles run their epilogues independently, so the tensor core works on one
-//     tile while the other tile's warps run theirs;
 //   - warps 8 and 9 issue tile 0's and tile 1's forward, backprop and W1-side MMAs (one
-//     elected lane each: a single thread issues a tcgen05.mma only every ~80-200 cycles,
+//     elected lane each: a single thread issues a tcgen05.mma only every ~100 cycles,
 //     so more issuers shorten each MMA phase); Y is split into the two tiles' partial sums
 //     over their hidden units, so those issuers never need ordering; warp 8 also issues
 //     the TMA loads (K, Q, V two chunks ahead);
-//   - warp 11 issues both tiles' W2-side weight GEMMs (S2^T accumulation, dW2^T_c);
+//   - warp 11 issues both tiles' W2-side weight GEMMs (dW2^T_c, then S2^T accumulation);
 //   - warp 10 prefetches the gates, runs the gate scan a chunk ahead and writes the scaled
 //     key tiles. The producer warpgroup (warps 8-11) hands registers to the epilogue
 //     warpgroups (setmaxnreg).
