@@ -12,7 +12,6 @@ namespace titans {
 // Device status bits (atomicOr'ed into the handle's status word).
 constexpr unsigned kStatusTimeoutTma = 1u;
 constexpr unsigned kStatusTimeoutMma = 2u;
-constexpr unsigned kStatusBadLaunch = 4u;
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;  // 1 s
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
