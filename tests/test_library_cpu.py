@@ -55,3 +55,21 @@ def test_null_arguments():
     assert rc == mem.EINVAL
     rc = L.titans_mem_step(None, None, None, None, None, None, None, None, None, None, None, None, None)
     assert rc == mem.EINVAL
+
+
+def test_host_staged_forward_rejects_null_handle_and_buffers():
+    L = mem.lib()
+    rc = L.titans_mem_forward_host(None, None, None, None, None, None, None, 16, 16, None, None, None, None, None,
+                                   None, 0, None)
+    assert rc == mem.EINVAL
+    assert "handle" in L.titans_last_error_string().decode()
+
+
+def test_noalloc_rejects_bad_config_before_cuda():
+    L = mem.lib()
+    assert L.titans_mem_forward_noalloc(None, None, None, None, None, None, None, 16, 16, None, None, None, None,
+                                        None, None) == mem.EINVAL
+    cfg = mem.Config(96, 0, 16, mem.FP32, 1, 1, 0)  # unsupported d
+    rc = L.titans_mem_forward_noalloc(ctypes.byref(cfg), None, None, None, None, None, None, 16, 16, None, None,
+                                      None, None, None, None)
+    assert rc in (mem.EINVAL, mem.EUNSUPPORTED)
