@@ -121,6 +121,7 @@ titans::ForwardArgs make_args(titans_mem* m, const void* k, const void* q, const
     a.alpha = al;
     a.eta = et;
     a.theta = th;
+    a.gate_ld = T;
     a.W1 = W1;
     a.W2 = W2;
     a.S1 = S1;
@@ -197,9 +198,14 @@ int titans_mem_path(titans_mem_t m, int chunk, int step) {
     return tc_eligible(m->cfg, chunk) ? TITANS_PATH_TC_MLP64 : TITANS_PATH_CUDA_CORES;
 }
 
-titans_status_t titans_mem_forward(titans_mem_t m, const void* k, const void* q, const void* v, const float* alpha,
-                                   const float* eta, const float* theta, long T, int chunk, float* W1, float* W2,
-                                   float* S1, float* S2, void* y, void* stream) {
+}  // extern "C"
+
+namespace {
+// titans_mem_forward with the gates' row stride given separately (gate_ld >= T): the host-staged
+// path reads the segments' gates in place from the full [units][T_total] arrays.
+titans_status_t forward_impl(titans_mem_t m, const void* k, const void* q, const void* v, const float* alpha,
+                             const float* eta, const float* theta, long gate_ld, long T, int chunk, float* W1,
+                             float* W2, float* S1, float* S2, void* y, void* stream) {
     if (!m) return fail(TITANS_EINVAL, "handle is NULL");
     titans_status_t s = check_ptrs(m, k, q, v, alpha, eta, theta, W1, W2, S1, S2, y);
     if (s != TITANS_OK) return s;
@@ -209,6 +215,7 @@ titans_status_t titans_mem_forward(titans_mem_t m, const void* k, const void* q,
         return fail(TITANS_EUNSUPPORTED, "chunk must be in 1..config.chunk");
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     titans::ForwardArgs a = make_args(m, k, q, v, alpha, eta, theta, T, chunk, W1, W2, S1, S2, y);
+    a.gate_ld = gate_ld;
     cudaError_t e;
     if (tc_eligible(m->cfg, chunk)) {
         if (T >= (1L << 31) || a.units >= (1L << 31)) return fail(TITANS_EUNSUPPORTED, "T or units too large");
@@ -222,6 +229,16 @@ titans_status_t titans_mem_forward(titans_mem_t m, const void* k, const void* q,
     }
     if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
     return TITANS_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+titans_status_t titans_mem_forward(titans_mem_t m, const void* k, const void* q, const void* v, const float* alpha,
+                                   const float* eta, const float* theta, long T, int chunk, float* W1, float* W2,
+                                   float* S1, float* S2, void* y, void* stream) {
+    return forward_impl(m, k, q, v, alpha, eta, theta, T, T, chunk, W1, W2, S1, S2, y, stream);
 }
 
 titans_status_t titans_mem_forward_host(titans_mem_t m, const void* k, const void* q, const void* v,
@@ -263,30 +280,35 @@ titans_status_t titans_mem_forward_host(titans_mem_t m, const void* k, const voi
     const size_t es = m->cfg.mode == TITANS_BF16 ? 2 : 4;  // token element size
     const size_t units = (size_t)m->cfg.B * m->cfg.H, d = (size_t)m->cfg.d;
     const size_t row_h = (size_t)T * d * es;  // one unit's host stream of k, q, v or y
-    // Copies and forward of segment i: tokens [t0, t0 + tn) of every unit, packed on the
-    // device as [units][tn][...] at the offset of the segments before it.
+    // The gates go over whole ([units][T], contiguous: one copy each, 12 B per head-token) and
+    // the forward of each segment reads its columns in place. The tokens of segment i, [t0, t0 +
+    // tn) of every unit, are packed on the device as [units][tn][d] at the offset of the segments
+    // before it, so that each segment's k, q, v copy overlaps the previous segment's compute.
     e = cudaEventRecord(m->ev[0], st);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(m->s_in, m->ev[0], 0);
     if (e != cudaSuccess) return cuda_fail(e, "ordering after the caller's stream");
+    {
+        float* dg[3] = {dev->alpha, dev->eta, dev->theta};
+        const float* hg[3] = {alpha, eta, theta};
+        for (int j = 0; j < 3 && e == cudaSuccess; ++j)
+            e = cudaMemcpyAsync(dg[j], hg[j], units * (size_t)T * 4, cudaMemcpyHostToDevice, m->s_in);
+        if (e != cudaSuccess) return cuda_fail(e, "copying the gates in");
+    }
     for (long i = 0; i < nseg; ++i) {
         const long t0 = i * t_seg, tn = std::min(t_seg, T - t0);
-        const size_t tok_off = units * (size_t)t0 * d * es, gate_off = units * (size_t)t0;
+        const size_t tok_off = units * (size_t)t0 * d * es;
         char* dk[3] = {static_cast<char*>(dev->k) + tok_off, static_cast<char*>(dev->q) + tok_off,
                        static_cast<char*>(dev->v) + tok_off};
         const char* hk[3] = {static_cast<const char*>(k), static_cast<const char*>(q), static_cast<const char*>(v)};
         for (int j = 0; j < 3 && e == cudaSuccess; ++j)
             e = cudaMemcpy2DAsync(dk[j], (size_t)tn * d * es, hk[j] + (size_t)t0 * d * es, row_h, (size_t)tn * d * es,
                                   units, cudaMemcpyHostToDevice, m->s_in);
-        float* dg[3] = {dev->alpha + gate_off, dev->eta + gate_off, dev->theta + gate_off};
-        const float* hg[3] = {alpha, eta, theta};
-        for (int j = 0; j < 3 && e == cudaSuccess; ++j)
-            e = cudaMemcpy2DAsync(dg[j], (size_t)tn * 4, hg[j] + t0, (size_t)T * 4, (size_t)tn * 4, units,
-                                  cudaMemcpyHostToDevice, m->s_in);
         if (e == cudaSuccess) e = cudaEventRecord(m->ev[2 + 2 * i], m->s_in);
         if (e == cudaSuccess) e = cudaStreamWaitEvent(st, m->ev[2 + 2 * i], 0);
         if (e != cudaSuccess) return cuda_fail(e, "copying a segment in");
         char* dy = static_cast<char*>(dev->y) + tok_off;
-        s = titans_mem_forward(m, dk[0], dk[1], dk[2], dg[0], dg[1], dg[2], tn, chunk, W1, W2, S1, S2, dy, stream);
+        s = forward_impl(m, dk[0], dk[1], dk[2], dev->alpha + t0, dev->eta + t0, dev->theta + t0, T, tn, chunk, W1,
+                         W2, S1, S2, dy, stream);
         if (s != TITANS_OK) return s;
         e = cudaEventRecord(m->ev[3 + 2 * i], st);
         if (e == cudaSuccess) e = cudaStreamWaitEvent(m->s_out, m->ev[3 + 2 * i], 0);

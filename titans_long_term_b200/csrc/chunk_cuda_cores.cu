@@ -34,7 +34,7 @@ __host__ size_t cuda_cores_ws_floats(int d, int h, int n) {
 
 template <typename Tin>
 __global__ void __launch_bounds__(kCcThreads) chunk_fwd_cuda_cores(
-    int d, int h, long T, int chunk, const Tin* __restrict__ k, const Tin* __restrict__ q,
+    int d, int h, long T, long gate_ld, int chunk, const Tin* __restrict__ k, const Tin* __restrict__ q,
     const Tin* __restrict__ v, const float* __restrict__ alpha, const float* __restrict__ eta,
     const float* __restrict__ theta, float* __restrict__ W1, float* __restrict__ W2, float* __restrict__ S1,
     float* __restrict__ S2, Tin* __restrict__ y, float* __restrict__ ws, size_t ws_per_unit) {
@@ -49,9 +49,9 @@ __global__ void __launch_bounds__(kCcThreads) chunk_fwd_cuda_cores(
     q += u * T * d;
     v += u * T * d;
     y += u * T * d;
-    alpha += u * T;
-    eta += u * T;
-    theta += u * T;
+    alpha += u * gate_ld;
+    eta += u * gate_ld;
+    theta += u * gate_ld;
     W1 += u * nW1;
     S1 += u * nW1;
     if (h) {
@@ -188,7 +188,7 @@ __global__ void __launch_bounds__(kCcThreads) chunk_fwd_cuda_cores(
 template <typename Tin>
 cudaError_t launch_cuda_cores(const ForwardArgs& a, cudaStream_t st) {
     chunk_fwd_cuda_cores<Tin><<<(unsigned)a.units, kCcThreads, 0, st>>>(
-        a.d, a.h, a.T, a.chunk, (const Tin*)a.k, (const Tin*)a.q, (const Tin*)a.v, a.alpha, a.eta, a.theta, a.W1,
+        a.d, a.h, a.T, a.gate_ld, a.chunk, (const Tin*)a.k, (const Tin*)a.q, (const Tin*)a.v, a.alpha, a.eta, a.theta, a.W1,
         a.W2, a.S1, a.S2, (Tin*)a.y, a.ws, a.ws_per_unit);
     return cudaGetLastError();
 }

@@ -205,7 +205,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ,
     const __grid_constant__ CUtensorMap tmV, const float* __restrict__ alpha, const float* __restrict__ eta,
     const float* __restrict__ theta, float* __restrict__ W1g, float* __restrict__ W2g, float* __restrict__ S1g,
-    float* __restrict__ S2g, __nv_bfloat16* __restrict__ yg, long T, int chunk, unsigned* status) {
+    float* __restrict__ S2g, __nv_bfloat16* __restrict__ yg, long T, long gate_ld, int chunk, unsigned* status) {
     using namespace tc;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -297,7 +297,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
             for (int i = 0; i < 2; ++i) {
                 const int j = lane + 32 * i;
                 const bool ok = j < n;
-                const long g = u * T + t0 + j;
+                const long g = u * gate_ld + t0 + j;
                 ga[i] = ok ? __ldg(alpha + g) : 0.f;
                 ge[i] = ok ? __ldg(eta + g) : 1.f;
                 gt[i] = ok ? __ldg(theta + g) : 0.f;
@@ -775,7 +775,7 @@ cudaError_t launch_chunk_tc_mlp64(const ForwardArgs& a, const CUtensorMap& tk, c
         attr_set.fetch_or(bit);
     }
     chunk_fwd_tc_mlp64<<<(unsigned)a.units, tc::kThreads, tc::kSmemBytes, st>>>(
-        tk, tq, tv, a.alpha, a.eta, a.theta, a.W1, a.W2, a.S1, a.S2, (__nv_bfloat16*)a.y, a.T, a.chunk, a.status);
+        tk, tq, tv, a.alpha, a.eta, a.theta, a.W1, a.W2, a.S1, a.S2, (__nv_bfloat16*)a.y, a.T, a.gate_ld, a.chunk, a.status);
     return cudaGetLastError();
 }
 

@@ -125,6 +125,7 @@ extern "C" titans_status_t titans_mem_forward_noalloc(const titans_mem_config* c
     a.alpha = alpha;
     a.eta = eta;
     a.theta = theta;
+    a.gate_ld = T;
     a.W1 = W1;
     a.W2 = W2;
     a.S1 = S1;

@@ -13,6 +13,7 @@ struct ForwardArgs {
     bool bf16;         // k, q, v, y dtype
     const void *k, *q, *v;
     const float *alpha, *eta, *theta;
+    long gate_ld;      // elements between consecutive units' gate rows (T for [B, H, T])
     float *W1, *W2, *S1, *S2;
     void* y;
     float* ws;         // CUDA-core path workspace
