@@ -294,4 +294,58 @@ def pin_unit_equivariance(fwd):
     assert np.array_equal(y[p], y2) and all(np.array_equal(a[nm][p], b[nm]) for nm in a)
 
 
+def pin_sign_symmetry(fwd):
+    """The loss ||W2 a - v||^2 is unchanged by (W2, v) -> (-W2, -v): the error e flips sign, the
+    W2 gradient 2 e a^T flips sign, and the W1 gradient (W2^T 2e) * silu' k^T does not. So negating
+    W2, S2 and v negates y, W2 and S2 and leaves W1 and S1 unchanged (bitwise: only negations)."""
+    d, h, T, n = 5, 8, 19, 4
+    k, q, v, al, et, th, st = _mk(1, T, d, h, 31)
+    st["S1"] = 0.01 * st["W1"][::-1].copy()
+    st["S2"] = 0.01 * st["W2"][::-1].copy()
+    y, a = fwd(k, q, v, al, et, th, st, n)
+    neg = dict(st, W2=-st["W2"], S2=-st["S2"])
+    y2, b = fwd(k, q, -v, al, et, th, neg, n)
+    assert np.array_equal(y2, -y)
+    assert np.array_equal(b["W1"], a["W1"]) and np.array_equal(b["S1"], a["S1"])
+    assert np.array_equal(b["W2"], -a["W2"]) and np.array_equal(b["S2"], -a["S2"])
+
+
+def pin_zero_w2_first_chunk(fwd):
+    """W2_0 = 0, S_0 = 0: the memory outputs 0, so within the first chunk every W1 gradient
+    vanishes and every W2 gradient is 2 (0 - v_j) a_j^T with a_j = silu(W1_0 k_j). Unrolling
+    S_t = eta_t S_{t-1} - theta_t g_t, W_t = (1 - alpha_t) W_{t-1} + S_t by hand over the chunk:
+      W2_n = sum_j c_j 2 v_j a_j^T,  S2_n = sum_j d_j 2 v_j a_j^T,  W1_n = prod_l (1 - alpha_l) W1_0,
+    with c_j = theta_j sum_{m >= j} prod_{j < l <= m} eta_l prod_{l > m} (1 - alpha_l) and
+    d_j = theta_j prod_{l > j} eta_l, evaluated here by nested loops; y = 0 in the chunk."""
+    d, h, n = 4, 7, 6
+    k, q, v, al, et, th, st = _mk(1, n, d, h, 37)
+    st["W2"][:] = 0.0
+    y, out = fwd(k, q, v, al, et, th, st, n)
+    assert not np.any(y)
+    W1 = st["W1"][0]
+    a = [torch.nn.functional.silu(torch.tensor(W1 @ k[0, j].astype(np.float64))).numpy() for j in range(n)]
+    al64, et64, th64 = (x[0].astype(np.float64) for x in (al, et, th))
+    W2n = np.zeros((d, h))
+    S2n = np.zeros((d, h))
+    for j in range(n):
+        c = 0.0
+        for m in range(j, n):
+            term = 1.0
+            for l in range(j + 1, m + 1):
+                term *= et64[l]
+            for l in range(m + 1, n):
+                term *= 1.0 - al64[l]
+            c += term
+        dj = 1.0
+        for l in range(j + 1, n):
+            dj *= et64[l]
+        outer = 2.0 * np.outer(v[0, j].astype(np.float64), a[j])
+        W2n += th64[j] * c * outer
+        S2n += th64[j] * dj * outer
+    _close(out["W2"][0], W2n, 1e-12, "W2 after the first chunk")
+    _close(out["S2"][0], S2n, 1e-12, "S2 after the first chunk")
+    _close(out["W1"][0], np.prod(1.0 - al64) * W1, 1e-12, "W1 (pure decay)")
+    assert not np.any(out["S1"])
+
+
 PINS = [v for k_, v in sorted(globals().items()) if k_.startswith("pin_")]
