@@ -83,11 +83,11 @@ enum Bar {
     B_Y0, B_Y1,          // partial Y of tile t (sum over its hidden units) done
     B_G,                 // G tiles written, Y read (all epilogue threads)
     B_S0, B_S1,          // tile t's momentum pre-pass done
-    B_GW0, B_GW1,        // (GW2)^T and the S2^T accumulation of tile t done
+    B_GW0, B_GW1,        // (GW2)^T of tile t done
     B_D0, B_D1,          // tile t wrote Delta^T rows
-    B_DW0, B_DW1,        // weighted W1 GEMMs of tile t done (dW1_c, S1 accumulation)
-    B_DX0, B_DX1,        // weighted W2 GEMMs of tile t done (S2^T accumulation, dW2^T_c)
-    B_W0, B_W1,          // tile t rewrote its bf16 weight rows (and read dW_c)
+    B_DW0, B_DW1,        // dW1_c of tile t done
+    B_DX0, B_DX1,        // dW2^T_c of tile t done
+    B_W0, B_W1,          // tile t rewrote its bf16 weight rows (and read dW1_c, dW2^T_c)
     B_SC0, B_SC1,        // gate scan of a chunk with parity 0 / 1 published
     B_KC,                // scaled key tiles of the chunk written
     B_RS,                // the four producer warps scaled S <- E S for the chunk
