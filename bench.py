@@ -186,7 +186,8 @@ def reference_arm(args, w, rank, world):
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
             "impl": "reference",
             "config": {"workload": w.name, "memory": f"MLP {w.d}-{w.h}-{w.d} SiLU" if w.h else f"linear {w.d}",
-                       "B": w.B, "H": w.H, "T": w.T, "chunk": w.chunk, "units": w.units},
+                       "B": w.B, "H": w.H, "T": w.T, "chunk": w.chunk, "units": w.units,
+                       "inputs": synth.describe(w)},
             "cpu_baseline": base,
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -311,7 +312,7 @@ def our_arm(args, w, rank, world, local_rank):
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "fp32",
         "data": "synthetic (seeded; k, v, q projections of one x_t)",
-        "config": {"workload": w.name,
+        "config": {"workload": w.name, "inputs": synth.describe(w),
                    "memory": f"MLP {w.d}-{w.h}-{w.d} SiLU" if w.h else f"linear {w.d}x{w.d}",
                    "B": w.B, "H": w.H, "T": w.T, "chunk": w.chunk, "units_per_gpu": w.units,
                    "kernel": {1: "tcgen05 chunk kernel", 2: "CUDA-core chunk kernel"}.get(path, str(path)),
@@ -331,17 +332,84 @@ def our_arm(args, w, rank, world, local_rank):
         "gpu_launches": args.steps,
         "clocks": clocks.summary(),
     }
+    if world == 1 and not args.no_extras:
+        del toks, gates, state0, state, y, host, y_host, staging, m
+        torch.cuda.empty_cache()
+        line["results"] = extra_results(args, dev)
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = oracle_sample(w)
     print(json.dumps(line), flush=True)
 
 
-def decode_arm(args, w, rank, world, local_rank):
+FP32_FMA_TFLOPS_NOMINAL = 148 * 128 * 2 * 1.965e9 / 1e12  # SMs x FMA lanes x 2 FLOP x max SM clock
+
+
+def time_launches(fn, stream, steps: int, warmup: int):
+    """Device time of `steps` calls of fn after `warmup` untimed ones: CUDA events on the launching
+    stream around the whole run and around each launch. Returns (total ms, [per-launch ms])."""
+    for _ in range(warmup):
+        fn()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for i in range(steps):
+        evs[i][0].record(stream)
+        fn()
+        evs[i][1].record(stream)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    return t0.elapsed_time(t1), [a.elapsed_time(b) for a, b in evs]
+
+
+def forward_measure(w, dev, steps: int, warmup: int, T=None):
+    """titans_mem_forward over the whole workload (or its first T tokens per unit), inputs resident in
+    HBM; one launch per step. Returns a result record with the dominant kernel's roofline."""
+    T = w.T if T is None else T
+    inp = synth.make_inputs(w, T=T)
+    toks = {n: inp[n].reshape(w.B, w.H, T, w.d).to(dev) for n in ("k", "q", "v")}
+    gates = {n: inp[n].reshape(w.B, w.H, T).to(dev) for n in ("alpha", "eta", "theta")}
+    state = {n: inp[n].reshape(w.B, w.H, *inp[n].shape[1:]).to(dev) for n in inp if n[0] in "WS"}
+    del inp
+    y = torch.empty_like(toks["k"])
+    m = mem.Memory(w.d, w.h, w.chunk, w.dtype, w.B, w.H)
+    path = m.path()
+    stream = torch.cuda.current_stream(dev)
+    fn = lambda: m.forward(toks["k"], toks["q"], toks["v"], gates["alpha"], gates["eta"], gates["theta"], state, y=y)
+    total, per = time_launches(fn, stream, steps, warmup)
+    m.sync_status()
+    ms = total / steps
+    avg = statistics.mean(per)
+    peaks, which = load_peaks()
+    flops = flops_per_head_token(w) * w.units * T
+    achieved = flops / (avg / 1e3) / 1e12
+    peak = peaks["bf16_tflops"]
+    algo_bytes = stream_bytes_per_head_token(w) * w.units * T + state_bytes_per_unit(w) * w.units
+    kernel = {mem.PATH_TC_MLP64: "chunk_fwd_tc_mlp64", mem.PATH_CUDA_CORES: "chunk_fwd_cuda_cores"}.get(path)
+    sms = min(w.units, 148)
+    rec = {"workload": w.name, "value": w.B * T / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms,
+           "steps": steps, "warmup": warmup, "head_tokens_per_s": w.B * T * w.H / (ms / 1e3),
+           "config": {"memory": f"MLP {w.d}-{w.h}-{w.d} SiLU" if w.h else f"linear {w.d}x{w.d}", "B": w.B,
+                      "H": w.H, "T": w.T, "T_timed": T, "chunk": w.chunk, "units": w.units,
+                      "inputs": synth.describe(w)},
+           "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                        "frac": achieved / peak, "traffic": None, "peak_source": f"bf16_tflops ({which})",
+                        "kernel": kernel, "flops_per_launch": flops, "avg_launch_ms": avg,
+                        "sms_used": sms, "frac_of_sms_used": achieved / (peak * sms / 148),
+                        "algorithmic_bytes_per_launch": algo_bytes},
+           "gpu_launches": steps}
+    if path == mem.PATH_CUDA_CORES:
+        rec["roofline"]["note"] = "CUDA-core fp32 FMA kernel; frac is against the bf16 tensor-core peak the work is bound by"
+        rec["roofline"]["frac_of_fp32_fma_nominal"] = achieved / FP32_FMA_TFLOPS_NOMINAL
+    del toks, gates, state, y, m
+    torch.cuda.empty_cache()
+    return rec
+
+
+def decode_measure(w, dev, steps: int, warmup: int):
     """One step = one titans_mem_step (single-token update + retrieve) for every decode unit
     (decode_B x H), starting from seeded states; bound by HBM: each unit reads and writes its
-    four fp32 state matrices once per step."""
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
+    four fp32 state matrices once per step. Returns (result record, list of per-launch ms)."""
     n = w.decode_B * w.H
     src = synth.decode_state_rows(w)
     st0 = synth.make_inputs(w, units=sorted(set(src.tolist())), T=1)
@@ -349,53 +417,69 @@ def decode_arm(args, w, rank, world, local_rank):
     idx = torch.as_tensor([pos[int(u)] for u in src])
     state = {nm: st0[nm][idx].reshape(w.decode_B, w.H, *st0[nm].shape[1:]).contiguous().to(dev)
              for nm in st0 if nm[0] in "WS"}
-    K = max(args.steps, 1)
+    K = max(steps, 1)
     steps_in = [synth.decode_step_inputs(w, s) for s in range(min(K, 16))]
     dev_in = [{k: v.reshape(w.decode_B, w.H, *v.shape[1:]).to(dev) for k, v in d.items()} for d in steps_in]
     m = mem.Memory(w.d, w.h, 1, w.dtype, w.decode_B, w.H)
     y = torch.empty_like(dev_in[0]["k"])
+    it = [0]
 
-    def step(i):
-        g = dev_in[i % len(dev_in)]
+    def step():
+        g = dev_in[it[0] % len(dev_in)]
+        it[0] += 1
         m.step(g["k"], g["q"], g["v"], g["alpha"], g["eta"], g["theta"], state, y=y)
 
-    for i in range(args.warmup):
-        step(i)
+    total, per = time_launches(step, torch.cuda.current_stream(dev), K, warmup)
     m.sync_status()
-    stream = torch.cuda.current_stream(dev)
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
-    torch.cuda.synchronize(dev)
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
-    for i in range(K):
-        evs[i][0].record(stream)
-        step(i)
-        evs[i][1].record(stream)
-    t1.record(stream)
-    torch.cuda.synchronize(dev)
-    m.sync_status()
-    elapsed = max_over_ranks(t0.elapsed_time(t1), dev, world)
-    if rank != 0:
-        return
-    ms = elapsed / K
-    avg = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    ms = total / K
+    avg = statistics.mean(per)
     peaks, which = load_peaks()
     state_bytes = n * 2 * (4 * w.d * w.h * 4)  # W1, W2, S1, S2 (fp32, d*h each): read once, written once
     io_bytes = n * (4 * w.d * (2 if w.dtype == "bf16" else 4) + 12)
     gbs = (state_bytes + io_bytes) / (avg / 1e3) / 1e9
+    rec = {"workload": w.name + " decode", "value": w.decode_B / (ms / 1e3), "unit": "tokens/s",
+           "ms_per_step": ms, "steps": K, "warmup": warmup,
+           "config": {"decode_B": w.decode_B, "H": w.H, "units": n, "inputs": synth.describe(w),
+                      "l2": "state larger than L2 (%.2f GB per step)" % (state_bytes / 1e9)},
+           "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                        "frac": gbs / peaks["hbm_gbs"], "traffic": None, "peak_source": f"hbm_gbs ({which})",
+                        "kernel": "step_mlp_cluster", "bytes_per_launch": state_bytes + io_bytes,
+                        "avg_launch_ms": avg},
+           "gpu_launches": K}
+    del state, dev_in, y, m
+    torch.cuda.empty_cache()
+    return rec
+
+
+def decode_arm(args, w, rank, world, local_rank):
+    """--phase decode: one JSON line for the decode step alone (every rank runs its own decode batch)."""
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    rec = decode_measure(w, dev, args.steps, args.warmup)
+    ms = max_over_ranks(rec["ms_per_step"], dev, world)
+    if rank != 0:
+        return
+    cfg = dict(rec["config"], workload=rec["workload"])
     print(json.dumps({
         "metric": "decode tokens/sec (single-token update+retrieve, every head) per B200",
-        "value": world * w.decode_B / (ms / 1e3), "unit": "tokens/s", "n_gpus": world, "steps": K,
+        "value": world * w.decode_B / (ms / 1e3), "unit": "tokens/s", "n_gpus": world, "steps": rec["steps"],
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": w.dtype, "data": "synthetic (seeded)",
-        "config": {"workload": w.name + " decode", "decode_B": w.decode_B, "H": w.H, "units": n,
-                   "l2": "state larger than L2 (%.2f GB per step)" % (state_bytes / 1e9)},
-        "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": gbs / peaks["hbm_gbs"], "traffic": None, "peak_source": f"hbm_gbs ({which})",
-                     "kernel": "step_mlp_cluster", "bytes_per_launch": state_bytes + io_bytes,
-                     "avg_launch_ms": avg},
-        "gpu_launches": K}), flush=True)
+        "vs_baseline": None, "dtype": w.dtype, "data": "synthetic (seeded)", "config": cfg,
+        "roofline": rec["roofline"], "gpu_launches": rec["gpu_launches"]}), flush=True)
+
+
+def extra_results(args, dev):
+    """The other workloads' numbers, nested in the one JSON line (rank 0 of a 1-GPU run):
+    the 2048-unit decode step (HBM-bound), the 16-unit long stream (occupancy-limited: one
+    CTA per unit) and the wide memory's prefill."""
+    out = {}
+    steps = max(3, min(args.steps, 20))
+    wide = synth.WORKLOADS["mlp-d128-b4h8-t16k"]
+    out["decode"] = decode_measure(wide, dev, steps, args.warmup)
+    out["long_stream"] = forward_measure(synth.WORKLOADS["mlp-d64-b1h16-t1m"], dev, max(3, min(args.steps, 5)),
+                                         args.warmup)
+    out["wide_prefill"] = forward_measure(wide, dev, max(3, min(args.steps, 5)), args.warmup)
+    return out
 
 
 def kernel_sha() -> str:
@@ -419,6 +503,8 @@ def main():
     ap.add_argument("--workload", default=None, choices=list(synth.WORKLOADS),
                     help="default: mlp-d64-b8h16-t4k for --phase forward, mlp-d128-b4h8-t16k for decode")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the nested decode / long-stream / wide-prefill results of a 1-GPU run")
     ap.add_argument("--phase", choices=["forward", "decode"], default="forward",
                     help="forward: the chunk-wise update + retrieve (default); decode: titans_mem_step")
     ap.add_argument("--decode-b", type=int, default=0, help="decode batch (default: the workload's, 256)")

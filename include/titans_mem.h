@@ -87,6 +87,12 @@ titans_status_t titans_mem_destroy(titans_mem_t m);
 
 /*
  * Chunk-wise forward over T tokens of every unit (update + retrieve).
+ * Defined by the walk-through's sec. 3.2 "How to Parallelize the Long-term Memory Training"
+ * (chunks of b tokens; every token's gradient at the chunk-start weights, t' = t - mod(t, b);
+ * the tensorized mini-batch form, here extended with the momentum term) applied to the
+ * update of sec. 3.1 ("Surprise Metric": S_t = eta_t S_{t-1} - theta_t grad l(M_{t-1}; x_t);
+ * "Forgetting Mechanism": M_t = (1 - alpha_t) M_{t-1} + S_t; "Objective": l = ||M(k) - v||^2)
+ * and the retrieval y_t = M*(q_t) of sec. 3.1 "Retrieving a Memory".
  *   k, q, v     [B, H, T, d]  bf16 (TITANS_BF16) or fp32 (TITANS_FP32)
  *   alpha, eta, theta [B, H, T] fp32; alpha in [0, 1], eta, theta >= 0
  *   MLP state:  W1, S1 [B, H, h, d], W2, S2 [B, H, d, h] fp32;
@@ -129,8 +135,10 @@ typedef struct {
  * queued on it afterwards starts after the last copy of y. The handle's two copy streams are
  * created on first use; calls on one handle must not overlap.
  * Returns TITANS_EINVAL for a null pointer, a misaligned device buffer or a t_seg that is
- * not a multiple of chunk, TITANS_ECUDA if a copy or launch fails (earlier segments may
- * then be queued already), and otherwise what titans_mem_forward returns per segment.
+ * not a multiple of chunk, TITANS_ECUDA if a copy or launch fails, and otherwise what
+ * titans_mem_forward returns per segment. After an error, copies and segments queued
+ * before it may still run; the call has made `stream` wait for them, so synchronize
+ * `stream` before freeing or reusing the buffers.
  */
 titans_status_t titans_mem_forward_host(titans_mem_t m, const void *k, const void *q, const void *v,
                                         const float *alpha, const float *eta, const float *theta,
@@ -140,7 +148,10 @@ titans_status_t titans_mem_forward_host(titans_mem_t m, const void *k, const voi
 
 /*
  * One decode step per unit with chunk = 1 semantics: y = M(q; W_{t-1}), then the
- * update with the gradient at W_{t-1}.
+ * update with the gradient at W_{t-1}. Defined by the walk-through's sec. 3.1: the
+ * per-token recurrence ("Surprise Metric", "Forgetting Mechanism", "Objective") and the
+ * retrieval of "Retrieving a Memory", read with the previous token's memory as the MAC
+ * variant's M*_{t-1} (sec. 4.1); it is sec. 3.2's chunked form with b = 1.
  *   k, q, v [B, H, d] (dtype of the mode); alpha, eta, theta [B, H] fp32;
  *   state as in titans_mem_forward, updated in place; y [B, H, d].
  */
@@ -156,16 +167,19 @@ titans_status_t titans_mem_step(titans_mem_t m, const void *k, const void *q, co
  * handle). The pages on the method have no counterpart: this is a deployment variant.
  *
  * Same arguments and semantics as titans_mem_forward, with the configuration passed
- * directly (cfg->flags is ignored); it always runs the CUDA-core (fp32 arithmetic) chunk
- * kernel. Its scratch is a fixed 16 MiB device array inside the library, held by every GPU
- * that loads the library until the process exits:
- *  - the first call on a device looks up the array there; make it before any stream
- *    capture meant to contain later calls;
+ * directly. cfg->flags and cfg->chunk are ignored: `chunk` may be any length in 1..128.
+ * It always runs the CUDA-core (fp32 arithmetic) chunk kernel, never the tensor-core one,
+ * so its results equal, bit for bit, those of titans_mem_forward on that kernel (fp32
+ * mode, or TITANS_FLAG_CUDA_CORES). Its scratch is a fixed 16 MiB device array inside the
+ * library, held by every GPU that loads the library until the process exits:
+ *  - the first call on a device looks up the array there and loads the kernel's code for
+ *    both modes; make it before any stream capture meant to contain later calls;
  *  - every call shares the array, so calls that overlap on a GPU race: serialize them;
  *  - nothing in the array needs clearing between calls;
  *  - a call needing more than the array holds -- B*H units x (4*chunk*h + chunk*d floats
  *    for the MLP memory, chunk*d for the linear one, each rounded up to 64 floats) -- returns
- *    TITANS_EUNSUPPORTED with a message in titans_last_error_string().
+ *    TITANS_EUNSUPPORTED with a message in titans_last_error_string(); B*H above 2^30
+ *    returns TITANS_EINVAL.
  * No device status word: the kernel has no waits to time out.
  */
 titans_status_t titans_mem_forward_noalloc(const titans_mem_config *cfg, const void *k, const void *q,

@@ -72,3 +72,17 @@ def compare(gy, gst, ry, rst, tol, units: Optional[Sequence[int]] = None, what="
 def workload_inputs(name: str, T: Optional[int] = None, units=None, dtype: Optional[str] = None):
     w = synth.WORKLOADS[name]
     return w, synth.make_inputs(w, units=units, T=T, dtype=dtype)
+
+
+def step_sequence(m, inp, B, H, steps):
+    """`steps` titans_mem_step calls over the first tokens of `inp`; returns y [U, steps, d] and the state."""
+    toks, gates, state = gpu_inputs(inp, B, H)
+    ys = []
+    for t in range(steps):
+        sl = lambda x: x[:, :, t].contiguous()
+        ys.append(m.step(sl(toks["k"]), sl(toks["q"]), sl(toks["v"]), sl(gates["alpha"]), sl(gates["eta"]),
+                         sl(gates["theta"]), state))
+    m.sync_status()
+    U = B * H
+    y = torch.stack(ys, dim=2).reshape(U, steps, -1).float().cpu().numpy()
+    return y, {n: t.reshape(U, *t.shape[2:]).float().cpu().numpy() for n, t in state.items()}

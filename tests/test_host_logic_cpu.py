@@ -131,3 +131,59 @@ def test_kernel_hash_ignores_comments(bench, tmp_path, monkeypatch):
     assert bench.kernel_sha() == h0
     (d / "chunk_tc_mlp64.cu").write_text(text.replace("kThreads = 384", "kThreads = 385"))
     assert bench.kernel_sha() != h0
+
+
+def test_stated_recipe_draws_independent_tokens_with_the_stated_gate_ranges():
+    """The stated recipe: k, q, v ~ N(0, I) drawn independently (k, q l2-normalised) and gates
+    alpha ~ U(0, 0.05), eta ~ U(0.8, 0.99), theta ~ U(0, 0.1). In the projected recipe v is a
+    linear image of the same x as k, so least squares recovers v from k almost exactly; in the
+    stated recipe it explains next to nothing."""
+    n = 4096
+    st = synth.unit_tokens(W_SMALL, 1, 0, n, recipe="stated")
+    pr = synth.unit_tokens(W_SMALL, 1, 0, n, recipe="projected")
+    for n_ in ("k", "q"):
+        norms = st[n_].norm(dim=1)
+        assert torch.allclose(norms, torch.ones_like(norms), atol=1e-5)
+    assert 0.95 < float(st["v"].std()) < 1.05 and abs(float(st["v"].mean())) < 0.02
+
+    def r2(k, v):
+        sol = torch.linalg.lstsq(k.double(), v.double()).solution
+        res = v.double() - k.double() @ sol
+        return 1.0 - float(res.pow(2).sum() / (v.double() - v.double().mean(0)).pow(2).sum())
+    assert r2(pr["k"], pr["v"]) > 0.5  # k is v's x, renormalised per token
+    assert r2(st["k"], st["v"]) < 0.05
+    amax, elo, ehi, tmax = synth._gate_ranges(W_SMALL, "stated")
+    assert (amax, elo, ehi, tmax) == (0.05, 0.8, 0.99, 0.1)
+    assert 0 <= float(st["alpha"].min()) and float(st["alpha"].max()) <= amax
+    assert float(st["alpha"].max()) > 0.99 * amax  # spans the range, not the projected recipe's
+    assert elo <= float(st["eta"].min()) and float(st["eta"].max()) <= ehi
+    assert 0 <= float(st["theta"].min()) and float(st["theta"].max()) <= tmax
+    assert float(st["theta"].max()) > 0.99 * tmax
+    # its own generators: no stream shared with the projected recipe
+    assert not torch.equal(st["alpha"], pr["alpha"])
+
+
+def test_linear_workload_defaults_to_the_stated_recipe():
+    w = synth.WORKLOADS["linear-d64"]
+    assert w.recipe == "stated"
+    a = synth.make_inputs(w, T=64)
+    b = synth.make_inputs(w, T=64, recipe="stated")
+    assert all(torch.equal(a[n], b[n]) for n in a)
+    d = synth.describe(w)
+    assert d["recipe"] == "stated" and d["alpha"] == "U(0, 0.05)" and d["theta"] == "U(0, 0.1)"
+    assert synth.describe(W_SMALL)["theta"] == "U(0, 0.003)"
+    with pytest.raises(ValueError):
+        synth.make_inputs(w, T=4, recipe="nope")
+
+
+def test_stated_recipe_decode_and_recall():
+    w = synth.WORKLOADS["mlp-d128-b4h8-t16k"]
+    a = synth.decode_step_inputs(w, 3, dtype="fp32", recipe="stated")
+    b = synth.decode_step_inputs(w, 3, dtype="fp32", recipe="stated")
+    assert all(torch.equal(a[n], b[n]) for n in a)
+    assert a["k"].shape == (w.decode_B * w.H, w.d)
+    assert float(a["theta"].max()) > 0.09
+    wl = synth.WORKLOADS["mlp-d64-b1h16-t1m"]
+    t = synth.unit_tokens(wl, 2, 0, 2 * synth.RECALL_EVERY, recipe="stated")
+    p = synth.recall_positions(wl, 0, 2 * synth.RECALL_EVERY)
+    assert torch.equal(t["k"][p[0]], t["k"][p[1]]) and torch.equal(t["q"][p[0]], t["k"][p[0]])

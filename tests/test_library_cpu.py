@@ -73,3 +73,13 @@ def test_noalloc_rejects_bad_config_before_cuda():
     rc = L.titans_mem_forward_noalloc(ctypes.byref(cfg), None, None, None, None, None, None, 16, 16, None, None,
                                       None, None, None, None)
     assert rc in (mem.EINVAL, mem.EUNSUPPORTED)
+
+
+def test_noalloc_rejects_too_many_units_before_cuda():
+    """B*H above 2^30 units is refused before the scratch size is computed (it could wrap)."""
+    L = mem.lib()
+    cfg = mem.Config(64, 256, 64, mem.BF16, 1 << 16, 1 << 15, 0)  # 2^31 units
+    rc = L.titans_mem_forward_noalloc(ctypes.byref(cfg), None, None, None, None, None, None, 16, 16, None, None,
+                                      None, None, None, None)
+    assert rc == mem.EINVAL
+    assert "units" in L.titans_last_error_string().decode()

@@ -6,7 +6,7 @@ import pytest
 import torch
 
 import oracle
-from parity import TOL, compare, gpu_inputs, run_gpu, run_oracle, workload_inputs
+from parity import TOL, compare, gpu_inputs, run_gpu, run_oracle, step_sequence, workload_inputs
 from titans_long_term_b200 import mem, synth
 
 pytestmark = pytest.mark.gpu
@@ -74,19 +74,6 @@ def test_mlp128_cuda_cores(mode):
 
 # ---------------------------------------------------------------- decode step
 
-def _step_sequence(m, inp, B, H, steps):
-    toks, gates, state = gpu_inputs(inp, B, H)
-    ys = []
-    for t in range(steps):
-        sl = lambda x: x[:, :, t].contiguous()
-        ys.append(m.step(sl(toks["k"]), sl(toks["q"]), sl(toks["v"]), sl(gates["alpha"]), sl(gates["eta"]),
-                         sl(gates["theta"]), state))
-    m.sync_status()
-    U = B * H
-    y = torch.stack(ys, dim=2).reshape(U, steps, -1).float().cpu().numpy()
-    return y, {n: t.reshape(U, *t.shape[2:]).float().cpu().numpy() for n, t in state.items()}
-
-
 @pytest.mark.parametrize("name,mode", [("mlp-d64-b2h4-t2k", "bf16"), ("mlp-d64-b2h4-t2k", "fp32"),
                                        ("mlp-d128-b4h8-t16k", "bf16"), ("mlp-d128-b4h8-t16k", "fp32"),
                                        ("linear-d64", "fp32")])
@@ -97,7 +84,7 @@ def test_decode_steps(name, mode):
     inp = synth.make_inputs(w, units=range(units), T=12, dtype=mode)
     B, H = (units // 2, 2) if units > 1 else (1, 1)
     m = mem.Memory(w.d, w.h, 1, mode, B, H)
-    gy, gst = _step_sequence(m, inp, B, H, 12)
+    gy, gst = step_sequence(m, inp, B, H, 12)
     ry, rst = run_oracle(inp, 1)
     compare(gy, gst, ry, rst, TOL[mode], what=f"step {name} {mode}")
 

@@ -287,12 +287,20 @@ titans_status_t titans_mem_forward_host(titans_mem_t m, const void* k, const voi
     e = cudaEventRecord(m->ev[0], st);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(m->s_in, m->ev[0], 0);
     if (e != cudaSuccess) return cuda_fail(e, "ordering after the caller's stream");
+    // From the first queued copy on, an error return first makes the caller's stream wait for
+    // everything already queued on the copy streams (best effort), so that a caller who frees or
+    // reuses the buffers once that stream is done cannot race with a copy still in flight.
+    auto settle = [&](titans_status_t status) -> titans_status_t {
+        if (cudaEventRecord(m->ev[0], m->s_in) == cudaSuccess) cudaStreamWaitEvent(st, m->ev[0], 0);
+        if (cudaEventRecord(m->ev[1], m->s_out) == cudaSuccess) cudaStreamWaitEvent(st, m->ev[1], 0);
+        return status;
+    };
     {
         float* dg[3] = {dev->alpha, dev->eta, dev->theta};
         const float* hg[3] = {alpha, eta, theta};
         for (int j = 0; j < 3 && e == cudaSuccess; ++j)
             e = cudaMemcpyAsync(dg[j], hg[j], units * (size_t)T * 4, cudaMemcpyHostToDevice, m->s_in);
-        if (e != cudaSuccess) return cuda_fail(e, "copying the gates in");
+        if (e != cudaSuccess) return settle(cuda_fail(e, "copying the gates in"));
     }
     for (long i = 0; i < nseg; ++i) {
         const long t0 = i * t_seg, tn = std::min(t_seg, T - t0);
@@ -305,21 +313,21 @@ titans_status_t titans_mem_forward_host(titans_mem_t m, const void* k, const voi
                                   units, cudaMemcpyHostToDevice, m->s_in);
         if (e == cudaSuccess) e = cudaEventRecord(m->ev[2 + 2 * i], m->s_in);
         if (e == cudaSuccess) e = cudaStreamWaitEvent(st, m->ev[2 + 2 * i], 0);
-        if (e != cudaSuccess) return cuda_fail(e, "copying a segment in");
+        if (e != cudaSuccess) return settle(cuda_fail(e, "copying a segment in"));
         char* dy = static_cast<char*>(dev->y) + tok_off;
         s = forward_impl(m, dk[0], dk[1], dk[2], dev->alpha + t0, dev->eta + t0, dev->theta + t0, T, tn, chunk, W1,
                          W2, S1, S2, dy, stream);
-        if (s != TITANS_OK) return s;
+        if (s != TITANS_OK) return settle(s);
         e = cudaEventRecord(m->ev[3 + 2 * i], st);
         if (e == cudaSuccess) e = cudaStreamWaitEvent(m->s_out, m->ev[3 + 2 * i], 0);
         if (e == cudaSuccess)
             e = cudaMemcpy2DAsync(static_cast<char*>(y) + (size_t)t0 * d * es, row_h, dy, (size_t)tn * d * es,
                                   (size_t)tn * d * es, units, cudaMemcpyDeviceToHost, m->s_out);
-        if (e != cudaSuccess) return cuda_fail(e, "copying a segment out");
+        if (e != cudaSuccess) return settle(cuda_fail(e, "copying a segment out"));
     }
     e = cudaEventRecord(m->ev[1], m->s_out);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(st, m->ev[1], 0);
-    if (e != cudaSuccess) return cuda_fail(e, "ordering the caller's stream after the copies");
+    if (e != cudaSuccess) return settle(cuda_fail(e, "ordering the caller's stream after the copies"));
     return TITANS_OK;
 }
 

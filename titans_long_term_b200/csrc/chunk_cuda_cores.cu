@@ -197,4 +197,13 @@ cudaError_t launch_chunk_cuda_cores(const ForwardArgs& a, cudaStream_t st) {
     return a.bf16 ? launch_cuda_cores<__nv_bfloat16>(a, st) : launch_cuda_cores<float>(a, st);
 }
 
+// Querying a kernel's attributes makes the runtime load its code on the current device, so
+// that no later launch has to (under lazy module loading the first launch would otherwise).
+cudaError_t preload_chunk_cuda_cores() {
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, chunk_fwd_cuda_cores<float>);
+    if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa, chunk_fwd_cuda_cores<__nv_bfloat16>);
+    return e;
+}
+
 }  // namespace titans

@@ -16,8 +16,10 @@
 //
 // Rules for callers:
 //  - The first call on a device looks up the array's device address there
-//    (cudaGetSymbolAddress, with that device current). Make that first call before any
-//    stream capture that should contain a later call.
+//    (cudaGetSymbolAddress, with that device current) and loads the kernel's code for both
+//    input dtypes (cudaFuncGetAttributes), so that no later call, in either mode, makes the
+//    runtime load code. Make that first call before any stream capture that should contain
+//    a later call.
 //  - All calls share the one array: calls whose kernels overlap on a GPU (different
 //    streams, or host threads) race on it and corrupt each other's results. Serialize them.
 //  - The array keeps the last call's contents; the kernel writes every scratch element of
@@ -50,7 +52,8 @@ titans_status_t fail(titans_status_t s, const std::string& m) {
 
 // Device address of g_noalloc_scratch for the current device. In host code the array's
 // name is a host-side stand-in, not a device address, so it is looked up once per device
-// (with that device current) and cached.
+// (with that device current) and cached. The same first call loads the CUDA-core kernel's
+// fp32- and bf16-input instantiations on that device.
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 float* g_ptr[kMaxDevices] = {};
@@ -64,6 +67,8 @@ cudaError_t scratch_for_current_device(float** out) {
     if (!g_ptr[dev]) {
         void* p = nullptr;
         e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return e;
+        e = preload_chunk_cuda_cores();
         if (e != cudaSuccess) return e;
         g_ptr[dev] = static_cast<float*>(p);
     }
@@ -83,6 +88,7 @@ extern "C" titans_status_t titans_mem_forward_noalloc(const titans_mem_config* c
     using namespace titans;
     if (!cfg) return fail(TITANS_EINVAL, "config is NULL");
     if (cfg->B <= 0 || cfg->H <= 0) return fail(TITANS_EINVAL, "B and H must be positive");
+    if ((long)cfg->B * cfg->H > (1L << 30)) return fail(TITANS_EINVAL, "too many units");
     if (cfg->d != 64 && cfg->d != 128) return fail(TITANS_EUNSUPPORTED, "d must be 64 or 128");
     if (cfg->d_hidden != 0 && cfg->d_hidden != 4 * cfg->d)
         return fail(TITANS_EUNSUPPORTED, "d_hidden must be 0 (linear memory) or 4*d");
@@ -103,6 +109,7 @@ extern "C" titans_status_t titans_mem_forward_noalloc(const titans_mem_config* c
     const long units = (long)cfg->B * cfg->H;
     size_t per_unit = cuda_cores_ws_floats(cfg->d, cfg->d_hidden, chunk);
     per_unit = (per_unit + 63) & ~size_t(63);
+    // units <= 2^30 and per_unit < 2^20 floats, so the product cannot wrap.
     const size_t need = per_unit * sizeof(float) * (size_t)units;
     if (need > kNoallocScratchBytes)
         return fail(TITANS_EUNSUPPORTED, "scratch of " + std::to_string(need) + " bytes (B*H units x chunk) exceeds " +

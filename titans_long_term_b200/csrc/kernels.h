@@ -23,6 +23,8 @@ struct ForwardArgs {
 
 size_t cuda_cores_ws_floats(int d, int h, int n);
 cudaError_t launch_chunk_cuda_cores(const ForwardArgs& a, cudaStream_t st);
+// Loads both instantiations (fp32 and bf16 inputs) of the CUDA-core kernel on the current device.
+cudaError_t preload_chunk_cuda_cores();
 cudaError_t launch_step_cluster(const ForwardArgs& a, cudaStream_t st);
 // Tensor-core chunk kernel (d = 64, h = 256, chunk <= 64, bf16). The tensor maps
 // describe k, q, v as [units][T][64] bf16 with a {64, chunk, 1} box and 128-byte swizzle.
