@@ -19,6 +19,13 @@ Two fp64 paths, both from the pages on "Titans: Learning to Memorize at Test Tim
   per-chunk scalars. It is pinned to :func:`forward` by the tests (1e-12) and
   is used where the token loop would take too long.
 
+* :func:`mag_gate` / :func:`forward_gated` -- the gated output of the
+  memory-as-a-gate architecture (walk-through sec. 4.2 "Gated Memory": o = y
+  (x) M(x~), y the sliding-window attention branch's output; the tencent review's
+  MAG bullet names (x) an element-wise product with a non-linear activation).
+  Reading taken: o_t = attn_t * sigmoid(M(q_t)) element-wise, the logistic
+  function applied to the memory's retrieval, which gates the attention output.
+
 Pins against things other than the oracle itself are in tests/test_oracle_pins.py.
 Parity of the oracle on the full-size workloads is "unpinned" beyond those pins:
 no page prints a worked numerical example.
@@ -192,3 +199,19 @@ def forward_closed_form(k, q, v, alpha, eta, theta, state: Dict, chunk: int, wan
     if not linear:
         st.update(W2=W2, S2=S2)
     return y, st
+
+
+def mag_gate(attn, y):
+    """o = attn * sigmoid(y), element-wise, in fp64: the attention branch's output `attn` gated by
+    the logistic function of the memory's retrieval `y` (walk-through sec. 4.2 "Gated Memory")."""
+    a = np.asarray(attn, np.float64)
+    yy = np.asarray(y, np.float64)
+    with np.errstate(over="ignore"):
+        return a / (1.0 + np.exp(-yy))
+
+
+def forward_gated(k, q, v, alpha, eta, theta, state: Dict, chunk: int, attn, n_threads: int = 0):
+    """The token loop of :func:`forward` with the gated output: returns (o [U, T, d] float64, state),
+    o_t = mag_gate(attn_t, M(q_t)) with M at the chunk-start weights. attn: [U, T, d]."""
+    y, st = forward(k, q, v, alpha, eta, theta, state, chunk, n_threads=n_threads)
+    return mag_gate(_np(attn, np.float32), y), st

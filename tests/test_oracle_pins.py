@@ -62,3 +62,55 @@ def test_chunk_scalars_match_direct_unroll():
         e[j] = 1.0
         W, S = unroll(0.0, 0.0, e)
         assert abs(-W - c[j]) < 1e-14 and abs(-S - dd[j]) < 1e-14
+
+
+# ---------------------------------------------------------------- the memory-as-a-gate output
+
+def _gate_pins(gate):
+    """Pins of o = attn (x) M(x~) read as attn * sigmoid(M): values the definition fixes exactly."""
+    r = np.random.default_rng(5)
+    attn = r.standard_normal((3, 7, 5))
+    y = 3.0 * r.standard_normal((3, 7, 5))
+    # a zero attention branch gives zero output, whatever the memory says
+    assert np.array_equal(gate(np.zeros_like(attn), y), np.zeros_like(attn))
+    # a memory that retrieves exactly zero (e.g. the MLP at its W = 0 fixed point) halves the attention
+    assert np.array_equal(gate(attn, np.zeros_like(y)), attn / 2)
+    # the logistic function's symmetry sigma(-y) = 1 - sigma(y)
+    np.testing.assert_allclose(gate(attn, y) + gate(attn, -y), attn, rtol=0, atol=1e-15)
+    # saturation: a large positive retrieval passes the attention through, a large negative blocks it
+    np.testing.assert_allclose(gate(attn, np.full_like(y, 50.0)), attn, rtol=1e-15)
+    assert np.abs(gate(attn, np.full_like(y, -800.0))).max() == 0.0
+    # element-wise: one element of y moves only the same element of o
+    y2 = y.copy()
+    y2[1, 2, 3] += 1.0
+    diff = gate(attn, y2) != gate(attn, y)
+    assert diff.sum() == 1 and diff[1, 2, 3]
+
+
+def test_mag_gate_pins():
+    _gate_pins(oracle.mag_gate)
+
+
+@pytest.mark.parametrize("name,wrong", [
+    ("gate_the_memory_by_the_attention", lambda a, y: y / (1.0 + np.exp(-a))),
+    ("silu_instead_of_sigmoid", lambda a, y: a * y / (1.0 + np.exp(-y))),
+    ("tanh_instead_of_sigmoid", lambda a, y: a * np.tanh(y)),
+    ("no_activation", lambda a, y: a * y),
+    ("sigmoid_of_minus_y", lambda a, y: a / (1.0 + np.exp(y))),
+])
+def test_mag_gate_pins_reject_plausible_mistakes(name, wrong):
+    with np.errstate(over="ignore"):
+        with pytest.raises(AssertionError):
+            _gate_pins(wrong)
+
+
+def test_gated_forward_after_reset_halves_the_attention():
+    """alpha = 1, eta = 0, theta = 0 on the last token of a chunk puts the MLP memory at W = 0, its
+    fixed point: every later retrieval is exactly 0, so every later gated output is attn / 2."""
+    k, q, v, al, et, th, st = _mk(2, 40, 6, 12, 77)
+    al[:, 15], et[:, 15], th[:, 15] = 1.0, 0.0, 0.0
+    attn = np.random.default_rng(3).standard_normal((2, 40, 6)).astype(np.float32)
+    o, _ = oracle.forward_gated(k, q, v, al, et, th, st, 8, attn)
+    assert np.array_equal(o[:, 16:], attn[:, 16:].astype(np.float64) / 2)
+    y, _ = oracle.forward(k, q, v, al, et, th, st, 8)
+    assert np.abs(o[:, :16] - oracle.mag_gate(attn[:, :16], y[:, :16])).max() == 0.0
