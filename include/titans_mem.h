@@ -109,6 +109,24 @@ titans_status_t titans_mem_forward(titans_mem_t m, const void *k, const void *q,
                                    long T, int chunk, float *W1, float *W2, float *S1, float *S2,
                                    void *y, void *stream);
 
+/*
+ * titans_mem_forward with the memory-as-a-gate output in place of y:
+ *   o_t = attn_t * sigmoid(M(q_t)), element-wise,
+ * where attn [B, H, T, d] (dtype of k, 16-byte aligned, read only) is the output of the
+ * layer's attention branch, computed by the caller, and M(q_t) is the retrieval that
+ * titans_mem_forward writes as y. The update of the state is unchanged.
+ * Defined by the walk-through's sec. 4.2 "Gated Memory" (o = y (x) M(x~), y the sliding-window
+ * attention output) with the tencent review's MAG bullet (the combination is an element-wise
+ * product with a non-linear activation); the reading taken is the logistic function of the
+ * memory's retrieval gating the attention output. The gate is fused into the kernels' output
+ * stores: o costs no extra pass over memory beyond reading attn.
+ * Returns what titans_mem_forward returns, and TITANS_EINVAL for a NULL or misaligned attn.
+ */
+titans_status_t titans_mem_forward_gated(titans_mem_t m, const void *k, const void *q, const void *v,
+                                         const float *alpha, const float *eta, const float *theta,
+                                         long T, int chunk, float *W1, float *W2, float *S1, float *S2,
+                                         const void *attn, void *o, void *stream);
+
 /* Device buffers that titans_mem_forward_host stages through, each the size of the host
  * array of the same name ([B, H, T, d] for k, q, v, y; [B, H, T] for the gates). The call
  * overwrites them; their contents afterwards are unspecified (segment-major layout). */
@@ -158,6 +176,13 @@ titans_status_t titans_mem_forward_host(titans_mem_t m, const void *k, const voi
 titans_status_t titans_mem_step(titans_mem_t m, const void *k, const void *q, const void *v,
                                 const float *alpha, const float *eta, const float *theta,
                                 float *W1, float *W2, float *S1, float *S2, void *y, void *stream);
+
+/* titans_mem_step with the memory-as-a-gate output o = attn * sigmoid(M(q; W_{t-1})) in place of
+ * y; attn [B, H, d] in the dtype of k, 16-byte aligned (see titans_mem_forward_gated). */
+titans_status_t titans_mem_step_gated(titans_mem_t m, const void *k, const void *q, const void *v,
+                                      const float *alpha, const float *eta, const float *theta,
+                                      float *W1, float *W2, float *S1, float *S2, const void *attn,
+                                      void *o, void *stream);
 
 /*
  * Chunk-wise forward that allocates no device memory, for callers that cannot call

@@ -205,10 +205,11 @@ namespace {
 // path reads the segments' gates in place from the full [units][T_total] arrays.
 titans_status_t forward_impl(titans_mem_t m, const void* k, const void* q, const void* v, const float* alpha,
                              const float* eta, const float* theta, long gate_ld, long T, int chunk, float* W1,
-                             float* W2, float* S1, float* S2, void* y, void* stream) {
+                             float* W2, float* S1, float* S2, void* y, void* stream, const void* attn = nullptr) {
     if (!m) return fail(TITANS_EINVAL, "handle is NULL");
     titans_status_t s = check_ptrs(m, k, q, v, alpha, eta, theta, W1, W2, S1, S2, y);
     if (s != TITANS_OK) return s;
+    if (attn && !aligned16(attn)) return fail(TITANS_EINVAL, "attn is not 16-byte aligned");
     if (T < 1) return fail(TITANS_EINVAL, "T must be >= 1");
     if (T * (long)m->cfg.d >= (1L << 31)) return fail(TITANS_EUNSUPPORTED, "T * d must be below 2^31");
     if (chunk < 1 || chunk > m->cfg.chunk)
@@ -216,6 +217,7 @@ titans_status_t forward_impl(titans_mem_t m, const void* k, const void* q, const
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     titans::ForwardArgs a = make_args(m, k, q, v, alpha, eta, theta, T, chunk, W1, W2, S1, S2, y);
     a.gate_ld = gate_ld;
+    a.attn = attn;
     cudaError_t e;
     if (tc_eligible(m->cfg, chunk)) {
         if (T >= (1L << 31) || a.units >= (1L << 31)) return fail(TITANS_EUNSUPPORTED, "T or units too large");
@@ -239,6 +241,14 @@ titans_status_t titans_mem_forward(titans_mem_t m, const void* k, const void* q,
                                    const float* eta, const float* theta, long T, int chunk, float* W1, float* W2,
                                    float* S1, float* S2, void* y, void* stream) {
     return forward_impl(m, k, q, v, alpha, eta, theta, T, T, chunk, W1, W2, S1, S2, y, stream);
+}
+
+titans_status_t titans_mem_forward_gated(titans_mem_t m, const void* k, const void* q, const void* v,
+                                         const float* alpha, const float* eta, const float* theta, long T, int chunk,
+                                         float* W1, float* W2, float* S1, float* S2, const void* attn, void* o,
+                                         void* stream) {
+    if (!attn) return fail(TITANS_EINVAL, "attn is NULL");
+    return forward_impl(m, k, q, v, alpha, eta, theta, T, T, chunk, W1, W2, S1, S2, o, stream, attn);
 }
 
 titans_status_t titans_mem_forward_host(titans_mem_t m, const void* k, const void* q, const void* v,
@@ -331,17 +341,38 @@ titans_status_t titans_mem_forward_host(titans_mem_t m, const void* k, const voi
     return TITANS_OK;
 }
 
-titans_status_t titans_mem_step(titans_mem_t m, const void* k, const void* q, const void* v, const float* alpha,
-                                const float* eta, const float* theta, float* W1, float* W2, float* S1, float* S2,
-                                void* y, void* stream) {
+}  // extern "C"
+
+namespace {
+titans_status_t step_impl(titans_mem_t m, const void* k, const void* q, const void* v, const float* alpha,
+                          const float* eta, const float* theta, float* W1, float* W2, float* S1, float* S2, void* y,
+                          void* stream, const void* attn) {
     if (!m) return fail(TITANS_EINVAL, "handle is NULL");
     titans_status_t s = check_ptrs(m, k, q, v, alpha, eta, theta, W1, W2, S1, S2, y);
     if (s != TITANS_OK) return s;
+    if (attn && !aligned16(attn)) return fail(TITANS_EINVAL, "attn is not 16-byte aligned");
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     titans::ForwardArgs a = make_args(m, k, q, v, alpha, eta, theta, 1, 1, W1, W2, S1, S2, y);
+    a.attn = attn;
     cudaError_t e = m->cfg.d_hidden ? titans::launch_step_cluster(a, st) : titans::launch_chunk_cuda_cores(a, st);
     if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
     return TITANS_OK;
+}
+}  // namespace
+
+extern "C" {
+
+titans_status_t titans_mem_step(titans_mem_t m, const void* k, const void* q, const void* v, const float* alpha,
+                                const float* eta, const float* theta, float* W1, float* W2, float* S1, float* S2,
+                                void* y, void* stream) {
+    return step_impl(m, k, q, v, alpha, eta, theta, W1, W2, S1, S2, y, stream, nullptr);
+}
+
+titans_status_t titans_mem_step_gated(titans_mem_t m, const void* k, const void* q, const void* v,
+                                      const float* alpha, const float* eta, const float* theta, float* W1, float* W2,
+                                      float* S1, float* S2, const void* attn, void* o, void* stream) {
+    if (!attn) return fail(TITANS_EINVAL, "attn is NULL");
+    return step_impl(m, k, q, v, alpha, eta, theta, W1, W2, S1, S2, o, stream, attn);
 }
 
 titans_status_t titans_mem_sync_status(titans_mem_t m, void* stream) {

@@ -23,6 +23,14 @@ __device__ __forceinline__ float ldin(const __nv_bfloat16* p) { return __bfloat1
 __device__ __forceinline__ void stout(float* p, float v) { *p = v; }
 __device__ __forceinline__ void stout(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
 
+// The retrieval M(q) itself, or the memory-as-a-gate output attn * sigmoid(M(q)) ("Titans",
+// walk-through sec. 4.2 "Gated Memory": the logistic function of the memory's retrieval gates
+// the attention branch's output element-wise).
+template <typename Tin>
+__device__ __forceinline__ float gated(float yq, const Tin* attn, long idx) {
+    return attn ? ldin(attn + idx) * (1.f / (1.f + expf(-yq))) : yq;
+}
+
 constexpr int kCcThreads = 256;
 constexpr int kCcMaxChunk = 128;
 
@@ -37,7 +45,8 @@ __global__ void __launch_bounds__(kCcThreads) chunk_fwd_cuda_cores(
     int d, int h, long T, long gate_ld, int chunk, const Tin* __restrict__ k, const Tin* __restrict__ q,
     const Tin* __restrict__ v, const float* __restrict__ alpha, const float* __restrict__ eta,
     const float* __restrict__ theta, float* __restrict__ W1, float* __restrict__ W2, float* __restrict__ S1,
-    float* __restrict__ S2, Tin* __restrict__ y, float* __restrict__ ws, size_t ws_per_unit) {
+    float* __restrict__ S2, Tin* __restrict__ y, const Tin* __restrict__ attn, float* __restrict__ ws,
+    size_t ws_per_unit) {
     __shared__ float s_alpha[kCcMaxChunk], s_eta[kCcMaxChunk], s_theta[kCcMaxChunk];
     __shared__ float s_c[kCcMaxChunk], s_d[kCcMaxChunk], s_scal[3];
 
@@ -49,6 +58,7 @@ __global__ void __launch_bounds__(kCcThreads) chunk_fwd_cuda_cores(
     q += u * T * d;
     v += u * T * d;
     y += u * T * d;
+    if (attn) attn += u * T * d;
     alpha += u * gate_ld;
     eta += u * gate_ld;
     theta += u * gate_ld;
@@ -103,7 +113,7 @@ __global__ void __launch_bounds__(kCcThreads) chunk_fwd_cuda_cores(
                     yq += w * ldin(Q + (size_t)t * d + m);
                 }
                 G[idx] = 2.f * (yh - ldin(V + idx));
-                stout(y + (t0 + t) * d + i, yq);
+                stout(y + (t0 + t) * d + i, gated(yq, attn, (t0 + t) * d + i));
             }
             __syncthreads();
             for (int idx = tid; idx < d * d; idx += blockDim.x) {
@@ -145,7 +155,7 @@ __global__ void __launch_bounds__(kCcThreads) chunk_fwd_cuda_cores(
                 yq += w * Aq[(size_t)t * h + j];
             }
             G[idx] = 2.f * (yh - ldin(V + idx));
-            stout(y + (t0 + t) * d + i, yq);
+            stout(y + (t0 + t) * d + i, gated(yq, attn, (t0 + t) * d + i));
         }
         __syncthreads();
         for (int idx = tid; idx < n * h; idx += blockDim.x) {
@@ -189,7 +199,7 @@ template <typename Tin>
 cudaError_t launch_cuda_cores(const ForwardArgs& a, cudaStream_t st) {
     chunk_fwd_cuda_cores<Tin><<<(unsigned)a.units, kCcThreads, 0, st>>>(
         a.d, a.h, a.T, a.gate_ld, a.chunk, (const Tin*)a.k, (const Tin*)a.q, (const Tin*)a.v, a.alpha, a.eta, a.theta, a.W1,
-        a.W2, a.S1, a.S2, (Tin*)a.y, a.ws, a.ws_per_unit);
+        a.W2, a.S1, a.S2, (Tin*)a.y, (const Tin*)a.attn, a.ws, a.ws_per_unit);
     return cudaGetLastError();
 }
 

@@ -205,7 +205,8 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ,
     const __grid_constant__ CUtensorMap tmV, const float* __restrict__ alpha, const float* __restrict__ eta,
     const float* __restrict__ theta, float* __restrict__ W1g, float* __restrict__ W2g, float* __restrict__ S1g,
-    float* __restrict__ S2g, __nv_bfloat16* __restrict__ yg, long T, long gate_ld, int chunk, unsigned* status) {
+    float* __restrict__ S2g, __nv_bfloat16* __restrict__ yg, const __nv_bfloat16* __restrict__ attn, long T,
+    long gate_ld, int chunk, unsigned* status) {
     using namespace tc;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -660,7 +661,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
                     tc_fence_before();
                     mbar_arrive(&bars[B_G]);
                 } else {  // query row: y, stored after the arrival (the TMEM reads are what GW waits for)
-                    uint32_t o[16];
+                    float yv[32];
 #pragma unroll
                     for (int hb = 0; hb < 2; ++hb) {
                         const int col0 = 32 * tile + 16 * hb;
@@ -669,16 +670,39 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
                         tmem_ld16(tmem + lane_off + 128 + 64 + col0, r2);
                         tmem_wait_ld();
 #pragma unroll
-                        for (int i = 0; i < 8; ++i)
-                            o[8 * hb + i] = pack_bf16x2(__uint_as_float(r[2 * i]) + __uint_as_float(r2[2 * i]),
-                                                        __uint_as_float(r[2 * i + 1]) + __uint_as_float(r2[2 * i + 1]));
+                        for (int i = 0; i < 16; ++i) yv[16 * hb + i] = __uint_as_float(r[i]) + __uint_as_float(r2[i]);
                     }
                     tc_fence_before();
                     mbar_arrive(&bars[B_G]);
                     if (row - kN < n) {
-                        uint4* dst = reinterpret_cast<uint4*>(yg + ((u * T + t0 + (row - kN)) * kD + 32 * tile));
+                        const long off = (u * T + t0 + (row - kN)) * kD + 32 * tile;
+                        uint4* dst = reinterpret_cast<uint4*>(yg + off);
+                        if (attn == nullptr) {
 #pragma unroll
-                        for (int q4 = 0; q4 < 4; ++q4) dst[q4] = make_uint4(o[4 * q4], o[4 * q4 + 1], o[4 * q4 + 2], o[4 * q4 + 3]);
+                            for (int q4 = 0; q4 < 4; ++q4)
+                                dst[q4] = make_uint4(pack_bf16x2(yv[8 * q4], yv[8 * q4 + 1]),
+                                                     pack_bf16x2(yv[8 * q4 + 2], yv[8 * q4 + 3]),
+                                                     pack_bf16x2(yv[8 * q4 + 4], yv[8 * q4 + 5]),
+                                                     pack_bf16x2(yv[8 * q4 + 6], yv[8 * q4 + 7]));
+                        } else {
+                            // The memory-as-a-gate output attn * sigmoid(y), sigmoid(y) = (1 + tanh(y / 2)) / 2
+                            // ("Titans", walk-through sec. 4.2 "Gated Memory").
+                            const uint4* arow = reinterpret_cast<const uint4*>(attn + off);
+#pragma unroll
+                            for (int q4 = 0; q4 < 4; ++q4) {
+                                const uint4 av = __ldg(arow + q4);
+                                const uint32_t aw[4] = {av.x, av.y, av.z, av.w};
+                                uint32_t ow[4];
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) {
+                                    const float2 a2 = unpack_bf16x2(aw[e]);
+                                    const float y0 = yv[8 * q4 + 2 * e], y1 = yv[8 * q4 + 2 * e + 1];
+                                    ow[e] = pack_bf16x2(a2.x * fmaf(0.5f, tanh_approx(0.5f * y0), 0.5f),
+                                                        a2.y * fmaf(0.5f, tanh_approx(0.5f * y1), 0.5f));
+                                }
+                                dst[q4] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+                            }
+                        }
                     }
                 }
             }
@@ -775,7 +799,8 @@ cudaError_t launch_chunk_tc_mlp64(const ForwardArgs& a, const CUtensorMap& tk, c
         attr_set.fetch_or(bit);
     }
     chunk_fwd_tc_mlp64<<<(unsigned)a.units, tc::kThreads, tc::kSmemBytes, st>>>(
-        tk, tq, tv, a.alpha, a.eta, a.theta, a.W1, a.W2, a.S1, a.S2, (__nv_bfloat16*)a.y, a.T, a.gate_ld, a.chunk, a.status);
+        tk, tq, tv, a.alpha, a.eta, a.theta, a.W1, a.W2, a.S1, a.S2, (__nv_bfloat16*)a.y,
+        (const __nv_bfloat16*)a.attn, a.T, a.gate_ld, a.chunk, a.status);
     return cudaGetLastError();
 }
 

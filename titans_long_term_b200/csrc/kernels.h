@@ -16,6 +16,7 @@ struct ForwardArgs {
     long gate_ld;      // elements between consecutive units' gate rows (T for [B, H, T])
     float *W1, *W2, *S1, *S2;
     void* y;
+    const void* attn;  // NULL: y = M(q); else y = attn * sigmoid(M(q)) (memory-as-a-gate output), dtype of y
     float* ws;         // CUDA-core path workspace
     size_t ws_per_unit;
     unsigned* status;  // device status word

@@ -49,7 +49,7 @@ __global__ void __launch_bounds__(kStepThreads, 2) step_mlp_cluster(
     const Tin* __restrict__ k, const Tin* __restrict__ q, const Tin* __restrict__ v,
     const float* __restrict__ alpha, const float* __restrict__ eta, const float* __restrict__ theta,
     float* __restrict__ W1, float* __restrict__ W2, float* __restrict__ S1, float* __restrict__ S2,
-    Tin* __restrict__ y) {
+    Tin* __restrict__ y, const Tin* __restrict__ attn) {
     constexpr int H = 4 * D;
     constexpr int C = H / kSlice;        // CTAs per unit (cluster size)
     constexpr int MC = D / 32;           // W1 columns per lane
@@ -162,10 +162,12 @@ __global__ void __launch_bounds__(kStepThreads, 2) step_mlp_cluster(
         }
         sG[i] = 2.f * (yh - sv[i]);
         if (r == 0) {
+            // the retrieval, or the memory-as-a-gate output attn * sigmoid(M(q))
+            const float o = attn ? ld1(attn + u * D + i) * (1.f / (1.f + expf(-yq))) : yq;
             if constexpr (sizeof(Tin) == 2)
-                y[u * D + i] = __float2bfloat16_rn(yq);
+                y[u * D + i] = __float2bfloat16_rn(o);
             else
-                y[u * D + i] = yq;
+                y[u * D + i] = o;
         }
     }
     // This CTA is done reading the other slices' partials: arrive now, wait only before
@@ -244,7 +246,7 @@ static cudaError_t launch_step(const ForwardArgs& a, cudaStream_t st) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, step_mlp_cluster<D, Tin>, (const Tin*)a.k, (const Tin*)a.q, (const Tin*)a.v,
-                              a.alpha, a.eta, a.theta, a.W1, a.W2, a.S1, a.S2, (Tin*)a.y);
+                              a.alpha, a.eta, a.theta, a.W1, a.W2, a.S1, a.S2, (Tin*)a.y, (const Tin*)a.attn);
 }
 
 cudaError_t launch_step_cluster(const ForwardArgs& a, cudaStream_t st) {

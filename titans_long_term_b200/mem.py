@@ -23,7 +23,8 @@ PATH_TC_MLP64, PATH_CUDA_CORES, PATH_STEP_CLUSTER = 1, 2, 3
 
 EXPORTED = ["titans_mem_init", "titans_mem_destroy", "titans_mem_forward", "titans_mem_step",
             "titans_mem_path", "titans_mem_sync_status", "titans_last_error_string", "titans_mem_version",
-            "titans_mem_forward_noalloc", "titans_mem_forward_host"]
+            "titans_mem_forward_noalloc", "titans_mem_forward_host", "titans_mem_forward_gated",
+            "titans_mem_step_gated"]
 
 
 class TitansError(RuntimeError):
@@ -62,11 +63,13 @@ def lib():
                                                  vp, vp, vp]
         L.titans_mem_forward_host.argtypes = [vp, vp, vp, vp, vp, vp, vp, l, i, vp, vp, vp, vp, vp,
                                               ctypes.POINTER(DeviceBuffers), l, vp]
+        L.titans_mem_forward_gated.argtypes = [vp, vp, vp, vp, vp, vp, vp, l, i, vp, vp, vp, vp, vp, vp, vp]
+        L.titans_mem_step_gated.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
         L.titans_mem_sync_status.argtypes = [vp, vp]
         L.titans_last_error_string.restype = ctypes.c_char_p
         for f in ("titans_mem_init", "titans_mem_destroy", "titans_mem_forward", "titans_mem_step",
                   "titans_mem_path", "titans_mem_sync_status", "titans_mem_version", "titans_mem_forward_noalloc",
-                  "titans_mem_forward_host"):
+                  "titans_mem_forward_host", "titans_mem_forward_gated", "titans_mem_step_gated"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -138,6 +141,21 @@ class Memory:
                                         _ptr(state["S1"]), _ptr(state.get("S2")), _ptr(y), _stream(stream)))
         return y
 
+    def forward_gated(self, k, q, v, alpha, eta, theta, attn, state: Dict[str, torch.Tensor],
+                      chunk: Optional[int] = None, o: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        """Memory-as-a-gate output: o = attn * sigmoid(M(q)) element-wise, attn [B, H, T, d] in the
+        dtype of k (the attention branch's output); otherwise as forward(). Returns o."""
+        T = k.shape[-2]
+        if o is None:
+            o = torch.empty_like(k)
+        self._check_tensors({"k": k, "q": q, "v": v, "attn": attn}, {"alpha": alpha, "eta": eta, "theta": theta},
+                            state, o, (self.B, self.H, T))
+        _check(lib().titans_mem_forward_gated(self._h, _ptr(k), _ptr(q), _ptr(v), _ptr(alpha), _ptr(eta),
+                                              _ptr(theta), T, chunk or self.chunk, _ptr(state["W1"]),
+                                              _ptr(state.get("W2")), _ptr(state["S1"]), _ptr(state.get("S2")),
+                                              _ptr(attn), _ptr(o), _stream(stream)))
+        return o
+
     def forward_host(self, k, q, v, alpha, eta, theta, state: Dict[str, torch.Tensor], y: torch.Tensor,
                      staging: Dict[str, torch.Tensor], chunk: Optional[int] = None, t_seg: int = 0,
                      stream=None) -> torch.Tensor:
@@ -173,6 +191,18 @@ class Memory:
                                      _ptr(state["W1"]), _ptr(state.get("W2")), _ptr(state["S1"]),
                                      _ptr(state.get("S2")), _ptr(y), _stream(stream)))
         return y
+
+    def step_gated(self, k, q, v, alpha, eta, theta, attn, state: Dict[str, torch.Tensor],
+                   o: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        """One decode token per unit with the memory-as-a-gate output o = attn * sigmoid(M(q)); attn [B, H, d]."""
+        if o is None:
+            o = torch.empty_like(k)
+        self._check_tensors({"k": k, "q": q, "v": v, "attn": attn}, {"alpha": alpha, "eta": eta, "theta": theta},
+                            state, o, (self.B, self.H))
+        _check(lib().titans_mem_step_gated(self._h, _ptr(k), _ptr(q), _ptr(v), _ptr(alpha), _ptr(eta), _ptr(theta),
+                                           _ptr(state["W1"]), _ptr(state.get("W2")), _ptr(state["S1"]),
+                                           _ptr(state.get("S2")), _ptr(attn), _ptr(o), _stream(stream)))
+        return o
 
     def sync_status(self, stream=None):
         _check(lib().titans_mem_sync_status(self._h, _stream(stream)))

@@ -314,3 +314,24 @@ def decode_state_rows(w: Workload) -> np.ndarray:
     rep = w.decode_B // w.B
     u = np.arange(w.decode_B * w.H)
     return (u // w.H // rep) * w.H + (u % w.H)
+
+
+def make_attn(w: Workload, units: Optional[Sequence[int]] = None, T: Optional[int] = None,
+              dtype: Optional[str] = None, t0: int = 0) -> torch.Tensor:
+    """The attention branch's output that a memory-as-a-gate layer multiplies by the gate: [U, T, d]
+    in the input dtype, N(0, 1) elements, from a counter-seeded generator per (unit, 4096-token
+    block), so any unit and token range can be drawn alone. It stands in for a sliding-window
+    attention output, which the memory's caller computes."""
+    units = list(range(w.units)) if units is None else list(units)
+    T = w.T - t0 if T is None else T
+    dtype = w.dtype if dtype is None else dtype
+    rows = []
+    for u in units:
+        parts = []
+        for blk in range(t0 // BLOCK, (t0 + T + BLOCK - 1) // BLOCK):
+            x = torch.randn(BLOCK, w.d, generator=_gen(w.seed, u, blk, 0xA77))
+            lo = max(t0 - blk * BLOCK, 0)
+            hi = min(t0 + T - blk * BLOCK, BLOCK)
+            parts.append(x[lo:hi])
+        rows.append(_cast(torch.cat(parts) if parts else torch.zeros(0, w.d), dtype))
+    return torch.stack(rows)
