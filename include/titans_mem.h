@@ -72,7 +72,8 @@ typedef struct titans_mem *titans_mem_t;
 typedef enum {
     TITANS_PATH_TC_MLP64 = 1,     /* tcgen05 bf16 chunk kernel, d=64, h=256, chunk<=64 */
     TITANS_PATH_CUDA_CORES = 2,   /* CUDA-core fp32 chunk kernel (any supported shape) */
-    TITANS_PATH_STEP_CLUSTER = 3  /* single-token decode, thread-block-cluster kernel (MLP) */
+    TITANS_PATH_STEP_CLUSTER = 3, /* single-token decode, thread-block-cluster kernel (MLP) */
+    TITANS_PATH_TC_PHASED = 4     /* tcgen05 bf16 chunk kernel over all SMs, d=128, h=512, chunk<=128 */
 } titans_path_t;
 
 /* Validates the configuration and allocates the handle, its device status word and

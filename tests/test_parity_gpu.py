@@ -66,7 +66,8 @@ def test_mlp128_cuda_cores(mode):
     """d=128, h=512, chunk=128 (wide memory prefill shape), 4 units, T = 300 (ragged)."""
     w = synth.WORKLOADS["mlp-d128-b4h8-t16k"]
     inp = synth.make_inputs(w, units=range(4), T=300, dtype=mode)
-    m = mem.Memory(128, 512, 128, mode, 2, 2)
+    m = mem.Memory(128, 512, 128, mode, 2, 2, cuda_cores=True)
+    assert m.path(128) == mem.PATH_CUDA_CORES
     gy, gst = run_gpu(m, inp, 2, 2, 128)
     ry, rst = run_oracle(inp, 128)
     compare(gy, gst, ry, rst, TOL[mode], what=f"d128 {mode}")

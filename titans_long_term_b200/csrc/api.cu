@@ -15,7 +15,7 @@
 struct titans_mem {
     titans_mem_config cfg;
     int device;
-    unsigned* status;   // device status word
+    unsigned* status;   // device status word, then the phased kernel's two grid-barrier words
     float* ws;          // CUDA-core path workspace
     size_t ws_per_unit; // floats
     // titans_mem_forward_host: copy streams and events, created on first use.
@@ -68,6 +68,11 @@ bool encode_tokens(CUtensorMap* m, const void* base, long T, long units, int chu
 bool tc_eligible(const titans_mem_config& c, int chunk) {
     return c.mode == TITANS_BF16 && !(c.flags & TITANS_FLAG_CUDA_CORES) && c.d == 64 && c.d_hidden == 256 &&
            chunk >= 1 && chunk <= 64;
+}
+
+bool phased_eligible(const titans_mem_config& c, int chunk) {
+    return c.mode == TITANS_BF16 && !(c.flags & TITANS_FLAG_CUDA_CORES) &&
+           titans::tc_phased_supported(c.d, c.d_hidden, chunk);
 }
 
 titans_status_t check_cfg(const titans_mem_config* c) {
@@ -162,14 +167,16 @@ titans_status_t titans_mem_init(const titans_mem_config* cfg, titans_mem_t* out)
         delete m;
         return cuda_fail(e, "cudaGetDevice");
     }
-    e = cudaMalloc(&m->status, sizeof(unsigned));
-    if (e == cudaSuccess) e = cudaMemset(m->status, 0, sizeof(unsigned));
+    e = cudaMalloc(&m->status, 4 * sizeof(unsigned));
+    if (e == cudaSuccess) e = cudaMemset(m->status, 0, 4 * sizeof(unsigned));
     if (e != cudaSuccess) {
         delete m;
         return cuda_fail(e, "allocating the status word");
     }
     m->ws_per_unit = titans::cuda_cores_ws_floats(cfg->d, cfg->d_hidden, cfg->chunk);
-    m->ws_per_unit = (m->ws_per_unit + 63) & ~size_t(63);
+    if (phased_eligible(*cfg, cfg->chunk))
+        m->ws_per_unit = std::max(m->ws_per_unit, titans::tc_phased_ws_bytes_per_unit() / sizeof(float));
+    m->ws_per_unit = (m->ws_per_unit + 255) & ~size_t(255);  // 1 KiB-aligned unit slices
     e = cudaMalloc(&m->ws, m->ws_per_unit * sizeof(float) * (size_t)cfg->B * cfg->H);
     if (e != cudaSuccess) {
         cudaFree(m->status);
@@ -195,7 +202,8 @@ int titans_mem_path(titans_mem_t m, int chunk, int step) {
     if (!m) return -1;
     if (step) return m->cfg.d_hidden ? TITANS_PATH_STEP_CLUSTER : TITANS_PATH_CUDA_CORES;
     if (chunk < 1 || chunk > m->cfg.chunk) return -1;
-    return tc_eligible(m->cfg, chunk) ? TITANS_PATH_TC_MLP64 : TITANS_PATH_CUDA_CORES;
+    if (tc_eligible(m->cfg, chunk)) return TITANS_PATH_TC_MLP64;
+    return phased_eligible(m->cfg, chunk) ? TITANS_PATH_TC_PHASED : TITANS_PATH_CUDA_CORES;
 }
 
 }  // extern "C"
@@ -226,6 +234,8 @@ titans_status_t forward_impl(titans_mem_t m, const void* k, const void* q, const
             !encode_tokens(&tv, v, T, a.units, chunk))
             return fail(TITANS_ECUDA, "cuTensorMapEncodeTiled failed");
         e = titans::launch_chunk_tc_mlp64(a, tk, tq, tv, st);
+    } else if (phased_eligible(m->cfg, chunk)) {
+        e = titans::launch_chunk_tc_phased(a, m->status + 2, st);
     } else {
         e = titans::launch_chunk_cuda_cores(a, st);
     }
@@ -386,7 +396,8 @@ titans_status_t titans_mem_sync_status(titans_mem_t m, void* stream) {
     if (e != cudaSuccess) return cuda_fail(e, "reading the status word");
     if (h) {
         char buf[128];
-        snprintf(buf, sizeof buf, "device status 0x%x (1: TMA wait timed out, 2: MMA wait timed out)", h);
+        snprintf(buf, sizeof buf,
+                 "device status 0x%x (1: TMA wait timed out, 2: MMA wait timed out, 4: grid barrier timed out)", h);
         return fail(TITANS_EDEVICE, buf);
     }
     return TITANS_OK;

@@ -1,0 +1,640 @@
+// Tensor-core chunk forward for the wide MLP memory M(x) = W2 silu(W1 x), d = 128, h = 512,
+// chunk n <= 128, bf16 operands with fp32 accumulation, fp32 state.
+//
+// Method ("Titans: Learning to Memorize at Test Time", walk-through sec. 3.1-3.2): every token of
+// a chunk takes its gradient of ||M(k) - v||^2 at the chunk-start weights, so the chunk's momentum
+// and forgetting recurrence folds into
+//   W <- A W + sigma S - sum_j c_j g_j,   S <- E S - sum_j d_j g_j,
+// with c_j, d_j, A, E, sigma from a division-free suffix scan of the gates, and the sums of
+// per-token outer products are weighted GEMMs.
+//
+// One unit's state is 1 MiB of fp32 (W1, S1 [512 x 128], W2, S2 [128 x 512]): it does not fit
+// one SM, so this kernel does not keep it on chip. Instead one persistent CTA per SM walks the
+// chunks of every unit together in four phases, each a set of 128-row tcgen05 tiles spread over
+// all SMs, separated by grid-wide barriers:
+//   P1  Z^T [h x tok] = W1 [K; Q]^T (128 hidden rows x 128 tokens per tile) -> silu(Z)^T (bf16)
+//       and silu'(Z_K)^T (fp32); plus, per unit, the gate scan and the scaled key tiles -c K, -d K.
+//   P2  Y [tok x d] = silu(Z) W2^T (128 tokens x 64 columns per tile) -> keys: G = 2 (Y - v) and
+//       its scaled copies -c G, -d G (bf16, each rounded once from fp32); queries: y (or the
+//       gated output attn * sigmoid(y)).
+//   P3  (GW2)^T [h x tok] = W2^T G^T -> Delta^T = (GW2)^T * silu'(Z_K)^T (bf16).
+//   P4  dW1_{c,d} [h x d] = Delta^T diag(-c|-d) K and dW2_{c,d} [d x h] = G^T diag(-c|-d) silu(Z_K),
+//       two TMEM accumulators per tile; the epilogue applies W <- A W + sigma S + dW_c,
+//       S <- E S + dW_d in fp32 and rewrites the bf16 copy of W that the next chunk's MMAs read.
+// The state and the intermediates (about 1 MiB per unit each) stay in L2 between phases. Operand
+// tiles are copied into shared memory with cp.async in the 128-byte swizzled layout the MMA
+// descriptors describe; one thread issues the MMAs, fp32 accumulators live in TMEM, and every
+// thread reads its own TMEM row in the epilogue.
+//
+// The grid barrier spins on a global counter with a 1 s bound; a timeout sets the device status
+// word and a global abort flag that every other CTA sees in its own spin, so all CTAs leave.
+// The kernel is launched cooperatively, which guarantees that all CTAs are resident together.
+#include <cuda_bf16.h>
+
+#include <atomic>
+#include <cstdint>
+
+#include "kernels.h"
+#include "ptx.cuh"
+
+namespace titans {
+
+namespace ph {
+constexpr int kD = 128, kH = 512, kNmax = 128;
+constexpr int kThreads = 256;  // 8 warps: warp w reads TMEM lane quadrant w % 4, column half w / 4
+// Per-unit workspace (bytes), each piece 1024-aligned.
+constexpr size_t W1B = 0;                                  // bf16 [h][d]   copy of W1
+constexpr size_t W2B = W1B + (size_t)kH * kD * 2;          // bf16 [d][h]   copy of W2
+constexpr size_t AT = W2B + (size_t)kD * kH * 2;           // bf16 [h][2 x 128 tok]  silu(Z)^T: keys, then queries
+constexpr size_t SP = AT + (size_t)kH * 256 * 2;           // fp32 [h][128 tok]      silu'(Z_K)^T
+constexpr size_t DT = SP + (size_t)kH * kNmax * 4;         // bf16 [h][128 tok]      Delta^T
+constexpr size_t GG = DT + (size_t)kH * kNmax * 2;         // bf16 [128 tok][d]      G
+constexpr size_t GC = GG + (size_t)kNmax * kD * 2;         // bf16 [128 tok][d]      -c G
+constexpr size_t GD = GC + (size_t)kNmax * kD * 2;         // bf16 [128 tok][d]      -d G
+constexpr size_t KC = GD + (size_t)kNmax * kD * 2;         // bf16 [128 tok][d]      -c K
+constexpr size_t KD = KC + (size_t)kNmax * kD * 2;         // bf16 [128 tok][d]      -d K
+constexpr size_t SC = KD + (size_t)kNmax * kD * 2;         // fp32 c[128], d[128], A, E, sigma
+constexpr size_t kWsBytes = SC + 2048;
+// Shared memory: operand tiles, each [rows][64] bf16 with the 128-byte swizzle.
+constexpr uint32_t kSmemOperands = 192 * 1024;
+constexpr uint32_t BAR = kSmemOperands;       // one mbarrier (MMA completion)
+constexpr uint32_t TPTR = BAR + 8;
+constexpr uint32_t OKF = TPTR + 4;            // the grid barrier's verdict for the CTA
+constexpr uint32_t END = OKF + 4;
+constexpr size_t kSmemBytes = END + 1024;
+constexpr uint32_t kTmemCols = 256;
+constexpr unsigned kStatusTimeoutGrid = 4u;
+}  // namespace ph
+
+static_assert(ph::kSmemBytes <= 232448, "shared memory budget");
+
+struct PhasedArgs {
+    const __nv_bfloat16 *k, *q, *v;
+    const float *alpha, *eta, *theta;
+    float *W1, *W2, *S1, *S2;
+    __nv_bfloat16* y;
+    const __nv_bfloat16* attn;
+    uint8_t* ws;
+    size_t ws_stride;  // bytes per unit
+    long T, gate_ld;
+    int chunk, units;
+    unsigned* status;
+    unsigned* sync;    // [0] barrier arrivals, [1] abort flag; zero at launch
+};
+
+namespace {
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;" ::: "memory");
+}
+
+// Copies `rows` rows of 64 bf16 (128 B) into a swizzled [rows][64] tile at shared address `tile`:
+// row r comes from src + r * stride (bytes). Rows r >= valid are zero.
+__device__ __forceinline__ void load_tile(uint32_t tile, const uint8_t* src, size_t stride, int rows, int valid) {
+    for (int i = threadIdx.x; i < rows * 8; i += ph::kThreads) {
+        const int r = i >> 3, c16 = i & 7;
+        const uint32_t dst = tile + (uint32_t)r * 128u + ((uint32_t)(c16 ^ (r & 7)) << 4);
+        if (r < valid)
+            cp_async16(dst, src + (size_t)r * stride + (size_t)c16 * 16);
+        else
+            st_shared_v4(dst, 0u, 0u, 0u, 0u);
+    }
+}
+
+// All operand copies of the tile have landed and are visible to the tensor core.
+__device__ __forceinline__ void operands_ready() {
+    cp_async_wait_all();
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+}
+
+__device__ __forceinline__ uint32_t pack2(float a, float b) { return pack_bf16x2(a, b); }
+
+// Grid-wide barrier with a bounded spin. Returns false if any CTA gave up (timeout anywhere).
+__device__ bool grid_sync(const PhasedArgs& a, unsigned& epoch, volatile uint32_t* s_ok) {
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        ++epoch;
+        bool ok = true;
+        __threadfence();
+        atomicAdd(&a.sync[0], 1u);
+        const unsigned target = epoch * gridDim.x;
+        const unsigned long long t0 = globaltimer_ns();
+        while (true) {
+            unsigned v;
+            asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(&a.sync[0]) : "memory");
+            if (v >= target) break;
+            unsigned ab;
+            asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(ab) : "l"(&a.sync[1]) : "memory");
+            if (ab) {
+                ok = false;
+                break;
+            }
+            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                atomicOr(a.status, ph::kStatusTimeoutGrid);
+                atomicExch(&a.sync[1], 1u);
+                ok = false;
+                break;
+            }
+        }
+        __threadfence();
+        *s_ok = ok ? 1u : 0u;
+    }
+    __syncthreads();
+    return *s_ok != 0;
+}
+
+}  // namespace
+
+__global__ void __launch_bounds__(ph::kThreads, 1) chunk_fwd_tc_phased(const __grid_constant__ PhasedArgs a) {
+    using namespace ph;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sb = smem_u32(sm);
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + BAR);
+    volatile uint32_t* s_ok = reinterpret_cast<volatile uint32_t*>(sm + OKF);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quad = warp & 3, half = warp >> 2;
+    const uint32_t lane_off = (uint32_t)(32 * quad) << 16;
+    const int row = 32 * quad + lane;  // this thread's TMEM lane = tile row
+
+    if (tid == 0) {
+        mbar_init(bar, 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(reinterpret_cast<uint32_t*>(sm + TPTR), kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sm + TPTR);
+    unsigned epoch = 0;
+    uint32_t mma_phase = 0;
+    bool ok = true;
+
+    // Issue on one thread, wait on all: the tile's MMAs are complete and TMEM is readable. The
+    // verdict is the same for every thread of the CTA (a timeout anywhere counts for all).
+    auto mma_done = [&]() -> bool {
+        if (tid == 0) umma_commit(bar);
+        const bool done = mbar_wait(bar, mma_phase);
+        mma_phase ^= 1u;
+        if (!done) {
+            atomicOr(a.status, kStatusTimeoutMma);
+            atomicExch(&a.sync[1], 1u);
+        }
+        const bool all = __syncthreads_or(!done) == 0;
+        tc_fence_after();
+        return all;
+    };
+    auto unit_ws = [&](int u) { return a.ws + (size_t)u * a.ws_stride; };
+
+    const int units = a.units;
+    const long T = a.T;
+    const int nchunks = (int)((T + a.chunk - 1) / a.chunk);
+
+    // ---- prologue: bf16 copies of the initial weights
+    for (long i = (long)blockIdx.x * kThreads + tid; i < (long)units * kH * kD / 4; i += (long)gridDim.x * kThreads) {
+        const long e = 4 * i;
+        const int u = (int)(e / (kH * kD));
+        const long r = e % (kH * kD);
+        const float4 w1 = __ldcg(reinterpret_cast<const float4*>(a.W1 + e));
+        const float4 w2 = __ldcg(reinterpret_cast<const float4*>(a.W2 + e));
+        uint2* d1 = reinterpret_cast<uint2*>(unit_ws(u) + W1B + 2 * r);
+        uint2* d2 = reinterpret_cast<uint2*>(unit_ws(u) + W2B + 2 * r);
+        __stcg(d1, make_uint2(pack2(w1.x, w1.y), pack2(w1.z, w1.w)));
+        __stcg(d2, make_uint2(pack2(w2.x, w2.y), pack2(w2.z, w2.w)));
+    }
+    ok = grid_sync(a, epoch, s_ok);
+
+    for (int c = 0; c < nchunks && ok; ++c) {
+        const long t0 = (long)c * a.chunk;
+        const int n = (int)min((long)a.chunk, T - t0);
+
+        // ================= P1: Z^T tiles (unit, 128 hidden rows, keys | queries) and gate scans
+        const int p1_gemm = units * 8;
+        for (int tile = blockIdx.x; tile < p1_gemm + units && ok; tile += gridDim.x) {
+            if (tile >= p1_gemm) {
+                // Gate scan of the chunk (sequential suffix scan, division-free) and the scaled keys.
+                const int u = tile - p1_gemm;
+                uint8_t* w = unit_ws(u);
+                float* s_c = reinterpret_cast<float*>(sm);  // shared scratch: c[128], d[128], A, E, sigma
+                float* s_d = s_c + 128;
+                if (tid == 0) {
+                    const float* al = a.alpha + (long)u * a.gate_ld + t0;
+                    const float* et = a.eta + (long)u * a.gate_ld + t0;
+                    const float* th = a.theta + (long)u * a.gate_ld + t0;
+                    float Pr = 1.f, Qr = 1.f, r_next = 0.f;
+                    for (int j = kNmax - 1; j >= n; --j) s_c[j] = s_d[j] = 0.f;
+                    for (int j = n - 1; j >= 0; --j) {
+                        // r_j = P_j + eta_{j+1} r_{j+1}, P_j = prod_{l>j} (1 - alpha_l), Q_j = prod_{l>j} eta_l
+                        const float r = Pr + (j + 1 < n ? __ldg(et + j + 1) * r_next : 0.f);
+                        const float thj = __ldg(th + j);
+                        s_c[j] = thj * r;
+                        s_d[j] = thj * Qr;
+                        r_next = r;
+                        Pr *= 1.f - __ldg(al + j);
+                        Qr *= __ldg(et + j);
+                    }
+                    s_c[256] = Pr;                      // A = prod (1 - alpha)
+                    s_c[257] = Qr;                      // E = prod eta
+                    s_c[258] = __ldg(et) * r_next;      // sigma = eta_0 r_0
+                }
+                __syncthreads();
+                float* gsc = reinterpret_cast<float*>(w + SC);
+                for (int i = tid; i < 259; i += kThreads) __stcg(gsc + i, s_c[i]);
+                // -c_j K_j and -d_j K_j, bf16 [128 tok][d]; rows j >= n are zero
+                const __nv_bfloat16* K = a.k + ((long)u * T + t0) * kD;
+                for (int i = tid; i < kNmax * kD / 8; i += kThreads) {
+                    const int j = i / (kD / 8), c8 = i % (kD / 8);
+                    uint4 oc = make_uint4(0, 0, 0, 0), od = oc;
+                    if (j < n) {
+                        const uint4 kv = __ldg(reinterpret_cast<const uint4*>(K + (long)j * kD) + c8);
+                        const uint32_t kin[4] = {kv.x, kv.y, kv.z, kv.w};
+                        uint32_t pc[4], pd[4];
+                        const float cj = -s_c[j], dj = -s_d[j];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 f = unpack_bf16x2(kin[e]);
+                            pc[e] = pack2(cj * f.x, cj * f.y);
+                            pd[e] = pack2(dj * f.x, dj * f.y);
+                        }
+                        oc = make_uint4(pc[0], pc[1], pc[2], pc[3]);
+                        od = make_uint4(pd[0], pd[1], pd[2], pd[3]);
+                    }
+                    __stcg(reinterpret_cast<uint4*>(w + KC) + i, oc);
+                    __stcg(reinterpret_cast<uint4*>(w + KD) + i, od);
+                }
+                __syncthreads();
+                continue;
+            }
+            const int u = tile >> 3, mt = (tile >> 1) & 3, part = tile & 1;  // part 0: keys, 1: queries
+            uint8_t* w = unit_ws(u);
+            const __nv_bfloat16* X = (part ? a.q : a.k) + ((long)u * T + t0) * kD;
+            // A = W1 rows [mt*128, +128) (K-major, two 64-column blocks), B = the chunk's tokens.
+            tc_fence_before();
+            __syncthreads();
+            for (int kb = 0; kb < 2; ++kb) {
+                load_tile(sb + kb * 16384, w + W1B + ((size_t)mt * 128 * kD + kb * 64) * 2, kD * 2, 128, 128);
+                load_tile(sb + 32768 + kb * 16384, reinterpret_cast<const uint8_t*>(X + kb * 64), kD * 2, 128, n);
+            }
+            operands_ready();
+            if (tid == 0) {
+                const uint32_t id = idesc_bf16_f32(128, 128, 0, 0);
+                for (int kb = 0; kb < 2; ++kb)
+                    for (int ks = 0; ks < 4; ++ks)
+                        umma_bf16(tmem, sdesc_sw128(sb + kb * 16384 + ks * 32, 16, 1024),
+                                  sdesc_sw128(sb + 32768 + kb * 16384 + ks * 32, 16, 1024), id, (kb | ks) != 0);
+            }
+            if (!mma_done()) {
+                ok = false;
+                break;
+            }
+            // Epilogue: hidden row h = mt*128 + row, tokens [64 half, +64).
+            const int h = mt * 128 + row;
+            uint8_t* at_row = w + AT + ((size_t)h * 256 + part * 128 + 64 * half) * 2;
+            float* sp_row = reinterpret_cast<float*>(w + SP) + (size_t)h * kNmax + 64 * half;
+#pragma unroll 1
+            for (int blk = 0; blk < 4; ++blk) {
+                uint32_t r[16];
+                tmem_ld16(tmem + lane_off + 64 * half + 16 * blk, r);
+                tmem_wait_ld();
+                uint32_t pk[8];
+                float spv[16];
+#pragma unroll
+                for (int i = 0; i < 16; i += 2) {
+                    const float z0 = __uint_as_float(r[i]), z1 = __uint_as_float(r[i + 1]);
+                    const float s0 = 1.f / (1.f + __expf(-z0)), s1 = 1.f / (1.f + __expf(-z1));
+                    const float a0 = z0 * s0, a1 = z1 * s1;
+                    pk[i / 2] = pack2(a0, a1);
+                    spv[i] = s0 + a0 * (1.f - s0);  // silu'(z) = sigma + silu (1 - sigma)
+                    spv[i + 1] = s1 + a1 * (1.f - s1);
+                }
+                uint4* dst = reinterpret_cast<uint4*>(at_row + 32 * blk);
+                __stcg(dst, make_uint4(pk[0], pk[1], pk[2], pk[3]));
+                __stcg(dst + 1, make_uint4(pk[4], pk[5], pk[6], pk[7]));
+                if (part == 0) {
+                    float4* sd = reinterpret_cast<float4*>(sp_row + 16 * blk);
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4)
+                        __stcg(sd + q4, make_float4(spv[4 * q4], spv[4 * q4 + 1], spv[4 * q4 + 2], spv[4 * q4 + 3]));
+                }
+            }
+        }
+        if (!grid_sync(a, epoch, s_ok) || !ok) {
+            ok = false;
+            break;
+        }
+
+        // ================= P2: Y tiles (unit, keys | queries, 64 output columns)
+        for (int tile = blockIdx.x; tile < units * 4 && ok; tile += gridDim.x) {
+            const int u = tile >> 2, part = (tile >> 1) & 1, nh = tile & 1;
+            uint8_t* w = unit_ws(u);
+            tc_fence_before();
+            __syncthreads();
+            // A = silu(Z) [tok x h] from silu(Z)^T (MN-major): per 64-hidden block kb two 64-token
+            // blocks 8 KB apart; B = W2 rows [nh*64, +64) (K-major: the hidden index is contiguous).
+            for (int kb = 0; kb < 8; ++kb) {
+                for (int mb = 0; mb < 2; ++mb)
+                    load_tile(sb + kb * 16384 + mb * 8192, w + AT + ((size_t)kb * 64 * 256 + part * 128 + mb * 64) * 2,
+                              256 * 2, 64, 64);
+                load_tile(sb + 131072 + kb * 8192, w + W2B + ((size_t)nh * 64 * kH + kb * 64) * 2, kH * 2, 64, 64);
+            }
+            operands_ready();
+            if (tid == 0) {
+                const uint32_t id = idesc_bf16_f32(128, 64, 1, 0);
+                for (int kb = 0; kb < 8; ++kb)
+                    for (int ks = 0; ks < 4; ++ks)
+                        umma_bf16(tmem, sdesc_sw128(sb + kb * 16384 + ks * 2048, 8192, 1024),
+                                  sdesc_sw128(sb + 131072 + kb * 8192 + ks * 32, 16, 1024), id, (kb | ks) != 0);
+            }
+            if (!mma_done()) {
+                ok = false;
+                break;
+            }
+            // Epilogue: token row `row`, output columns nh*64 + 32 half + [0, 32).
+            const int col0 = nh * 64 + 32 * half;
+            float yv[32];
+#pragma unroll
+            for (int b = 0; b < 2; ++b) {
+                uint32_t r[16];
+                tmem_ld16(tmem + lane_off + 32 * half + 16 * b, r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 16; ++i) yv[16 * b + i] = __uint_as_float(r[i]);
+            }
+            if (part == 0) {
+                const float* gsc = reinterpret_cast<const float*>(w + SC);
+                const float cr = -__ldcg(gsc + row), dr = -__ldcg(gsc + 128 + row);
+                const bool valid = row < n;
+                const uint4* vrow = reinterpret_cast<const uint4*>(a.v + ((long)u * T + t0 + row) * kD + col0);
+                const size_t off = ((size_t)row * kD + col0) * 2;
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    uint32_t og[4] = {0, 0, 0, 0}, oc[4] = {0, 0, 0, 0}, od[4] = {0, 0, 0, 0};
+                    if (valid) {
+                        const uint4 vv = __ldg(vrow + q4);
+                        const uint32_t vin[4] = {vv.x, vv.y, vv.z, vv.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 vf = unpack_bf16x2(vin[e]);
+                            const float g0 = 2.f * (yv[8 * q4 + 2 * e] - vf.x), g1 = 2.f * (yv[8 * q4 + 2 * e + 1] - vf.y);
+                            og[e] = pack2(g0, g1);
+                            oc[e] = pack2(cr * g0, cr * g1);
+                            od[e] = pack2(dr * g0, dr * g1);
+                        }
+                    }
+                    __stcg(reinterpret_cast<uint4*>(w + GG + off) + q4, make_uint4(og[0], og[1], og[2], og[3]));
+                    __stcg(reinterpret_cast<uint4*>(w + GC + off) + q4, make_uint4(oc[0], oc[1], oc[2], oc[3]));
+                    __stcg(reinterpret_cast<uint4*>(w + GD + off) + q4, make_uint4(od[0], od[1], od[2], od[3]));
+                }
+            } else if (row < n) {
+                const long off = ((long)u * T + t0 + row) * kD + col0;
+                uint4* dst = reinterpret_cast<uint4*>(a.y + off);
+                const uint4* arow = a.attn ? reinterpret_cast<const uint4*>(a.attn + off) : nullptr;
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    uint32_t o[4];
+                    uint4 av = make_uint4(0, 0, 0, 0);
+                    if (arow) av = __ldg(arow + q4);
+                    const uint32_t aw[4] = {av.x, av.y, av.z, av.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        float y0 = yv[8 * q4 + 2 * e], y1 = yv[8 * q4 + 2 * e + 1];
+                        if (arow) {  // memory-as-a-gate output attn * sigmoid(y) (walk-through sec. 4.2)
+                            const float2 a2 = unpack_bf16x2(aw[e]);
+                            y0 = a2.x / (1.f + __expf(-y0));
+                            y1 = a2.y / (1.f + __expf(-y1));
+                        }
+                        o[e] = pack2(y0, y1);
+                    }
+                    dst[q4] = make_uint4(o[0], o[1], o[2], o[3]);
+                }
+            }
+        }
+        if (!grid_sync(a, epoch, s_ok) || !ok) {
+            ok = false;
+            break;
+        }
+
+        // ================= P3: (GW2)^T tiles (unit, 128 hidden rows) -> Delta^T
+        for (int tile = blockIdx.x; tile < units * 4 && ok; tile += gridDim.x) {
+            const int u = tile >> 2, mt = tile & 3;
+            uint8_t* w = unit_ws(u);
+            tc_fence_before();
+            __syncthreads();
+            // A = W2^T rows [mt*128, +128) from W2 [d][h] (MN-major: per 64-column block kb of d, two
+            // 64-hidden blocks 8 KB apart); B = G [tok][d] (K-major).
+            for (int kb = 0; kb < 2; ++kb) {
+                for (int mb = 0; mb < 2; ++mb)
+                    load_tile(sb + kb * 16384 + mb * 8192, w + W2B + ((size_t)kb * 64 * kH + mt * 128 + mb * 64) * 2,
+                              kH * 2, 64, 64);
+                load_tile(sb + 32768 + kb * 16384, w + GG + (size_t)kb * 64 * 2, kD * 2, 128, 128);
+            }
+            operands_ready();
+            if (tid == 0) {
+                const uint32_t id = idesc_bf16_f32(128, 128, 1, 0);
+                for (int kb = 0; kb < 2; ++kb)
+                    for (int ks = 0; ks < 4; ++ks)
+                        umma_bf16(tmem, sdesc_sw128(sb + kb * 16384 + ks * 2048, 8192, 1024),
+                                  sdesc_sw128(sb + 32768 + kb * 16384 + ks * 32, 16, 1024), id, (kb | ks) != 0);
+            }
+            if (!mma_done()) {
+                ok = false;
+                break;
+            }
+            const int h = mt * 128 + row;
+            const float* sp_row = reinterpret_cast<const float*>(w + SP) + (size_t)h * kNmax + 64 * half;
+            uint8_t* dt_row = w + DT + ((size_t)h * kNmax + 64 * half) * 2;
+#pragma unroll 1
+            for (int blk = 0; blk < 4; ++blk) {
+                uint32_t r[16];
+                tmem_ld16(tmem + lane_off + 64 * half + 16 * blk, r);
+                tmem_wait_ld();
+                uint32_t pk[8];
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    const float4 s = __ldcg(reinterpret_cast<const float4*>(sp_row + 16 * blk) + q4);
+                    pk[2 * q4] = pack2(__uint_as_float(r[4 * q4]) * s.x, __uint_as_float(r[4 * q4 + 1]) * s.y);
+                    pk[2 * q4 + 1] = pack2(__uint_as_float(r[4 * q4 + 2]) * s.z, __uint_as_float(r[4 * q4 + 3]) * s.w);
+                }
+                uint4* dst = reinterpret_cast<uint4*>(dt_row + 32 * blk);
+                __stcg(dst, make_uint4(pk[0], pk[1], pk[2], pk[3]));
+                __stcg(dst + 1, make_uint4(pk[4], pk[5], pk[6], pk[7]));
+            }
+        }
+        if (!grid_sync(a, epoch, s_ok) || !ok) {
+            ok = false;
+            break;
+        }
+
+        // ================= P4: weight GEMMs and the state update (unit, W1 | W2, 128-row block)
+        for (int tile = blockIdx.x; tile < units * 8 && ok; tile += gridDim.x) {
+            const int u = tile >> 3, which = (tile >> 2) & 1, mt = tile & 3;
+            uint8_t* w = unit_ws(u);
+            tc_fence_before();
+            __syncthreads();
+            const uint32_t A0 = sb, B0 = sb + 32768, C0 = sb + 65536;  // A | B c-part | B d-part (or A c/d, B)
+            if (which == 0) {
+                // dW1_{c,d} [h x d] = Delta^T (K-major [h][tok]) x diag(-c|-d) K (MN-major [tok][d]).
+                for (int kb = 0; kb < 2; ++kb) {
+                    load_tile(A0 + kb * 16384, w + DT + ((size_t)mt * 128 * kNmax + kb * 64) * 2, kNmax * 2, 128, 128);
+                    for (int mb = 0; mb < 2; ++mb) {
+                        load_tile(B0 + kb * 16384 + mb * 8192, w + KC + ((size_t)kb * 64 * kD + mb * 64) * 2, kD * 2,
+                                  64, 64);
+                        load_tile(C0 + kb * 16384 + mb * 8192, w + KD + ((size_t)kb * 64 * kD + mb * 64) * 2, kD * 2,
+                                  64, 64);
+                    }
+                }
+            } else {
+                // dW2_{c,d} [d x h] = (diag(-c|-d) G)^T (MN-major [tok][d]) x silu(Z_K) (K-major [h][tok]).
+                for (int kb = 0; kb < 2; ++kb) {
+                    for (int mb = 0; mb < 2; ++mb) {
+                        load_tile(A0 + kb * 16384 + mb * 8192, w + GC + ((size_t)kb * 64 * kD + mb * 64) * 2, kD * 2,
+                                  64, 64);
+                        load_tile(C0 + kb * 16384 + mb * 8192, w + GD + ((size_t)kb * 64 * kD + mb * 64) * 2, kD * 2,
+                                  64, 64);
+                    }
+                    load_tile(B0 + kb * 16384, w + AT + ((size_t)mt * 128 * 256 + kb * 64) * 2, 256 * 2, 128, 128);
+                }
+            }
+            operands_ready();
+            if (tid == 0) {
+                for (int kb = 0; kb < 2; ++kb)
+                    for (int ks = 0; ks < 4; ++ks) {
+                        const uint32_t acc = (kb | ks) != 0;
+                        if (which == 0) {
+                            const uint32_t id = idesc_bf16_f32(128, 128, 0, 1);
+                            const uint64_t da = sdesc_sw128(A0 + kb * 16384 + ks * 32, 16, 1024);
+                            umma_bf16(tmem, da, sdesc_sw128(B0 + kb * 16384 + ks * 2048, 8192, 1024), id, acc);
+                            umma_bf16(tmem + 128, da, sdesc_sw128(C0 + kb * 16384 + ks * 2048, 8192, 1024), id, acc);
+                        } else {
+                            const uint32_t id = idesc_bf16_f32(128, 128, 1, 0);
+                            const uint64_t db = sdesc_sw128(B0 + kb * 16384 + ks * 32, 16, 1024);
+                            umma_bf16(tmem, sdesc_sw128(A0 + kb * 16384 + ks * 2048, 8192, 1024), db, id, acc);
+                            umma_bf16(tmem + 128, sdesc_sw128(C0 + kb * 16384 + ks * 2048, 8192, 1024), db, id, acc);
+                        }
+                    }
+            }
+            if (!mma_done()) {
+                ok = false;
+                break;
+            }
+            // Epilogue: W <- A W + sigma S + dW_c, S <- E S + dW_d for this thread's row of the block.
+            const float* gsc = reinterpret_cast<const float*>(w + SC);
+            const float An = __ldcg(gsc + 256), En = __ldcg(gsc + 257), sig = __ldcg(gsc + 258);
+            float *Wr, *Sr;
+            uint8_t* Wb;
+            if (which == 0) {  // W1 row h, columns [64 half, +64)
+                const size_t e0 = ((size_t)u * kH + mt * 128 + row) * kD + 64 * half;
+                Wr = a.W1 + e0;
+                Sr = a.S1 + e0;
+                Wb = w + W1B + (((size_t)mt * 128 + row) * kD + 64 * half) * 2;
+            } else {  // W2 row i (of d), hidden columns mt*128 + [64 half, +64)
+                const size_t e0 = ((size_t)u * kD + row) * kH + mt * 128 + 64 * half;
+                Wr = a.W2 + e0;
+                Sr = a.S2 + e0;
+                Wb = w + W2B + ((size_t)row * kH + mt * 128 + 64 * half) * 2;
+            }
+#pragma unroll 1
+            for (int blk = 0; blk < 4; ++blk) {
+                uint32_t rc[16], rd[16];
+                tmem_ld16(tmem + lane_off + 64 * half + 16 * blk, rc);
+                tmem_ld16(tmem + lane_off + 128 + 64 * half + 16 * blk, rd);
+                tmem_wait_ld();
+                uint32_t pk[8];
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    float4 wv = __ldcg(reinterpret_cast<const float4*>(Wr + 16 * blk) + q4);
+                    float4 sv = __ldcg(reinterpret_cast<const float4*>(Sr + 16 * blk) + q4);
+                    float wn[4] = {wv.x, wv.y, wv.z, wv.w}, sn[4] = {sv.x, sv.y, sv.z, sv.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float wo = wn[e], so = sn[e];
+                        wn[e] = fmaf(An, wo, sig * so) + __uint_as_float(rc[4 * q4 + e]);
+                        sn[e] = fmaf(En, so, __uint_as_float(rd[4 * q4 + e]));
+                    }
+                    __stcg(reinterpret_cast<float4*>(Wr + 16 * blk) + q4, make_float4(wn[0], wn[1], wn[2], wn[3]));
+                    __stcg(reinterpret_cast<float4*>(Sr + 16 * blk) + q4, make_float4(sn[0], sn[1], sn[2], sn[3]));
+                    pk[2 * q4] = pack2(wn[0], wn[1]);
+                    pk[2 * q4 + 1] = pack2(wn[2], wn[3]);
+                }
+                uint4* dst = reinterpret_cast<uint4*>(Wb + 32 * blk);
+                __stcg(dst, make_uint4(pk[0], pk[1], pk[2], pk[3]));
+                __stcg(dst + 1, make_uint4(pk[4], pk[5], pk[6], pk[7]));
+            }
+        }
+        if (!grid_sync(a, epoch, s_ok) || !ok) {
+            ok = false;
+            break;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+size_t tc_phased_ws_bytes_per_unit() { return ph::kWsBytes; }
+
+bool tc_phased_supported(int d, int h, int chunk) { return d == 128 && h == 512 && chunk >= 1 && chunk <= 128; }
+
+cudaError_t launch_chunk_tc_phased(const ForwardArgs& f, unsigned* sync, cudaStream_t st) {
+    static std::atomic<unsigned long long> attr_set{0};
+    static std::atomic<int> sm_count[64];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    const unsigned long long bit = 1ull << dev;
+    if (!(attr_set.load() & bit)) {
+        e = cudaFuncSetAttribute(chunk_fwd_tc_phased, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ph::kSmemBytes);
+        if (e != cudaSuccess) return e;
+        int sms = 0;
+        e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return e;
+        int per_sm = 0;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, chunk_fwd_tc_phased, ph::kThreads, ph::kSmemBytes);
+        if (e != cudaSuccess) return e;
+        if (per_sm < 1) return cudaErrorInvalidConfiguration;
+        sm_count[dev].store(sms);
+        attr_set.fetch_or(bit);
+    }
+    PhasedArgs a{};
+    a.k = (const __nv_bfloat16*)f.k;
+    a.q = (const __nv_bfloat16*)f.q;
+    a.v = (const __nv_bfloat16*)f.v;
+    a.alpha = f.alpha;
+    a.eta = f.eta;
+    a.theta = f.theta;
+    a.W1 = f.W1;
+    a.W2 = f.W2;
+    a.S1 = f.S1;
+    a.S2 = f.S2;
+    a.y = (__nv_bfloat16*)f.y;
+    a.attn = (const __nv_bfloat16*)f.attn;
+    a.ws = reinterpret_cast<uint8_t*>(f.ws);
+    a.ws_stride = f.ws_per_unit * sizeof(float);
+    a.T = f.T;
+    a.gate_ld = f.gate_ld;
+    a.chunk = f.chunk;
+    a.units = (int)f.units;
+    a.status = f.status;
+    a.sync = sync;
+    e = cudaMemsetAsync(sync, 0, 2 * sizeof(unsigned), st);
+    if (e != cudaSuccess) return e;
+    void* params[] = {&a};
+    return cudaLaunchCooperativeKernel((const void*)chunk_fwd_tc_phased, dim3((unsigned)sm_count[dev].load()),
+                                       dim3(ph::kThreads), params, ph::kSmemBytes, st);
+}
+
+}  // namespace titans

@@ -32,5 +32,12 @@ cudaError_t launch_step_cluster(const ForwardArgs& a, cudaStream_t st);
 cudaError_t launch_chunk_tc_mlp64(const ForwardArgs& a, const CUtensorMap& tk, const CUtensorMap& tq,
                                   const CUtensorMap& tv, cudaStream_t st);
 size_t chunk_tc_mlp64_smem_bytes();
+// Phased tensor-core chunk kernel of the wide memory (d = 128, h = 512, chunk <= 128, bf16): a
+// cooperative persistent launch over all SMs. Needs tc_phased_ws_bytes_per_unit() bytes of
+// workspace per unit (a.ws, a.ws_per_unit floats apart) and two device words `sync` for its grid
+// barrier (zeroed by the launch itself).
+size_t tc_phased_ws_bytes_per_unit();
+bool tc_phased_supported(int d, int h, int chunk);
+cudaError_t launch_chunk_tc_phased(const ForwardArgs& a, unsigned* sync, cudaStream_t st);
 
 }  // namespace titans

@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(HERE, "libtitans_mem.so")
 OK, EINVAL, EUNSUPPORTED, ECUDA, EDEVICE = 0, 1, 2, 3, 4
 BF16, FP32 = 0, 1
 FLAG_CUDA_CORES = 1
-PATH_TC_MLP64, PATH_CUDA_CORES, PATH_STEP_CLUSTER = 1, 2, 3
+PATH_TC_MLP64, PATH_CUDA_CORES, PATH_STEP_CLUSTER, PATH_TC_PHASED = 1, 2, 3, 4
 
 EXPORTED = ["titans_mem_init", "titans_mem_destroy", "titans_mem_forward", "titans_mem_step",
             "titans_mem_path", "titans_mem_sync_status", "titans_last_error_string", "titans_mem_version",
