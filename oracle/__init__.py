@@ -19,6 +19,10 @@ Two fp64 paths, both from the pages on "Titans: Learning to Memorize at Test Tim
   per-chunk scalars. It is pinned to :func:`forward` by the tests (1e-12) and
   is used where the token loop would take too long.
 
+* :func:`forward_deep` / :func:`forward_deep_closed_form` -- the deep memory
+  (walk-through sec. 3.1 "Memory Architecture", L_M >= 2 layers; sec. 5.5):
+  M(x) = W_L silu(W_{L-1} ... silu(W_1 x)), every hidden layer h wide, no bias,
+  the L layers packed one after another per unit (:func:`deep_shapes`).
 * :func:`mag_gate` / :func:`forward_gated` -- the gated output of the
   memory-as-a-gate architecture (walk-through sec. 4.2 "Gated Memory": o = y
   (x) M(x~), y the sliding-window attention branch's output; the tencent review's
@@ -50,6 +54,14 @@ def _open(path: str):
     f.argtypes = [ctypes.c_long, ctypes.c_long, ctypes.c_int, ctypes.c_int, ctypes.c_int] + \
         [ctypes.c_void_p] * 11 + [ctypes.c_int]
     lib.titans_oracle_threads.restype = ctypes.c_int
+    return _open_deep(lib)
+
+
+def _open_deep(lib):
+    f = lib.titans_oracle_forward_deep
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_long, ctypes.c_long, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int] + \
+        [ctypes.c_void_p] * 9 + [ctypes.c_int]
     return lib
 
 
@@ -215,3 +227,94 @@ def forward_gated(k, q, v, alpha, eta, theta, state: Dict, chunk: int, attn, n_t
     o_t = mag_gate(attn_t, M(q_t)) with M at the chunk-start weights. attn: [U, T, d]."""
     y, st = forward(k, q, v, alpha, eta, theta, state, chunk, n_threads=n_threads)
     return mag_gate(_np(attn, np.float32), y), st
+
+
+def deep_shapes(d: int, h: int, layers: int):
+    """[out, in] of every layer of the deep memory: W_1 [h, d], W_2 .. W_{L-1} [h, h], W_L [d, h]."""
+    return [(h, d)] + [(h, h)] * (layers - 2) + [(d, h)]
+
+
+def _deep_hidden(P: int, d: int, layers: int) -> int:
+    """Hidden width h of a packed deep state of P elements per unit."""
+    for h in range(1, 1 << 14):
+        n = sum(a * b for a, b in deep_shapes(d, h, layers))
+        if n == P:
+            return h
+        if n > P:
+            break
+    raise ValueError(f"a packed state of {P} elements per unit fits no {layers}-layer memory of width {d}")
+
+
+def pack_deep(mats):
+    """[U, out, in] per layer -> [U, P], layers one after another (row-major each)."""
+    return np.concatenate([np.asarray(m, np.float64).reshape(m.shape[0], -1) for m in mats], axis=1)
+
+
+def unpack_deep(W, d: int, h: int, layers: int):
+    W = np.asarray(W)
+    out, o = [], 0
+    for (a, b) in deep_shapes(d, h, layers):
+        out.append(W[:, o:o + a * b].reshape(W.shape[0], a, b))
+        o += a * b
+    return out
+
+
+def forward_deep(k, q, v, alpha, eta, theta, state: Dict, chunk: int, layers: int, want_y: bool = True,
+                 n_threads: int = 0, _lib_override=None):
+    """Token-by-token fp64 recurrence of the deep memory. state: {"W": [U, P], "S": [U, P]} packed
+    (pack_deep). Returns (y [U, T, d] or None, {"W", "S"} float64)."""
+    kf, qf, vf = (_np(x, np.float32) for x in (k, q, v))
+    al, et, th = (_np(x, np.float32) for x in (alpha, eta, theta))
+    U, T, d = kf.shape
+    W = _np(state["W"], np.float64).copy()
+    S = _np(state["S"], np.float64).copy()
+    h = _deep_hidden(W.shape[1], d, layers)
+    y = np.zeros((U, T, d), np.float64) if want_y else None
+    lib = _load() if _lib_override is None else _open_deep(_lib_override)
+    rc = lib.titans_oracle_forward_deep(U, T, d, h, layers, int(chunk), _ptr(kf), _ptr(qf), _ptr(vf), _ptr(al),
+                                        _ptr(et), _ptr(th), _ptr(W), _ptr(S), _ptr(y), int(n_threads))
+    if rc != 0:
+        raise RuntimeError("oracle: bad arguments or out of memory")
+    return y, {"W": W, "S": S}
+
+
+def forward_deep_closed_form(k, q, v, alpha, eta, theta, state: Dict, chunk: int, layers: int, want_y: bool = True):
+    """Chunk closed form of the deep memory in fp64 (numpy matmuls), same arguments as forward_deep:
+    per chunk every key goes forward through the chunk-start layers, the error 2 (M(k) - v) goes back
+    through them, and each layer's c- and d-weighted sums of per-token outer products update W, S."""
+    K, Qm, V = (_np(x, np.float64) for x in (k, q, v))
+    al, et, th = (_np(x, np.float64) for x in (alpha, eta, theta))
+    U, T, d = K.shape
+    h = _deep_hidden(_np(state["W"], np.float64).shape[1], d, layers)
+    Ws = [w.copy() for w in unpack_deep(_np(state["W"], np.float64), d, h, layers)]
+    Ss = [x.copy() for x in unpack_deep(_np(state["S"], np.float64), d, h, layers)]
+    y = np.zeros((U, T, d), np.float64) if want_y else None
+    tr = lambda x: np.swapaxes(x, -1, -2)
+
+    def fwd(X):
+        zs, acts = [], [X]
+        for l in range(layers - 1):
+            z = acts[-1] @ tr(Ws[l])
+            s_, a_ = _silu_parts(z)
+            zs.append((z, s_))
+            acts.append(a_)
+        return zs, acts, acts[-1] @ tr(Ws[-1])
+
+    for t0 in range(0, T, chunk):
+        t1 = min(t0 + chunk, T)
+        c, dd, A, E, sig = chunk_scalars(al[:, t0:t1], et[:, t0:t1], th[:, t0:t1])
+        A, E, sig = A[:, None, None], E[:, None, None], sig[:, None, None]
+        if want_y:
+            y[:, t0:t1] = fwd(Qm[:, t0:t1])[2]
+        zs, acts, out = fwd(K[:, t0:t1])
+        delta = 2.0 * (out - V[:, t0:t1])  # dl/d out, then dl/dz of each hidden layer going back
+        grads_c, grads_d = [None] * layers, [None] * layers
+        for l in range(layers - 1, -1, -1):
+            grads_c[l] = tr(delta * c[..., None]) @ acts[l]
+            grads_d[l] = tr(delta * dd[..., None]) @ acts[l]
+            if l > 0:
+                z, s_ = zs[l - 1]
+                delta = (delta @ Ws[l]) * (s_ * (1.0 + z * (1.0 - s_)))
+        for l in range(layers):
+            Ws[l], Ss[l] = A * Ws[l] + sig * Ss[l] - grads_c[l], E * Ss[l] - grads_d[l]
+    return y, {"W": pack_deep(Ws), "S": pack_deep(Ss)}

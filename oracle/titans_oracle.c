@@ -185,6 +185,130 @@ int titans_oracle_forward(long units, long T, int d, int h, int chunk, const flo
     return err;
 }
 
+/*
+ * Deep memory (walk-through sec. 3.1 "Memory Architecture": an MLP with L_M >= 2 layers; sec. 5.5
+ * "The Effect of Deep Memory"): M(x) = W_L silu(W_{L-1} ... silu(W_1 x)), every hidden layer h
+ * wide, no bias. The L layers' weights of one unit are packed one after another, each row-major
+ * [out][in]: W_1 [h][d], W_2 .. W_{L-1} [h][h], W_L [d][h].
+ */
+static size_t deep_size(int d, int h, int L) { return 2 * (size_t)h * d + (size_t)(L - 2) * h * h; }
+
+static size_t deep_offset(int d, int h, int l) { /* start of layer l (0-based, l < L) */
+    return l == 0 ? 0 : (size_t)h * d + (size_t)(l - 1) * h * h;
+}
+
+/* Forward of one input x: z[l] = W_l a[l-1] (a[-1] = x), a[l] = silu(z[l]) for the L-1 hidden
+ * layers (z, a are [L-1][h]); out = W_L a[L-2] (d). */
+static void deep_forward(int d, int h, int L, const double *W, const double *x, double *z, double *a,
+                         double *out) {
+    const double *in = x;
+    int n_in = d;
+    for (int l = 0; l < L - 1; ++l) {
+        const double *Wl = W + deep_offset(d, h, l);
+        for (int j = 0; j < h; ++j) {
+            double s = 0.0;
+            for (int m = 0; m < n_in; ++m) s += Wl[(size_t)j * n_in + m] * in[m];
+            z[(size_t)l * h + j] = s;
+            a[(size_t)l * h + j] = s * sigmoid(s);
+        }
+        in = a + (size_t)l * h;
+        n_in = h;
+    }
+    const double *WL = W + deep_offset(d, h, L - 1);
+    for (int i = 0; i < d; ++i) {
+        double s = 0.0;
+        for (int j = 0; j < h; ++j) s += WL[(size_t)i * h + j] * in[j];
+        out[i] = s;
+    }
+}
+
+/*
+ * Gradient of || M(k) - v ||^2 with respect to every layer, by the chain rule from the output:
+ *   e = 2 (out - v) is dl/d out; the output layer's gradient is e a[L-2]^T;
+ *   delta = dl/dz[l] = (W_{l+1}^T dl/dz[l+1]) * silu'(z[l]), silu'(z) = s (1 + z (1 - s));
+ *   layer l's gradient is delta (its input)^T, the input of layer 0 being k.
+ * g has the packed layout of W; delta and back are scratch of h doubles each.
+ */
+static void deep_grad(int d, int h, int L, const double *W, const double *k, const double *v, double *z,
+                      double *a, double *out, double *e, double *delta, double *back, double *g) {
+    deep_forward(d, h, L, W, k, z, a, out);
+    for (int i = 0; i < d; ++i) e[i] = 2.0 * (out[i] - v[i]);
+    /* output layer */
+    const double *WL = W + deep_offset(d, h, L - 1);
+    double *gL = g + deep_offset(d, h, L - 1);
+    const double *aL = a + (size_t)(L - 2) * h;
+    for (int i = 0; i < d; ++i)
+        for (int j = 0; j < h; ++j) gL[(size_t)i * h + j] = e[i] * aL[j];
+    for (int j = 0; j < h; ++j) {
+        double b = 0.0;
+        for (int i = 0; i < d; ++i) b += WL[(size_t)i * h + j] * e[i];
+        const double zz = z[(size_t)(L - 2) * h + j], s = sigmoid(zz);
+        delta[j] = b * s * (1.0 + zz * (1.0 - s));
+    }
+    /* hidden layers, from the last to the first */
+    for (int l = L - 2; l >= 0; --l) {
+        const double *in = l == 0 ? k : a + (size_t)(l - 1) * h;
+        const int n_in = l == 0 ? d : h;
+        double *gl = g + deep_offset(d, h, l);
+        for (int j = 0; j < h; ++j)
+            for (int m = 0; m < n_in; ++m) gl[(size_t)j * n_in + m] = delta[j] * in[m];
+        if (l > 0) {
+            const double *Wl = W + deep_offset(d, h, l);
+            for (int m = 0; m < h; ++m) {
+                double b = 0.0;
+                for (int j = 0; j < h; ++j) b += Wl[(size_t)j * h + m] * delta[j];
+                const double zz = z[(size_t)(l - 1) * h + m], s = sigmoid(zz);
+                back[m] = b * s * (1.0 + zz * (1.0 - s));
+            }
+            memcpy(delta, back, (size_t)h * sizeof(double));
+        }
+    }
+}
+
+static int run_unit_deep(long T, int d, int h, int L, int chunk, const float *k, const float *q,
+                         const float *v, const float *alpha, const float *eta, const float *theta,
+                         double *W, double *S, double *y) {
+    const size_t P = deep_size(d, h, L);
+    const size_t need = 2 * P + 3 * (size_t)d + 2 * (size_t)(L - 1) * h + 2 * (size_t)h + 2 * (size_t)d;
+    double *buf = (double *)malloc(need * sizeof(double));
+    if (!buf) return 1;
+    double *Wbar = buf, *g = Wbar + P, *kx = g + P, *vx = kx + d, *qx = vx + d;
+    double *z = qx + d, *a = z + (size_t)(L - 1) * h, *delta = a + (size_t)(L - 1) * h, *back = delta + h;
+    double *out = back + h, *e = out + d;
+    for (long t = 0; t < T; ++t) {
+        if (t % chunk == 0) memcpy(Wbar, W, P * sizeof(double)); /* chunk-start weights */
+        load_row(d, k + (size_t)t * d, kx);
+        load_row(d, v + (size_t)t * d, vx);
+        load_row(d, q + (size_t)t * d, qx);
+        if (y) deep_forward(d, h, L, Wbar, qx, z, a, y + (size_t)t * d); /* retrieval, no update */
+        deep_grad(d, h, L, Wbar, kx, vx, z, a, out, e, delta, back, g);
+        update(P, alpha[t], eta[t], theta[t], g, W, S);
+    }
+    free(buf);
+    return 0;
+}
+
+/* Deep memory forward; W, S: [units][deep_size] packed; returns 0, or 1 on a bad argument or an
+ * allocation failure. */
+int titans_oracle_forward_deep(long units, long T, int d, int h, int L, int chunk, const float *k,
+                               const float *q, const float *v, const float *alpha, const float *eta,
+                               const float *theta, double *W, double *S, double *y, int n_threads) {
+    if (units < 0 || T < 0 || d <= 0 || h <= 0 || L < 2 || chunk <= 0 || !W || !S) return 1;
+    const size_t P = deep_size(d, h, L);
+    int err = 0;
+#ifdef _OPENMP
+    if (n_threads > 0) omp_set_num_threads(n_threads);
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : err)
+#endif
+    for (long u = 0; u < units; ++u) {
+        err |= run_unit_deep(T, d, h, L, chunk, k + (size_t)u * T * d, q + (size_t)u * T * d,
+                             v + (size_t)u * T * d, alpha + (size_t)u * T, eta + (size_t)u * T,
+                             theta + (size_t)u * T, W + u * P, S + u * P, y ? y + (size_t)u * T * d : NULL);
+    }
+    (void)n_threads;
+    return err;
+}
+
 int titans_oracle_threads(void) {
 #ifdef _OPENMP
     return omp_get_max_threads();
