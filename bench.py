@@ -33,6 +33,8 @@ sys.path.insert(0, HERE)
 from titans_long_term_b200 import mem, synth  # noqa: E402
 
 METRIC = "memory tokens/sec (update+retrieve) per B200; % bf16 tensor-core peak"
+KERNEL_NAMES = {mem.PATH_TC_MLP64: "chunk_fwd_tc_mlp64", mem.PATH_CUDA_CORES: "chunk_fwd_cuda_cores",
+                mem.PATH_TC_PHASED: "chunk_fwd_tc_phased"}
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -315,13 +317,13 @@ def our_arm(args, w, rank, world, local_rank):
         "config": {"workload": w.name, "inputs": synth.describe(w),
                    "memory": f"MLP {w.d}-{w.h}-{w.d} SiLU" if w.h else f"linear {w.d}x{w.d}",
                    "B": w.B, "H": w.H, "T": w.T, "chunk": w.chunk, "units_per_gpu": w.units,
-                   "kernel": {1: "tcgen05 chunk kernel", 2: "CUDA-core chunk kernel"}.get(path, str(path)),
+                   "kernel": KERNEL_NAMES.get(path, str(path)),
                    "l2": "inputs larger than L2 (k, q, v, y, state = %.0f MB per step)" % (algo_bytes / 1e6)},
         "head_tokens_per_s": value * w.H,
         "pct_bf16_peak": 100.0 * achieved / peak,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": traffic,
-                     "peak_source": f"bf16_tflops ({which})", "kernel": "chunk_fwd_tc_mlp64",
+                     "peak_source": f"bf16_tflops ({which})", "kernel": KERNEL_NAMES.get(path, str(path)),
                      "flops_per_launch": flops, "avg_launch_ms": avg_launch,
                      "frac_of_sustained": achieved / peaks.get("bf16_tflops_sustained", peak),
                      "algorithmic_bytes_per_launch": algo_bytes,
@@ -385,7 +387,7 @@ def forward_measure(w, dev, steps: int, warmup: int, T=None):
     achieved = flops / (avg / 1e3) / 1e12
     peak = peaks["bf16_tflops"]
     algo_bytes = stream_bytes_per_head_token(w) * w.units * T + state_bytes_per_unit(w) * w.units
-    kernel = {mem.PATH_TC_MLP64: "chunk_fwd_tc_mlp64", mem.PATH_CUDA_CORES: "chunk_fwd_cuda_cores"}.get(path)
+    kernel = KERNEL_NAMES.get(path)
     sms = min(w.units, 148)
     rec = {"workload": w.name, "value": w.B * T / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms,
            "steps": steps, "warmup": warmup, "head_tokens_per_s": w.B * T * w.H / (ms / 1e3),

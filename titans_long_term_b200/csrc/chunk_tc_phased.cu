@@ -56,7 +56,10 @@ constexpr size_t KD = KC + (size_t)kNmax * kD * 2;         // bf16 [128 tok][d] 
 constexpr size_t SC = KD + (size_t)kNmax * kD * 2;         // fp32 c[128], d[128], A, E, sigma
 constexpr size_t kWsBytes = SC + 2048;
 // Shared memory: operand tiles, each [rows][64] bf16 with the 128-byte swizzle.
-constexpr uint32_t kSmemOperands = 192 * 1024;
+constexpr uint32_t kSmemOperands = 224 * 1024;
+// P4 stages the fp32 W and S tiles it updates ([128 rows][128 floats] each) after its 96 KB of
+// MMA operands.
+constexpr uint32_t kStageW = 96 * 1024, kStageS = 160 * 1024;
 constexpr uint32_t BAR = kSmemOperands;       // one mbarrier (MMA completion)
 constexpr uint32_t TPTR = BAR + 8;
 constexpr uint32_t OKF = TPTR + 4;            // the grid barrier's verdict for the CTA
@@ -104,6 +107,21 @@ __device__ __forceinline__ void load_tile(uint32_t tile, const uint8_t* src, siz
     }
 }
 
+// Byte offset of 16-byte chunk c (0..31) of row r in a [128][128] fp32 tile staged in shared memory:
+// the chunk index is XORed with r % 8 within its group of eight, so that the 32 lanes of a warp,
+// one row each, spread their 16-byte accesses over all banks.
+__device__ __forceinline__ uint32_t stage_off(int r, int c) {
+    return (uint32_t)r * 512u + ((uint32_t)((c & ~7) | ((c ^ r) & 7)) << 4);
+}
+
+// Coalesced copy of a [128 rows][128 floats] tile (row r at src + r * ld floats) into the staging layout.
+__device__ __forceinline__ void stage_in(uint32_t tile, const float* src, size_t ld) {
+    for (int i = threadIdx.x; i < 128 * 32; i += ph::kThreads) {
+        const int r = i >> 5, c = i & 31;
+        cp_async16(tile + stage_off(r, c), src + (size_t)r * ld + 4 * c);
+    }
+}
+
 // All operand copies of the tile have landed and are visible to the tensor core.
 __device__ __forceinline__ void operands_ready() {
     cp_async_wait_all();
@@ -115,6 +133,13 @@ __device__ __forceinline__ void operands_ready() {
 
 __device__ __forceinline__ uint32_t pack2(float a, float b) { return pack_bf16x2(a, b); }
 
+// tanh via the hardware approximation (one MUFU op, relative error about 2^-11).
+__device__ __forceinline__ float tanh_approx(float x) {
+    float y;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // Grid-wide barrier with a bounded spin. Returns false if any CTA gave up (timeout anywhere).
 __device__ bool grid_sync(const PhasedArgs& a, unsigned& epoch, volatile uint32_t* s_ok) {
     __syncthreads();
@@ -125,10 +150,14 @@ __device__ bool grid_sync(const PhasedArgs& a, unsigned& epoch, volatile uint32_
         atomicAdd(&a.sync[0], 1u);
         const unsigned target = epoch * gridDim.x;
         const unsigned long long t0 = globaltimer_ns();
-        while (true) {
+        // Every CTA polls the same word: back off between polls so that the spinning CTAs do not
+        // flood the L2 slice that holds it (the other CTAs' traffic goes through the same slices).
+        for (unsigned it = 0;; ++it) {
             unsigned v;
             asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(&a.sync[0]) : "memory");
             if (v >= target) break;
+            __nanosleep(128);
+            if ((it & 15u) != 15u) continue;
             unsigned ab;
             asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(ab) : "l"(&a.sync[1]) : "memory");
             if (ab) {
@@ -226,25 +255,31 @@ __global__ void __launch_bounds__(ph::kThreads, 1) chunk_fwd_tc_phased(const __g
                 uint8_t* w = unit_ws(u);
                 float* s_c = reinterpret_cast<float*>(sm);  // shared scratch: c[128], d[128], A, E, sigma
                 float* s_d = s_c + 128;
+                float* s_g = s_c + 512;                     // the chunk's gates: alpha, eta, theta [3][128]
+                for (int i = tid; i < 3 * kNmax; i += kThreads) {
+                    const int which = i / kNmax, j = i % kNmax;
+                    const float* g = which == 0 ? a.alpha : (which == 1 ? a.eta : a.theta);
+                    s_g[i] = j < n ? __ldg(g + (long)u * a.gate_ld + t0 + j) : 0.f;
+                }
+                __syncthreads();
                 if (tid == 0) {
-                    const float* al = a.alpha + (long)u * a.gate_ld + t0;
-                    const float* et = a.eta + (long)u * a.gate_ld + t0;
-                    const float* th = a.theta + (long)u * a.gate_ld + t0;
+                    const float* al = s_g;
+                    const float* et = s_g + kNmax;
+                    const float* th = s_g + 2 * kNmax;
                     float Pr = 1.f, Qr = 1.f, r_next = 0.f;
                     for (int j = kNmax - 1; j >= n; --j) s_c[j] = s_d[j] = 0.f;
                     for (int j = n - 1; j >= 0; --j) {
                         // r_j = P_j + eta_{j+1} r_{j+1}, P_j = prod_{l>j} (1 - alpha_l), Q_j = prod_{l>j} eta_l
-                        const float r = Pr + (j + 1 < n ? __ldg(et + j + 1) * r_next : 0.f);
-                        const float thj = __ldg(th + j);
-                        s_c[j] = thj * r;
-                        s_d[j] = thj * Qr;
+                        const float r = Pr + (j + 1 < n ? et[j + 1] * r_next : 0.f);
+                        s_c[j] = th[j] * r;
+                        s_d[j] = th[j] * Qr;
                         r_next = r;
-                        Pr *= 1.f - __ldg(al + j);
-                        Qr *= __ldg(et + j);
+                        Pr *= 1.f - al[j];
+                        Qr *= et[j];
                     }
-                    s_c[256] = Pr;                      // A = prod (1 - alpha)
-                    s_c[257] = Qr;                      // E = prod eta
-                    s_c[258] = __ldg(et) * r_next;      // sigma = eta_0 r_0
+                    s_c[256] = Pr;                 // A = prod (1 - alpha)
+                    s_c[257] = Qr;                 // E = prod eta
+                    s_c[258] = et[0] * r_next;     // sigma = eta_0 r_0
                 }
                 __syncthreads();
                 float* gsc = reinterpret_cast<float*>(w + SC);
@@ -309,8 +344,10 @@ __global__ void __launch_bounds__(ph::kThreads, 1) chunk_fwd_tc_phased(const __g
                 float spv[16];
 #pragma unroll
                 for (int i = 0; i < 16; i += 2) {
+                    // sigma(z) = (1 + tanh(z / 2)) / 2 (one MUFU op), silu(z) = z sigma(z)
                     const float z0 = __uint_as_float(r[i]), z1 = __uint_as_float(r[i + 1]);
-                    const float s0 = 1.f / (1.f + __expf(-z0)), s1 = 1.f / (1.f + __expf(-z1));
+                    const float s0 = fmaf(0.5f, tanh_approx(0.5f * z0), 0.5f);
+                    const float s1 = fmaf(0.5f, tanh_approx(0.5f * z1), 0.5f);
                     const float a0 = z0 * s0, a1 = z1 * s1;
                     pk[i / 2] = pack2(a0, a1);
                     spv[i] = s0 + a0 * (1.f - s0);  // silu'(z) = sigma + silu (1 - sigma)
@@ -375,11 +412,14 @@ __global__ void __launch_bounds__(ph::kThreads, 1) chunk_fwd_tc_phased(const __g
                 const bool valid = row < n;
                 const uint4* vrow = reinterpret_cast<const uint4*>(a.v + ((long)u * T + t0 + row) * kD + col0);
                 const size_t off = ((size_t)row * kD + col0) * 2;
+                uint4 vq[4];
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) vq[q4] = valid ? __ldg(vrow + q4) : make_uint4(0, 0, 0, 0);
 #pragma unroll
                 for (int q4 = 0; q4 < 4; ++q4) {
                     uint32_t og[4] = {0, 0, 0, 0}, oc[4] = {0, 0, 0, 0}, od[4] = {0, 0, 0, 0};
                     if (valid) {
-                        const uint4 vv = __ldg(vrow + q4);
+                        const uint4 vv = vq[q4];
                         const uint32_t vin[4] = {vv.x, vv.y, vv.z, vv.w};
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
@@ -409,8 +449,8 @@ __global__ void __launch_bounds__(ph::kThreads, 1) chunk_fwd_tc_phased(const __g
                         float y0 = yv[8 * q4 + 2 * e], y1 = yv[8 * q4 + 2 * e + 1];
                         if (arow) {  // memory-as-a-gate output attn * sigmoid(y) (walk-through sec. 4.2)
                             const float2 a2 = unpack_bf16x2(aw[e]);
-                            y0 = a2.x / (1.f + __expf(-y0));
-                            y1 = a2.y / (1.f + __expf(-y1));
+                            y0 = a2.x * fmaf(0.5f, tanh_approx(0.5f * y0), 0.5f);
+                            y1 = a2.y * fmaf(0.5f, tanh_approx(0.5f * y1), 0.5f);
                         }
                         o[e] = pack2(y0, y1);
                     }
@@ -452,7 +492,10 @@ __global__ void __launch_bounds__(ph::kThreads, 1) chunk_fwd_tc_phased(const __g
             const int h = mt * 128 + row;
             const float* sp_row = reinterpret_cast<const float*>(w + SP) + (size_t)h * kNmax + 64 * half;
             uint8_t* dt_row = w + DT + ((size_t)h * kNmax + 64 * half) * 2;
-#pragma unroll 1
+            float4 spv[16];  // this thread's 64 silu' values, read before any store
+#pragma unroll
+            for (int i = 0; i < 16; ++i) spv[i] = __ldcg(reinterpret_cast<const float4*>(sp_row) + i);
+#pragma unroll
             for (int blk = 0; blk < 4; ++blk) {
                 uint32_t r[16];
                 tmem_ld16(tmem + lane_off + 64 * half + 16 * blk, r);
@@ -460,7 +503,7 @@ __global__ void __launch_bounds__(ph::kThreads, 1) chunk_fwd_tc_phased(const __g
                 uint32_t pk[8];
 #pragma unroll
                 for (int q4 = 0; q4 < 4; ++q4) {
-                    const float4 s = __ldcg(reinterpret_cast<const float4*>(sp_row + 16 * blk) + q4);
+                    const float4 s = spv[4 * blk + q4];
                     pk[2 * q4] = pack2(__uint_as_float(r[4 * q4]) * s.x, __uint_as_float(r[4 * q4 + 1]) * s.y);
                     pk[2 * q4 + 1] = pack2(__uint_as_float(r[4 * q4 + 2]) * s.z, __uint_as_float(r[4 * q4 + 3]) * s.w);
                 }
@@ -504,6 +547,22 @@ __global__ void __launch_bounds__(ph::kThreads, 1) chunk_fwd_tc_phased(const __g
                     load_tile(B0 + kb * 16384, w + AT + ((size_t)mt * 128 * 256 + kb * 64) * 2, 256 * 2, 128, 128);
                 }
             }
+            // The fp32 rows this tile updates, staged with coalesced copies: W1 rows [mt*128, +128)
+            // (one contiguous 64 KB block) or W2 rows 0..127 at hidden columns [mt*128, +128).
+            float* Wg;
+            float* Sg;
+            size_t ldw;
+            if (which == 0) {
+                Wg = a.W1 + ((size_t)u * kH + mt * 128) * kD;
+                Sg = a.S1 + ((size_t)u * kH + mt * 128) * kD;
+                ldw = kD;
+            } else {
+                Wg = a.W2 + (size_t)u * kD * kH + mt * 128;
+                Sg = a.S2 + (size_t)u * kD * kH + mt * 128;
+                ldw = kH;
+            }
+            stage_in(sb + kStageW, Wg, ldw);
+            stage_in(sb + kStageS, Sg, ldw);
             operands_ready();
             if (tid == 0) {
                 for (int kb = 0; kb < 2; ++kb)
@@ -526,22 +585,12 @@ __global__ void __launch_bounds__(ph::kThreads, 1) chunk_fwd_tc_phased(const __g
                 ok = false;
                 break;
             }
-            // Epilogue: W <- A W + sigma S + dW_c, S <- E S + dW_d for this thread's row of the block.
+            // Epilogue: W <- A W + sigma S + dW_c, S <- E S + dW_d for this thread's row of the tile,
+            // in place in the staged tiles; then the bf16 copy of the row, and coalesced copies out.
             const float* gsc = reinterpret_cast<const float*>(w + SC);
             const float An = __ldcg(gsc + 256), En = __ldcg(gsc + 257), sig = __ldcg(gsc + 258);
-            float *Wr, *Sr;
-            uint8_t* Wb;
-            if (which == 0) {  // W1 row h, columns [64 half, +64)
-                const size_t e0 = ((size_t)u * kH + mt * 128 + row) * kD + 64 * half;
-                Wr = a.W1 + e0;
-                Sr = a.S1 + e0;
-                Wb = w + W1B + (((size_t)mt * 128 + row) * kD + 64 * half) * 2;
-            } else {  // W2 row i (of d), hidden columns mt*128 + [64 half, +64)
-                const size_t e0 = ((size_t)u * kD + row) * kH + mt * 128 + 64 * half;
-                Wr = a.W2 + e0;
-                Sr = a.S2 + e0;
-                Wb = w + W2B + ((size_t)row * kH + mt * 128 + 64 * half) * 2;
-            }
+            uint8_t* Wb = which == 0 ? w + W1B + (((size_t)mt * 128 + row) * kD + 64 * half) * 2
+                                     : w + W2B + ((size_t)row * kH + mt * 128 + 64 * half) * 2;
 #pragma unroll 1
             for (int blk = 0; blk < 4; ++blk) {
                 uint32_t rc[16], rd[16];
@@ -551,8 +600,9 @@ __global__ void __launch_bounds__(ph::kThreads, 1) chunk_fwd_tc_phased(const __g
                 uint32_t pk[8];
 #pragma unroll
                 for (int q4 = 0; q4 < 4; ++q4) {
-                    float4 wv = __ldcg(reinterpret_cast<const float4*>(Wr + 16 * blk) + q4);
-                    float4 sv = __ldcg(reinterpret_cast<const float4*>(Sr + 16 * blk) + q4);
+                    const uint32_t o = stage_off(row, 16 * half + 4 * blk + q4);
+                    const float4 wv = *reinterpret_cast<const float4*>(sm + kStageW + o);
+                    const float4 sv = *reinterpret_cast<const float4*>(sm + kStageS + o);
                     float wn[4] = {wv.x, wv.y, wv.z, wv.w}, sn[4] = {sv.x, sv.y, sv.z, sv.w};
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
@@ -560,14 +610,23 @@ __global__ void __launch_bounds__(ph::kThreads, 1) chunk_fwd_tc_phased(const __g
                         wn[e] = fmaf(An, wo, sig * so) + __uint_as_float(rc[4 * q4 + e]);
                         sn[e] = fmaf(En, so, __uint_as_float(rd[4 * q4 + e]));
                     }
-                    __stcg(reinterpret_cast<float4*>(Wr + 16 * blk) + q4, make_float4(wn[0], wn[1], wn[2], wn[3]));
-                    __stcg(reinterpret_cast<float4*>(Sr + 16 * blk) + q4, make_float4(sn[0], sn[1], sn[2], sn[3]));
+                    *reinterpret_cast<float4*>(sm + kStageW + o) = make_float4(wn[0], wn[1], wn[2], wn[3]);
+                    *reinterpret_cast<float4*>(sm + kStageS + o) = make_float4(sn[0], sn[1], sn[2], sn[3]);
                     pk[2 * q4] = pack2(wn[0], wn[1]);
                     pk[2 * q4 + 1] = pack2(wn[2], wn[3]);
                 }
                 uint4* dst = reinterpret_cast<uint4*>(Wb + 32 * blk);
                 __stcg(dst, make_uint4(pk[0], pk[1], pk[2], pk[3]));
                 __stcg(dst + 1, make_uint4(pk[4], pk[5], pk[6], pk[7]));
+            }
+            __syncthreads();
+            for (int i = tid; i < 128 * 32; i += kThreads) {
+                const int r = i >> 5, cc = i & 31;
+                const uint32_t o = stage_off(r, cc);
+                __stcg(reinterpret_cast<float4*>(Wg + (size_t)r * ldw + 4 * cc),
+                       *reinterpret_cast<const float4*>(sm + kStageW + o));
+                __stcg(reinterpret_cast<float4*>(Sg + (size_t)r * ldw + 4 * cc),
+                       *reinterpret_cast<const float4*>(sm + kStageS + o));
             }
         }
         if (!grid_sync(a, epoch, s_ok) || !ok) {
