@@ -73,7 +73,8 @@ typedef enum {
     TITANS_PATH_TC_MLP64 = 1,     /* tcgen05 bf16 chunk kernel, d=64, h=256, chunk<=64 */
     TITANS_PATH_CUDA_CORES = 2,   /* CUDA-core fp32 chunk kernel (any supported shape) */
     TITANS_PATH_STEP_CLUSTER = 3, /* single-token decode, thread-block-cluster kernel (MLP) */
-    TITANS_PATH_TC_PHASED = 4     /* tcgen05 bf16 chunk kernel over all SMs, d=128, h=512, chunk<=128 */
+    TITANS_PATH_TC_PHASED = 4,    /* tcgen05 bf16 chunk kernel over all SMs, d=128, h=512, chunk<=128 */
+    TITANS_PATH_DEEP_CUDA_CORES = 5 /* deep memory (titans_mem_init_deep), CUDA-core chunk kernel */
 } titans_path_t;
 
 /* Validates the configuration and allocates the handle, its device status word and
@@ -82,6 +83,15 @@ typedef enum {
  * TITANS_EUNSUPPORTED for d not in {64, 128}, d_hidden not in {0, 4d} or chunk
  * outside 1..128, TITANS_ECUDA if an allocation fails. */
 titans_status_t titans_mem_init(const titans_mem_config *cfg, titans_mem_t *out);
+
+/* titans_mem_init for a deep memory of `layers` layers (2..8), every hidden layer d_hidden wide:
+ *   M(x) = W_L silu(W_{L-1} ... silu(W_1 x)),  no bias.
+ * Defined by the walk-through's sec. 3.1 "Memory Architecture" (an MLP memory with L_M >= 2
+ * layers, deeper ones strictly more expressive than the linear one) and sec. 5.5 "The Effect of
+ * Deep Memory" (more layers remember better and cost throughput). Such a handle runs
+ * titans_mem_forward_deep only. Returns TITANS_EUNSUPPORTED for layers outside 2..8, TITANS_EINVAL
+ * for d_hidden = 0, and otherwise what titans_mem_init returns. */
+titans_status_t titans_mem_init_deep(const titans_mem_config *cfg, int layers, titans_mem_t *out);
 
 /* Frees the handle and its device memory. Must not race with work in flight. */
 titans_status_t titans_mem_destroy(titans_mem_t m);
@@ -127,6 +137,22 @@ titans_status_t titans_mem_forward_gated(titans_mem_t m, const void *k, const vo
                                          const float *alpha, const float *eta, const float *theta,
                                          long T, int chunk, float *W1, float *W2, float *S1, float *S2,
                                          const void *attn, void *o, void *stream);
+
+/*
+ * Chunk-wise forward of a deep memory (handle from titans_mem_init_deep; the same update and
+ * retrieval rules as titans_mem_forward, sec. 3.1-3.2, applied to every layer).
+ *   W, S  [B, H, P] fp32, P = 2 h d + (L - 2) h^2: per unit the layers one after another, each
+ *         row-major [out][in]: W_1 [h][d], W_2 .. W_{L-1} [h][h], W_L [d][h]; read at entry and
+ *         overwritten with the state after token T-1.
+ *   attn  NULL for y = M(q), or the attention branch's output for the memory-as-a-gate output
+ *         y = attn * sigmoid(M(q)) (see titans_mem_forward_gated).
+ *   Other arguments as in titans_mem_forward. Runs the CUDA-core chunk kernel (fp32 arithmetic;
+ *   k, q, v, y in the handle's dtype).
+ */
+titans_status_t titans_mem_forward_deep(titans_mem_t m, const void *k, const void *q, const void *v,
+                                        const float *alpha, const float *eta, const float *theta,
+                                        long T, int chunk, float *W, float *S, const void *attn, void *y,
+                                        void *stream);
 
 /* Device buffers that titans_mem_forward_host stages through, each the size of the host
  * array of the same name ([B, H, T, d] for k, q, v, y; [B, H, T] for the gates). The call

@@ -83,3 +83,22 @@ def test_noalloc_rejects_too_many_units_before_cuda():
                                       None, None, None, None)
     assert rc == mem.EINVAL
     assert "units" in L.titans_last_error_string().decode()
+
+
+@pytest.mark.parametrize("d,h,layers,status", [
+    (64, 256, 9, mem.EUNSUPPORTED),   # too deep
+    (64, 256, 1, mem.EUNSUPPORTED),   # below two layers
+    (64, 0, 3, mem.EINVAL),           # a deep memory needs hidden layers
+    (96, 384, 3, mem.EUNSUPPORTED),   # unsupported width, as for titans_mem_init
+])
+def test_init_deep_rejects_bad_configs(d, h, layers, status):
+    cfg = mem.Config(d, h, 64, mem.FP32, 1, 1, 0)
+    out = ctypes.c_void_p()
+    assert mem.lib().titans_mem_init_deep(ctypes.byref(cfg), layers, ctypes.byref(out)) == status
+    assert out.value is None
+
+
+def test_deep_forward_rejects_null_handle():
+    L = mem.lib()
+    rc = L.titans_mem_forward_deep(None, None, None, None, None, None, None, 16, 16, None, None, None, None, None)
+    assert rc == mem.EINVAL

@@ -14,6 +14,7 @@
 
 struct titans_mem {
     titans_mem_config cfg;
+    int layers = 2;     // memory depth; titans_mem_init_deep sets it
     int device;
     unsigned* status;   // device status word, then the phased kernel's two grid-barrier words
     float* ws;          // CUDA-core path workspace
@@ -155,13 +156,19 @@ int titans_mem_version(void) { return 100; }
 
 const char* titans_last_error_string(void) { return g_err.c_str(); }
 
-titans_status_t titans_mem_init(const titans_mem_config* cfg, titans_mem_t* out) {
+}  // extern "C"
+
+namespace {
+titans_status_t init_impl(const titans_mem_config* cfg, int layers, titans_mem_t* out) {
     if (!out) return fail(TITANS_EINVAL, "out is NULL");
     *out = nullptr;
     titans_status_t s = check_cfg(cfg);
     if (s != TITANS_OK) return s;
+    if (layers != 2 && (layers < 2 || layers > 8)) return fail(TITANS_EUNSUPPORTED, "layers must be in 2..8");
+    if (layers > 2 && cfg->d_hidden == 0) return fail(TITANS_EINVAL, "a deep memory needs d_hidden > 0");
     titans_mem* m = new titans_mem();
     m->cfg = *cfg;
+    m->layers = layers;
     cudaError_t e = cudaGetDevice(&m->device);
     if (e != cudaSuccess) {
         delete m;
@@ -174,6 +181,8 @@ titans_status_t titans_mem_init(const titans_mem_config* cfg, titans_mem_t* out)
         return cuda_fail(e, "allocating the status word");
     }
     m->ws_per_unit = titans::cuda_cores_ws_floats(cfg->d, cfg->d_hidden, cfg->chunk);
+    if (cfg->d_hidden)
+        m->ws_per_unit = std::max(m->ws_per_unit, titans::deep_ws_floats(cfg->d, cfg->d_hidden, layers, cfg->chunk));
     if (phased_eligible(*cfg, cfg->chunk))
         m->ws_per_unit = std::max(m->ws_per_unit, titans::tc_phased_ws_bytes_per_unit() / sizeof(float));
     m->ws_per_unit = (m->ws_per_unit + 255) & ~size_t(255);  // 1 KiB-aligned unit slices
@@ -185,6 +194,15 @@ titans_status_t titans_mem_init(const titans_mem_config* cfg, titans_mem_t* out)
     }
     *out = m;
     return TITANS_OK;
+}
+}  // namespace
+
+extern "C" {
+
+titans_status_t titans_mem_init(const titans_mem_config* cfg, titans_mem_t* out) { return init_impl(cfg, 2, out); }
+
+titans_status_t titans_mem_init_deep(const titans_mem_config* cfg, int layers, titans_mem_t* out) {
+    return init_impl(cfg, layers, out);
 }
 
 titans_status_t titans_mem_destroy(titans_mem_t m) {
@@ -200,6 +218,7 @@ titans_status_t titans_mem_destroy(titans_mem_t m) {
 
 int titans_mem_path(titans_mem_t m, int chunk, int step) {
     if (!m) return -1;
+    if (m->layers > 2) return (!step && chunk >= 1 && chunk <= m->cfg.chunk) ? TITANS_PATH_DEEP_CUDA_CORES : -1;
     if (step) return m->cfg.d_hidden ? TITANS_PATH_STEP_CLUSTER : TITANS_PATH_CUDA_CORES;
     if (chunk < 1 || chunk > m->cfg.chunk) return -1;
     if (tc_eligible(m->cfg, chunk)) return TITANS_PATH_TC_MLP64;
@@ -215,6 +234,7 @@ titans_status_t forward_impl(titans_mem_t m, const void* k, const void* q, const
                              const float* eta, const float* theta, long gate_ld, long T, int chunk, float* W1,
                              float* W2, float* S1, float* S2, void* y, void* stream, const void* attn = nullptr) {
     if (!m) return fail(TITANS_EINVAL, "handle is NULL");
+    if (m->layers > 2) return fail(TITANS_EINVAL, "a deep memory handle runs titans_mem_forward_deep");
     titans_status_t s = check_ptrs(m, k, q, v, alpha, eta, theta, W1, W2, S1, S2, y);
     if (s != TITANS_OK) return s;
     if (attn && !aligned16(attn)) return fail(TITANS_EINVAL, "attn is not 16-byte aligned");
@@ -259,6 +279,24 @@ titans_status_t titans_mem_forward_gated(titans_mem_t m, const void* k, const vo
                                          void* stream) {
     if (!attn) return fail(TITANS_EINVAL, "attn is NULL");
     return forward_impl(m, k, q, v, alpha, eta, theta, T, T, chunk, W1, W2, S1, S2, o, stream, attn);
+}
+
+titans_status_t titans_mem_forward_deep(titans_mem_t m, const void* k, const void* q, const void* v,
+                                        const float* alpha, const float* eta, const float* theta, long T, int chunk,
+                                        float* W, float* S, const void* attn, void* y, void* stream) {
+    if (!m) return fail(TITANS_EINVAL, "handle is NULL");
+    if (!m->cfg.d_hidden) return fail(TITANS_EINVAL, "the deep forward needs an MLP memory (d_hidden > 0)");
+    titans_status_t s = check_ptrs(m, k, q, v, alpha, eta, theta, W, W, S, S, y);
+    if (s != TITANS_OK) return s;
+    if (attn && !aligned16(attn)) return fail(TITANS_EINVAL, "attn is not 16-byte aligned");
+    if (T < 1) return fail(TITANS_EINVAL, "T must be >= 1");
+    if (T * (long)m->cfg.d >= (1L << 31)) return fail(TITANS_EUNSUPPORTED, "T * d must be below 2^31");
+    if (chunk < 1 || chunk > m->cfg.chunk) return fail(TITANS_EUNSUPPORTED, "chunk must be in 1..config.chunk");
+    titans::ForwardArgs a = make_args(m, k, q, v, alpha, eta, theta, T, chunk, W, nullptr, S, nullptr, y);
+    a.attn = attn;
+    cudaError_t e = titans::launch_chunk_deep_cuda_cores(a, m->layers, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
+    return TITANS_OK;
 }
 
 titans_status_t titans_mem_forward_host(titans_mem_t m, const void* k, const void* q, const void* v,
@@ -358,6 +396,7 @@ titans_status_t step_impl(titans_mem_t m, const void* k, const void* q, const vo
                           const float* eta, const float* theta, float* W1, float* W2, float* S1, float* S2, void* y,
                           void* stream, const void* attn) {
     if (!m) return fail(TITANS_EINVAL, "handle is NULL");
+    if (m->layers > 2) return fail(TITANS_EUNSUPPORTED, "no decode step for a deep memory handle");
     titans_status_t s = check_ptrs(m, k, q, v, alpha, eta, theta, W1, W2, S1, S2, y);
     if (s != TITANS_OK) return s;
     if (attn && !aligned16(attn)) return fail(TITANS_EINVAL, "attn is not 16-byte aligned");

@@ -36,6 +36,11 @@ size_t chunk_tc_mlp64_smem_bytes();
 // cooperative persistent launch over all SMs. Needs tc_phased_ws_bytes_per_unit() bytes of
 // workspace per unit (a.ws, a.ws_per_unit floats apart) and two device words `sync` for its grid
 // barrier (zeroed by the launch itself).
+// Deep memory (L >= 2 layers, packed state W, S [units][deep_state_floats] in ForwardArgs::W1 / S1),
+// CUDA-core chunk kernel; workspace deep_ws_floats per unit.
+size_t deep_ws_floats(int d, int h, int layers, int n);
+__host__ __device__ size_t deep_state_floats(int d, int h, int layers);
+cudaError_t launch_chunk_deep_cuda_cores(const ForwardArgs& a, int layers, cudaStream_t st);
 size_t tc_phased_ws_bytes_per_unit();
 bool tc_phased_supported(int d, int h, int chunk);
 cudaError_t launch_chunk_tc_phased(const ForwardArgs& a, unsigned* sync, cudaStream_t st);

@@ -19,12 +19,12 @@ LIB_PATH = os.path.join(HERE, "libtitans_mem.so")
 OK, EINVAL, EUNSUPPORTED, ECUDA, EDEVICE = 0, 1, 2, 3, 4
 BF16, FP32 = 0, 1
 FLAG_CUDA_CORES = 1
-PATH_TC_MLP64, PATH_CUDA_CORES, PATH_STEP_CLUSTER, PATH_TC_PHASED = 1, 2, 3, 4
+PATH_TC_MLP64, PATH_CUDA_CORES, PATH_STEP_CLUSTER, PATH_TC_PHASED, PATH_DEEP_CUDA_CORES = 1, 2, 3, 4, 5
 
 EXPORTED = ["titans_mem_init", "titans_mem_destroy", "titans_mem_forward", "titans_mem_step",
             "titans_mem_path", "titans_mem_sync_status", "titans_last_error_string", "titans_mem_version",
             "titans_mem_forward_noalloc", "titans_mem_forward_host", "titans_mem_forward_gated",
-            "titans_mem_step_gated"]
+            "titans_mem_step_gated", "titans_mem_init_deep", "titans_mem_forward_deep"]
 
 
 class TitansError(RuntimeError):
@@ -65,11 +65,14 @@ def lib():
                                               ctypes.POINTER(DeviceBuffers), l, vp]
         L.titans_mem_forward_gated.argtypes = [vp, vp, vp, vp, vp, vp, vp, l, i, vp, vp, vp, vp, vp, vp, vp]
         L.titans_mem_step_gated.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+        L.titans_mem_init_deep.argtypes = [ctypes.POINTER(Config), i, ctypes.POINTER(vp)]
+        L.titans_mem_forward_deep.argtypes = [vp, vp, vp, vp, vp, vp, vp, l, i, vp, vp, vp, vp, vp]
         L.titans_mem_sync_status.argtypes = [vp, vp]
         L.titans_last_error_string.restype = ctypes.c_char_p
         for f in ("titans_mem_init", "titans_mem_destroy", "titans_mem_forward", "titans_mem_step",
                   "titans_mem_path", "titans_mem_sync_status", "titans_mem_version", "titans_mem_forward_noalloc",
-                  "titans_mem_forward_host", "titans_mem_forward_gated", "titans_mem_step_gated"):
+                  "titans_mem_forward_host", "titans_mem_forward_gated", "titans_mem_step_gated",
+                  "titans_mem_init_deep", "titans_mem_forward_deep"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -93,14 +96,19 @@ class Memory:
     """A configured memory: B*H independent units of a linear (d_hidden = 0) or
     2-layer SiLU MLP memory (d_hidden = 4d)."""
 
-    def __init__(self, d: int, d_hidden: int, chunk: int, mode: str, B: int, H: int, cuda_cores: bool = False):
+    def __init__(self, d: int, d_hidden: int, chunk: int, mode: str, B: int, H: int, cuda_cores: bool = False,
+                 layers: Optional[int] = None):
         self.d, self.h, self.chunk, self.B, self.H = d, d_hidden, chunk, B, H
         self.mode = mode
+        self.layers = layers or 2
         self.dtype = torch.bfloat16 if mode == "bf16" else torch.float32
         cfg = Config(d, d_hidden, chunk, BF16 if mode == "bf16" else FP32, B, H,
                      FLAG_CUDA_CORES if cuda_cores else 0)
         h = ctypes.c_void_p()
-        _check(lib().titans_mem_init(ctypes.byref(cfg), ctypes.byref(h)))
+        if layers is None:
+            _check(lib().titans_mem_init(ctypes.byref(cfg), ctypes.byref(h)))
+        else:
+            _check(lib().titans_mem_init_deep(ctypes.byref(cfg), layers, ctypes.byref(h)))
         self._h = h
 
     def close(self):
@@ -155,6 +163,22 @@ class Memory:
                                               _ptr(state.get("W2")), _ptr(state["S1"]), _ptr(state.get("S2")),
                                               _ptr(attn), _ptr(o), _stream(stream)))
         return o
+
+    def forward_deep(self, k, q, v, alpha, eta, theta, state: Dict[str, torch.Tensor], chunk: Optional[int] = None,
+                     attn: Optional[torch.Tensor] = None, y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        """Deep memory (a handle made with layers=L): state {"W", "S"} [B, H, P] fp32, the layers packed
+        per unit (W_1 [h, d], W_2 .. W_{L-1} [h, h], W_L [d, h]); optional attn for the gated output."""
+        T = k.shape[-2]
+        if y is None:
+            y = torch.empty_like(k)
+        toks = {"k": k, "q": q, "v": v}
+        if attn is not None:
+            toks["attn"] = attn
+        self._check_tensors(toks, {"alpha": alpha, "eta": eta, "theta": theta}, state, y, (self.B, self.H, T))
+        _check(lib().titans_mem_forward_deep(self._h, _ptr(k), _ptr(q), _ptr(v), _ptr(alpha), _ptr(eta), _ptr(theta),
+                                             T, chunk or self.chunk, _ptr(state["W"]), _ptr(state["S"]), _ptr(attn),
+                                             _ptr(y), _stream(stream)))
+        return y
 
     def forward_host(self, k, q, v, alpha, eta, theta, state: Dict[str, torch.Tensor], y: torch.Tensor,
                      staging: Dict[str, torch.Tensor], chunk: Optional[int] = None, t_seg: int = 0,

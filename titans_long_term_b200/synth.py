@@ -335,3 +335,26 @@ def make_attn(w: Workload, units: Optional[Sequence[int]] = None, T: Optional[in
             parts.append(x[lo:hi])
         rows.append(_cast(torch.cat(parts) if parts else torch.zeros(0, w.d), dtype))
     return torch.stack(rows)
+
+
+def deep_shapes(d: int, h: int, layers: int):
+    """[out, in] of every layer of a deep memory: W_1 [h, d], W_2 .. W_{L-1} [h, h], W_L [d, h]."""
+    return [(h, d)] + [(h, h)] * (layers - 2) + [(d, h)]
+
+
+def make_deep_state(w: Workload, layers: int, units: Optional[Sequence[int]] = None) -> Dict[str, torch.Tensor]:
+    """Initial state of a deep memory for a list of units: W [U, P] with each layer ~ N(0, 1/fan_in),
+    packed layer after layer (row-major [out][in] each); S = 0. At 2 layers W_1, W_2 are the
+    2-layer memory's initial weights of the same units."""
+    units = list(range(w.units)) if units is None else list(units)
+    rows = []
+    for u in units:
+        st = unit_state(w, u)
+        mats = [st["W1"]]
+        g = _gen(w.seed, u, 0xDEE9)
+        for (o, i) in deep_shapes(w.d, w.h, layers)[1:-1]:
+            mats.append(torch.randn(o, i, generator=g) / np.sqrt(i))
+        mats.append(st["W2"])
+        rows.append(torch.cat([m.reshape(-1) for m in mats]))
+    W = torch.stack(rows).contiguous()
+    return {"W": W, "S": torch.zeros_like(W)}
