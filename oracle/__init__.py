@@ -318,3 +318,11 @@ def forward_deep_closed_form(k, q, v, alpha, eta, theta, state: Dict, chunk: int
         for l in range(layers):
             Ws[l], Ss[l] = A * Ws[l] + sig * Ss[l] - grads_c[l], E * Ss[l] - grads_d[l]
     return y, {"W": pack_deep(Ws), "S": pack_deep(Ss)}
+
+
+def expand_chunk_gates(g, T: int, chunk: int):
+    """Chunk-shared gates [U, ceil(T / chunk)] -> per-token gates [U, T]: every token of chunk c takes
+    the chunk's value (walk-through sec. 3.2, "Parameters as the Function of Chunks"). The forward
+    with chunk-shared gates is the token loop run on these."""
+    g = np.asarray(g, np.float32)
+    return np.ascontiguousarray(np.repeat(g, chunk, axis=1)[:, :T])

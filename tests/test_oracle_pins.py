@@ -114,3 +114,31 @@ def test_gated_forward_after_reset_halves_the_attention():
     assert np.array_equal(o[:, 16:], attn[:, 16:].astype(np.float64) / 2)
     y, _ = oracle.forward(k, q, v, al, et, th, st, 8)
     assert np.abs(o[:, :16] - oracle.mag_gate(attn[:, :16], y[:, :16])).max() == 0.0
+
+
+# ---------------------------------------------------------------- chunk-shared gates (the LTI variant)
+
+def test_chunk_coefficients_with_chunk_shared_gates_are_geometric_sums():
+    """With alpha, eta, theta shared by a chunk's tokens (walk-through sec. 3.2, "Parameters as the
+    Function of Chunks": the system is then linear time-invariant), the coefficients have closed
+    forms: P_j = (1-a)^(n-1-j), Q_j = e^(n-1-j), r_j = sum_{m=j}^{n-1} (1-a)^(n-1-m) e^(m-j)
+    = ((1-a)^(n-j) - e^(n-j)) / ((1-a) - e), c_j = th r_j, d_j = th e^(n-1-j), A = (1-a)^n, E = e^n,
+    sigma = e r_0. The oracle's scan must reach them; its coefficients depend on j only through
+    n-1-j (a convolution kernel)."""
+    for n, a, e, th in [(16, 0.03, 0.9, 0.07), (7, 0.0, 0.5, 0.1), (64, 0.01, 0.95, 0.002), (5, 0.3, 0.2, 1.0)]:
+        c, dd, A, E, sig = oracle.chunk_scalars(np.full(n, a), np.full(n, e), np.full(n, th))
+        j = np.arange(n)
+        keep = 1.0 - a
+        r = (keep ** (n - j) - e ** (n - j)) / (keep - e)
+        np.testing.assert_allclose(c, th * r, rtol=1e-12)
+        np.testing.assert_allclose(dd, th * e ** (n - 1 - j), rtol=1e-12)
+        np.testing.assert_allclose([A, E, sig], [keep ** n, e ** n, e * r[0]], rtol=1e-12)
+
+
+def test_forward_with_chunk_gates_is_the_forward_with_repeated_gates():
+    """oracle.expand_chunk_gates repeats each chunk's gates over its tokens (a ragged last chunk
+    included); running the token loop on them defines the chunk-shared-gate forward."""
+    g = np.arange(2 * 3, dtype=np.float32).reshape(2, 3)
+    x = oracle.expand_chunk_gates(g, T=7, chunk=3)
+    assert x.shape == (2, 7)
+    assert np.array_equal(x[0], [0, 0, 0, 1, 1, 1, 2]) and np.array_equal(x[1], [3, 3, 3, 4, 4, 4, 5])
