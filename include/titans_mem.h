@@ -56,6 +56,12 @@ typedef enum {
 
 /* flags */
 #define TITANS_FLAG_CUDA_CORES 1u  /* run the CUDA-core chunk kernel even where the tensor-core one applies */
+/* Chunk-shared gates (walk-through sec. 3.2, "Parameters as the Function of Chunks": alpha, eta,
+ * theta shared by the tokens of a chunk make the memory's recurrence time-invariant inside the
+ * chunk): the chunked forward calls then take alpha, eta, theta as [B, H, ceil(T / chunk)], one
+ * value per chunk of the call, applied to each of the chunk's tokens (a ragged last chunk too).
+ * titans_mem_step and titans_mem_forward_noalloc keep per-token gates. */
+#define TITANS_FLAG_CHUNK_GATES 2u
 
 typedef struct {
     int d;             /* key/value width: 64 or 128 */

@@ -127,7 +127,8 @@ titans::ForwardArgs make_args(titans_mem* m, const void* k, const void* q, const
     a.alpha = al;
     a.eta = et;
     a.theta = th;
-    a.gate_ld = T;
+    a.chunk_gates = (m->cfg.flags & TITANS_FLAG_CHUNK_GATES) != 0;
+    a.gate_ld = a.chunk_gates ? (T + chunk - 1) / chunk : T;
     a.W1 = W1;
     a.W2 = W2;
     a.S1 = S1;
@@ -137,6 +138,11 @@ titans::ForwardArgs make_args(titans_mem* m, const void* k, const void* q, const
     a.ws_per_unit = m->ws_per_unit;
     a.status = m->status;
     return a;
+}
+
+// Elements in one unit's gate row: T per-token gates, or one per chunk with TITANS_FLAG_CHUNK_GATES.
+long gate_row(const titans_mem* m, long T, int chunk) {
+    return (m && (m->cfg.flags & TITANS_FLAG_CHUNK_GATES) && chunk > 0) ? (T + chunk - 1) / chunk : T;
 }
 
 titans_status_t cuda_fail(cudaError_t e, const char* what) {
@@ -270,7 +276,7 @@ extern "C" {
 titans_status_t titans_mem_forward(titans_mem_t m, const void* k, const void* q, const void* v, const float* alpha,
                                    const float* eta, const float* theta, long T, int chunk, float* W1, float* W2,
                                    float* S1, float* S2, void* y, void* stream) {
-    return forward_impl(m, k, q, v, alpha, eta, theta, T, T, chunk, W1, W2, S1, S2, y, stream);
+    return forward_impl(m, k, q, v, alpha, eta, theta, gate_row(m, T, chunk), T, chunk, W1, W2, S1, S2, y, stream);
 }
 
 titans_status_t titans_mem_forward_gated(titans_mem_t m, const void* k, const void* q, const void* v,
@@ -278,7 +284,8 @@ titans_status_t titans_mem_forward_gated(titans_mem_t m, const void* k, const vo
                                          float* W1, float* W2, float* S1, float* S2, const void* attn, void* o,
                                          void* stream) {
     if (!attn) return fail(TITANS_EINVAL, "attn is NULL");
-    return forward_impl(m, k, q, v, alpha, eta, theta, T, T, chunk, W1, W2, S1, S2, o, stream, attn);
+    return forward_impl(m, k, q, v, alpha, eta, theta, gate_row(m, T, chunk), T, chunk, W1, W2, S1, S2, o, stream,
+                        attn);
 }
 
 titans_status_t titans_mem_forward_deep(titans_mem_t m, const void* k, const void* q, const void* v,
@@ -338,6 +345,7 @@ titans_status_t titans_mem_forward_host(titans_mem_t m, const void* k, const voi
     const size_t es = m->cfg.mode == TITANS_BF16 ? 2 : 4;  // token element size
     const size_t units = (size_t)m->cfg.B * m->cfg.H, d = (size_t)m->cfg.d;
     const size_t row_h = (size_t)T * d * es;  // one unit's host stream of k, q, v or y
+    const long G = gate_row(m, T, chunk);     // one unit's gate row
     // The gates go over whole ([units][T], contiguous: one copy each, 12 B per head-token) and
     // the forward of each segment reads its columns in place. The tokens of segment i, [t0, t0 +
     // tn) of every unit, are packed on the device as [units][tn][d] at the offset of the segments
@@ -357,7 +365,7 @@ titans_status_t titans_mem_forward_host(titans_mem_t m, const void* k, const voi
         float* dg[3] = {dev->alpha, dev->eta, dev->theta};
         const float* hg[3] = {alpha, eta, theta};
         for (int j = 0; j < 3 && e == cudaSuccess; ++j)
-            e = cudaMemcpyAsync(dg[j], hg[j], units * (size_t)T * 4, cudaMemcpyHostToDevice, m->s_in);
+            e = cudaMemcpyAsync(dg[j], hg[j], units * (size_t)G * 4, cudaMemcpyHostToDevice, m->s_in);
         if (e != cudaSuccess) return settle(cuda_fail(e, "copying the gates in"));
     }
     for (long i = 0; i < nseg; ++i) {
@@ -373,7 +381,8 @@ titans_status_t titans_mem_forward_host(titans_mem_t m, const void* k, const voi
         if (e == cudaSuccess) e = cudaStreamWaitEvent(st, m->ev[2 + 2 * i], 0);
         if (e != cudaSuccess) return settle(cuda_fail(e, "copying a segment in"));
         char* dy = static_cast<char*>(dev->y) + tok_off;
-        s = forward_impl(m, dk[0], dk[1], dk[2], dev->alpha + t0, dev->eta + t0, dev->theta + t0, T, tn, chunk, W1,
+        const long g0 = G == T ? t0 : t0 / chunk;  // the segment's first gate column
+        s = forward_impl(m, dk[0], dk[1], dk[2], dev->alpha + g0, dev->eta + g0, dev->theta + g0, G, tn, chunk, W1,
                          W2, S1, S2, dy, stream);
         if (s != TITANS_OK) return settle(s);
         e = cudaEventRecord(m->ev[3 + 2 * i], st);

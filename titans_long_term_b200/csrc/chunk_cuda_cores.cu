@@ -42,7 +42,7 @@ __host__ size_t cuda_cores_ws_floats(int d, int h, int n) {
 
 template <typename Tin>
 __global__ void __launch_bounds__(kCcThreads) chunk_fwd_cuda_cores(
-    int d, int h, long T, long gate_ld, int chunk, const Tin* __restrict__ k, const Tin* __restrict__ q,
+    int d, int h, long T, long gate_ld, int chunk, int chunk_gates, const Tin* __restrict__ k, const Tin* __restrict__ q,
     const Tin* __restrict__ v, const float* __restrict__ alpha, const float* __restrict__ eta,
     const float* __restrict__ theta, float* __restrict__ W1, float* __restrict__ W2, float* __restrict__ S1,
     float* __restrict__ S2, Tin* __restrict__ y, const Tin* __restrict__ attn, float* __restrict__ ws,
@@ -78,9 +78,10 @@ __global__ void __launch_bounds__(kCcThreads) chunk_fwd_cuda_cores(
     for (long t0 = 0; t0 < T; t0 += chunk) {
         const int n = (int)min((long)chunk, T - t0);
         for (int i = tid; i < n; i += blockDim.x) {
-            s_alpha[i] = alpha[t0 + i];
-            s_eta[i] = eta[t0 + i];
-            s_theta[i] = theta[t0 + i];
+            const long gi = chunk_gates ? t0 / chunk : t0 + i;  // chunk-shared or per-token gates
+            s_alpha[i] = alpha[gi];
+            s_eta[i] = eta[gi];
+            s_theta[i] = theta[gi];
         }
         __syncthreads();
         if (tid == 0) {  // suffix scan, division-free
@@ -198,7 +199,7 @@ __global__ void __launch_bounds__(kCcThreads) chunk_fwd_cuda_cores(
 template <typename Tin>
 cudaError_t launch_cuda_cores(const ForwardArgs& a, cudaStream_t st) {
     chunk_fwd_cuda_cores<Tin><<<(unsigned)a.units, kCcThreads, 0, st>>>(
-        a.d, a.h, a.T, a.gate_ld, a.chunk, (const Tin*)a.k, (const Tin*)a.q, (const Tin*)a.v, a.alpha, a.eta, a.theta, a.W1,
+        a.d, a.h, a.T, a.gate_ld, a.chunk, (int)a.chunk_gates, (const Tin*)a.k, (const Tin*)a.q, (const Tin*)a.v, a.alpha, a.eta, a.theta, a.W1,
         a.W2, a.S1, a.S2, (Tin*)a.y, (const Tin*)a.attn, a.ws, a.ws_per_unit);
     return cudaGetLastError();
 }

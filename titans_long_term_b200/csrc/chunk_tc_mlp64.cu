@@ -191,7 +191,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
     const __grid_constant__ CUtensorMap tmV, const float* __restrict__ alpha, const float* __restrict__ eta,
     const float* __restrict__ theta, float* __restrict__ W1g, float* __restrict__ W2g, float* __restrict__ S1g,
     float* __restrict__ S2g, __nv_bfloat16* __restrict__ yg, const __nv_bfloat16* __restrict__ attn, long T,
-    long gate_ld, int chunk, unsigned* status) {
+    long gate_ld, int chunk, int chunk_gates, unsigned* status) {
     using namespace tc;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -283,7 +283,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
             for (int i = 0; i < 2; ++i) {
                 const int j = lane + 32 * i;
                 const bool ok = j < n;
-                const long g = u * gate_ld + t0 + j;
+                const long g = u * gate_ld + (chunk_gates ? (long)c : t0 + j);  // chunk-shared or per-token
                 ga[i] = ok ? __ldg(alpha + g) : 0.f;
                 ge[i] = ok ? __ldg(eta + g) : 1.f;
                 gt[i] = ok ? __ldg(theta + g) : 0.f;
@@ -785,7 +785,7 @@ cudaError_t launch_chunk_tc_mlp64(const ForwardArgs& a, const CUtensorMap& tk, c
     }
     chunk_fwd_tc_mlp64<<<(unsigned)a.units, tc::kThreads, tc::kSmemBytes, st>>>(
         tk, tq, tv, a.alpha, a.eta, a.theta, a.W1, a.W2, a.S1, a.S2, (__nv_bfloat16*)a.y,
-        (const __nv_bfloat16*)a.attn, a.T, a.gate_ld, a.chunk, a.status);
+        (const __nv_bfloat16*)a.attn, a.T, a.gate_ld, a.chunk, (int)a.chunk_gates, a.status);
     return cudaGetLastError();
 }
 

@@ -81,6 +81,7 @@ struct PhasedArgs {
     size_t ws_stride;  // bytes per unit
     long T, gate_ld;
     int chunk, units;
+    int chunk_gates;   // gates shared by a chunk's tokens ([units][chunks]) instead of per token
     unsigned* status;
     unsigned* sync;    // [0] barrier arrivals, [1] abort flag; zero at launch
 };
@@ -259,7 +260,7 @@ __global__ void __launch_bounds__(ph::kThreads, 1) chunk_fwd_tc_phased(const __g
                 for (int i = tid; i < 3 * kNmax; i += kThreads) {
                     const int which = i / kNmax, j = i % kNmax;
                     const float* g = which == 0 ? a.alpha : (which == 1 ? a.eta : a.theta);
-                    s_g[i] = j < n ? __ldg(g + (long)u * a.gate_ld + t0 + j) : 0.f;
+                    s_g[i] = j < n ? __ldg(g + (long)u * a.gate_ld + (a.chunk_gates ? t0 / a.chunk : t0 + j)) : 0.f;
                 }
                 __syncthreads();
                 if (tid == 0) {
@@ -687,6 +688,7 @@ cudaError_t launch_chunk_tc_phased(const ForwardArgs& f, unsigned* sync, cudaStr
     a.gate_ld = f.gate_ld;
     a.chunk = f.chunk;
     a.units = (int)f.units;
+    a.chunk_gates = f.chunk_gates ? 1 : 0;
     a.status = f.status;
     a.sync = sync;
     e = cudaMemsetAsync(sync, 0, 2 * sizeof(unsigned), st);

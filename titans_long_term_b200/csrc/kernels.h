@@ -14,6 +14,7 @@ struct ForwardArgs {
     const void *k, *q, *v;
     const float *alpha, *eta, *theta;
     long gate_ld;      // elements between consecutive units' gate rows (T for [B, H, T])
+    bool chunk_gates;  // gates shared by a chunk's tokens: [units][ceil(T / chunk)], token t reads t / chunk
     float *W1, *W2, *S1, *S2;
     void* y;
     const void* attn;  // NULL: y = M(q); else y = attn * sigmoid(M(q)) (memory-as-a-gate output), dtype of y

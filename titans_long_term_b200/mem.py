@@ -19,6 +19,7 @@ LIB_PATH = os.path.join(HERE, "libtitans_mem.so")
 OK, EINVAL, EUNSUPPORTED, ECUDA, EDEVICE = 0, 1, 2, 3, 4
 BF16, FP32 = 0, 1
 FLAG_CUDA_CORES = 1
+FLAG_CHUNK_GATES = 2
 PATH_TC_MLP64, PATH_CUDA_CORES, PATH_STEP_CLUSTER, PATH_TC_PHASED, PATH_DEEP_CUDA_CORES = 1, 2, 3, 4, 5
 
 EXPORTED = ["titans_mem_init", "titans_mem_destroy", "titans_mem_forward", "titans_mem_step",
@@ -97,13 +98,14 @@ class Memory:
     2-layer SiLU MLP memory (d_hidden = 4d)."""
 
     def __init__(self, d: int, d_hidden: int, chunk: int, mode: str, B: int, H: int, cuda_cores: bool = False,
-                 layers: Optional[int] = None):
+                 layers: Optional[int] = None, chunk_gates: bool = False):
         self.d, self.h, self.chunk, self.B, self.H = d, d_hidden, chunk, B, H
         self.mode = mode
         self.layers = layers or 2
+        self.chunk_gates = chunk_gates
         self.dtype = torch.bfloat16 if mode == "bf16" else torch.float32
         cfg = Config(d, d_hidden, chunk, BF16 if mode == "bf16" else FP32, B, H,
-                     FLAG_CUDA_CORES if cuda_cores else 0)
+                     (FLAG_CUDA_CORES if cuda_cores else 0) | (FLAG_CHUNK_GATES if chunk_gates else 0))
         h = ctypes.c_void_p()
         if layers is None:
             _check(lib().titans_mem_init(ctypes.byref(cfg), ctypes.byref(h)))
@@ -125,13 +127,20 @@ class Memory:
     def path(self, chunk: Optional[int] = None, step: bool = False) -> int:
         return lib().titans_mem_path(self._h, chunk or self.chunk, int(step))
 
-    def _check_tensors(self, toks, gates, state, y, lead):
+    def _gate_lead(self, lead, chunk):
+        """Shape of a gate array: one value per token, or per chunk with chunk-shared gates."""
+        if not self.chunk_gates or len(lead) < 3:
+            return lead
+        return lead[:-1] + ((lead[-1] + chunk - 1) // chunk,)
+
+    def _check_tensors(self, toks, gates, state, y, lead, chunk=None):
         for n, t in list(toks.items()) + [("y", y)]:
             if t.dtype != self.dtype or not t.is_cuda or not t.is_contiguous() or tuple(t.shape) != lead + (self.d,):
                 raise ValueError(f"{n}: expected contiguous CUDA {self.dtype} of shape {lead + (self.d,)}")
+        glead = self._gate_lead(lead, chunk or self.chunk)
         for n, t in gates.items():
-            if t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous() or tuple(t.shape) != lead:
-                raise ValueError(f"{n}: expected contiguous CUDA float32 of shape {lead}")
+            if t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous() or tuple(t.shape) != glead:
+                raise ValueError(f"{n}: expected contiguous CUDA float32 of shape {glead}")
         for n, t in state.items():
             if t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous():
                 raise ValueError(f"{n}: expected contiguous CUDA float32")
@@ -143,7 +152,7 @@ class Memory:
         if y is None:
             y = torch.empty_like(k)
         self._check_tensors({"k": k, "q": q, "v": v}, {"alpha": alpha, "eta": eta, "theta": theta}, state, y,
-                            (self.B, self.H, T))
+                            (self.B, self.H, T), chunk)
         _check(lib().titans_mem_forward(self._h, _ptr(k), _ptr(q), _ptr(v), _ptr(alpha), _ptr(eta), _ptr(theta),
                                         T, chunk or self.chunk, _ptr(state["W1"]), _ptr(state.get("W2")),
                                         _ptr(state["S1"]), _ptr(state.get("S2")), _ptr(y), _stream(stream)))
@@ -157,7 +166,7 @@ class Memory:
         if o is None:
             o = torch.empty_like(k)
         self._check_tensors({"k": k, "q": q, "v": v, "attn": attn}, {"alpha": alpha, "eta": eta, "theta": theta},
-                            state, o, (self.B, self.H, T))
+                            state, o, (self.B, self.H, T), chunk)
         _check(lib().titans_mem_forward_gated(self._h, _ptr(k), _ptr(q), _ptr(v), _ptr(alpha), _ptr(eta),
                                               _ptr(theta), T, chunk or self.chunk, _ptr(state["W1"]),
                                               _ptr(state.get("W2")), _ptr(state["S1"]), _ptr(state.get("S2")),
@@ -174,7 +183,7 @@ class Memory:
         toks = {"k": k, "q": q, "v": v}
         if attn is not None:
             toks["attn"] = attn
-        self._check_tensors(toks, {"alpha": alpha, "eta": eta, "theta": theta}, state, y, (self.B, self.H, T))
+        self._check_tensors(toks, {"alpha": alpha, "eta": eta, "theta": theta}, state, y, (self.B, self.H, T), chunk)
         _check(lib().titans_mem_forward_deep(self._h, _ptr(k), _ptr(q), _ptr(v), _ptr(alpha), _ptr(eta), _ptr(theta),
                                              T, chunk or self.chunk, _ptr(state["W"]), _ptr(state["S"]), _ptr(attn),
                                              _ptr(y), _stream(stream)))
@@ -192,11 +201,12 @@ class Memory:
         for n, t in (("k", k), ("q", q), ("v", v), ("y", y)):
             if t.is_cuda or t.dtype != self.dtype or not t.is_contiguous() or tuple(t.shape) != lead + (self.d,):
                 raise ValueError(f"{n}: expected contiguous host {self.dtype} of shape {lead + (self.d,)}")
+        glead = self._gate_lead(lead, chunk or self.chunk)
         for n, t in (("alpha", alpha), ("eta", eta), ("theta", theta)):
-            if t.is_cuda or t.dtype != torch.float32 or not t.is_contiguous() or tuple(t.shape) != lead:
-                raise ValueError(f"{n}: expected contiguous host float32 of shape {lead}")
+            if t.is_cuda or t.dtype != torch.float32 or not t.is_contiguous() or tuple(t.shape) != glead:
+                raise ValueError(f"{n}: expected contiguous host float32 of shape {glead}")
         self._check_tensors({n: staging[n] for n in ("k", "q", "v")},
-                            {n: staging[n] for n in ("alpha", "eta", "theta")}, state, staging["y"], lead)
+                            {n: staging[n] for n in ("alpha", "eta", "theta")}, state, staging["y"], lead, chunk)
         dev = DeviceBuffers(*(staging[n].data_ptr() for n in ("k", "q", "v", "alpha", "eta", "theta", "y")))
         _check(lib().titans_mem_forward_host(self._h, _ptr(k), _ptr(q), _ptr(v), _ptr(alpha), _ptr(eta),
                                              _ptr(theta), T, chunk or self.chunk, _ptr(state["W1"]),
