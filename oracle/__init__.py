@@ -23,6 +23,12 @@ Two fp64 paths, both from the pages on "Titans: Learning to Memorize at Test Tim
   (walk-through sec. 3.1 "Memory Architecture", L_M >= 2 layers; sec. 5.5):
   M(x) = W_L silu(W_{L-1} ... silu(W_1 x)), every hidden layer h wide, no bias,
   the L layers packed one after another per unit (:func:`deep_shapes`).
+* :func:`linear_chunk_map` / :func:`forward_linear_scan` -- for the linear memory
+  the chunk update is affine in the row state X = [W | S]: X -> X M_c + N_c, so
+  the chunks combine by an associative scan (German summary, "Parallelisiertes
+  Training": parallel associative scans; tencent review, the same): segments
+  of chunks compose their maps independently, a short scan over the segments
+  gives every segment's start state, and each segment then runs its chunks.
 * :func:`mag_gate` / :func:`forward_gated` -- the gated output of the
   memory-as-a-gate architecture (walk-through sec. 4.2 "Gated Memory": o = y
   (x) M(x~), y the sliding-window attention branch's output; the tencent review's
@@ -326,3 +332,67 @@ def expand_chunk_gates(g, T: int, chunk: int):
     with chunk-shared gates is the token loop run on these."""
     g = np.asarray(g, np.float32)
     return np.ascontiguousarray(np.repeat(g, chunk, axis=1)[:, :T])
+
+
+def linear_chunk_map(K, V, alpha, eta, theta):
+    """The affine map of one chunk of the linear memory M(x) = W x on the row state X = [W | S]
+    (d x 2d): X' = X M + N with (K, V: [n, d] rows k_j, v_j; C = diag(c), D = diag(d) of the chunk)
+        M = [[A I - 2 K^T C K, -2 K^T D K], [sigma I, E I]]   (2d x 2d)
+        N = [2 V^T C K, 2 V^T D K]                            (d x 2d)
+    from W' = A W + sigma S - sum_j c_j 2 (W k_j - v_j) k_j^T and S' = E S - sum_j d_j 2 (W k_j - v_j) k_j^T."""
+    K = np.asarray(K, np.float64)
+    V = np.asarray(V, np.float64)
+    d = K.shape[1]
+    c, dd, A, E, sig = chunk_scalars(alpha, eta, theta)
+    I = np.eye(d)
+    M = np.block([[A * I - 2.0 * K.T @ (c[:, None] * K), -2.0 * K.T @ (dd[:, None] * K)],
+                  [sig * I, E * I]])
+    N = np.concatenate([2.0 * V.T @ (c[:, None] * K), 2.0 * V.T @ (dd[:, None] * K)], axis=1)
+    return M, N
+
+
+def forward_linear_scan(k, q, v, alpha, eta, theta, state: Dict, chunk: int, segments: int, tree: bool = False):
+    """Linear memory forward by the cross-chunk scan, fp64: the chunk maps of each of `segments`
+    segments are composed (tree=True: pairwise, as a parallel scan would), the segment totals are
+    scanned to give each segment's start state, and each segment's chunks are then applied in order
+    (y_t = W q_t with the chunk-start W). Same arguments and returns as forward() for the linear
+    memory."""
+    K, Qm, V = (_np(x, np.float64) for x in (k, q, v))
+    al, et, th = (_np(x, np.float64) for x in (alpha, eta, theta))
+    U, T, d = K.shape
+    W = _np(state["W1"], np.float64).copy()
+    S = _np(state["S1"], np.float64).copy()
+    y = np.zeros((U, T, d))
+    nch = (T + chunk - 1) // chunk
+    G = (nch + segments - 1) // segments
+    bounds = [(s * G, min((s + 1) * G, nch)) for s in range(segments) if s * G < nch]
+
+    def compose(m1, m2):  # apply m1 then m2
+        return m1[0] @ m2[0], m1[1] @ m2[0] + m2[1]
+    for u in range(U):
+        maps = []
+        for c in range(nch):
+            t0, t1 = c * chunk, min((c + 1) * chunk, T)
+            maps.append(linear_chunk_map(K[u, t0:t1], V[u, t0:t1], al[u, t0:t1], et[u, t0:t1], th[u, t0:t1]))
+        seg = []
+        for c0, c1 in bounds:
+            ms = maps[c0:c1]
+            if tree:
+                while len(ms) > 1:
+                    ms = [compose(ms[i], ms[i + 1]) if i + 1 < len(ms) else ms[i] for i in range(0, len(ms), 2)]
+                seg.append(ms[0])
+            else:
+                tot = (np.eye(2 * d), np.zeros((d, 2 * d)))
+                for mp in ms:
+                    tot = compose(tot, mp)
+                seg.append(tot)
+        X = np.concatenate([W[u], S[u]], axis=1)
+        for (c0, c1), (Ms, Ns) in zip(bounds, seg):
+            Xc = X
+            for c in range(c0, c1):
+                t0, t1 = c * chunk, min((c + 1) * chunk, T)
+                y[u, t0:t1] = Qm[u, t0:t1] @ Xc[:, :d].T
+                Xc = Xc @ maps[c][0] + maps[c][1]
+            X = X @ Ms + Ns
+        W[u], S[u] = X[:, :d], X[:, d:]
+    return y, {"W1": W, "S1": S}

@@ -142,3 +142,35 @@ def test_forward_with_chunk_gates_is_the_forward_with_repeated_gates():
     x = oracle.expand_chunk_gates(g, T=7, chunk=3)
     assert x.shape == (2, 7)
     assert np.array_equal(x[0], [0, 0, 0, 1, 1, 1, 2]) and np.array_equal(x[1], [3, 3, 3, 4, 4, 4, 5])
+
+
+# ---------------------------------------------------------------- the linear memory's cross-chunk scan
+
+@pytest.mark.parametrize("T,chunk,segments", [(64, 16, 1), (100, 16, 3), (96, 8, 12), (37, 5, 4)])
+@pytest.mark.parametrize("tree", [False, True])
+def test_cross_chunk_scan_matches_the_token_loop(T, chunk, segments, tree):
+    """The linear memory's chunk update is an affine map of [W | S]; composing the maps per segment
+    (in order or pairwise) and scanning the segments gives the defining recurrence's result."""
+    k, q, v, al, et, th, st = _mk(2, T, 6, 0, 71 + T)
+    y, a = oracle.forward(k, q, v, al, et, th, st, chunk)
+    ys, b = oracle.forward_linear_scan(k, q, v, al, et, th, st, chunk, segments, tree=tree)
+    assert np.abs(ys - y).max() <= 1e-12 * np.abs(y).max()
+    for n in a:
+        assert np.abs(b[n] - a[n]).max() <= 1e-12 * np.abs(a[n]).max(), n
+
+
+def test_chunk_map_against_the_recurrence_on_a_basis():
+    """M and N of one chunk, against the token loop started from W = e_i rows / S = e_i rows with v = 0
+    (the columns of M) and from W = S = 0 (N)."""
+    k, q, v, al, et, th, _ = _mk(1, 9, 3, 0, 81)
+    d = 3
+    M, N = oracle.linear_chunk_map(k[0], v[0], al[0], et[0], th[0])
+    zero = np.zeros_like(v)
+    for i in range(2 * d):
+        X = np.zeros((1, d, 2 * d))
+        X[0, 0, i] = 1.0  # row 0 of [W | S] is the basis row e_i
+        _, out = oracle.forward(k, q, zero, al, et, th, {"W1": X[:, :, :d], "S1": X[:, :, d:]}, 9)
+        got = np.concatenate([out["W1"][0, 0], out["S1"][0, 0]])
+        np.testing.assert_allclose(got, M[i], rtol=1e-12, atol=1e-14)
+    _, out = oracle.forward(k, q, v, al, et, th, {"W1": np.zeros((1, d, d)), "S1": np.zeros((1, d, d))}, 9)
+    np.testing.assert_allclose(np.concatenate([out["W1"][0], out["S1"][0]], axis=1), N, rtol=1e-12, atol=1e-14)
