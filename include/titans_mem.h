@@ -62,6 +62,13 @@ typedef enum {
  * value per chunk of the call, applied to each of the chunk's tokens (a ragged last chunk too).
  * titans_mem_step and titans_mem_forward_noalloc keep per-token gates. */
 #define TITANS_FLAG_CHUNK_GATES 2u
+/* Linear memory only: run the chunks by a cross-chunk scan instead of one after another. One
+ * chunk of the linear memory is an affine map of [W | S], so segments of chunks compose their
+ * maps in parallel, a short scan over the segments gives each segment's start state, and the
+ * segments then run their chunks in parallel (the associative scan of the German summary's
+ * "Parallelisiertes Training" and the tencent review). A handle spreads a unit over about
+ * (SMs / units) segments, which pays for long streams of few units. fp32 arithmetic. */
+#define TITANS_FLAG_CHUNK_SCAN 4u
 
 typedef struct {
     int d;             /* key/value width: 64 or 128 */
@@ -80,7 +87,8 @@ typedef enum {
     TITANS_PATH_CUDA_CORES = 2,   /* CUDA-core fp32 chunk kernel (any supported shape) */
     TITANS_PATH_STEP_CLUSTER = 3, /* single-token decode, thread-block-cluster kernel (MLP) */
     TITANS_PATH_TC_PHASED = 4,    /* tcgen05 bf16 chunk kernel over all SMs, d=128, h=512, chunk<=128 */
-    TITANS_PATH_DEEP_CUDA_CORES = 5 /* deep memory (titans_mem_init_deep), CUDA-core chunk kernel */
+    TITANS_PATH_DEEP_CUDA_CORES = 5, /* deep memory (titans_mem_init_deep), CUDA-core chunk kernel */
+    TITANS_PATH_LINEAR_SCAN = 6      /* linear memory, cross-chunk scan (TITANS_FLAG_CHUNK_SCAN) */
 } titans_path_t;
 
 /* Validates the configuration and allocates the handle, its device status word and

@@ -15,6 +15,7 @@
 struct titans_mem {
     titans_mem_config cfg;
     int layers = 2;     // memory depth; titans_mem_init_deep sets it
+    int nseg_max = 1;   // segments per unit of the linear memory's cross-chunk scan
     int device;
     unsigned* status;   // device status word, then the phased kernel's two grid-barrier words
     float* ws;          // CUDA-core path workspace
@@ -191,6 +192,19 @@ titans_status_t init_impl(const titans_mem_config* cfg, int layers, titans_mem_t
         m->ws_per_unit = std::max(m->ws_per_unit, titans::deep_ws_floats(cfg->d, cfg->d_hidden, layers, cfg->chunk));
     if (phased_eligible(*cfg, cfg->chunk))
         m->ws_per_unit = std::max(m->ws_per_unit, titans::tc_phased_ws_bytes_per_unit() / sizeof(float));
+    if (cfg->d_hidden == 0 && (cfg->flags & TITANS_FLAG_CHUNK_SCAN)) {
+        int sms = 0;
+        e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, m->device);
+        if (e != cudaSuccess) {
+            cudaFree(m->status);
+            delete m;
+            return cuda_fail(e, "querying the SM count");
+        }
+        // Enough segments to give every SM a CTA, at most 4096 per unit.
+        m->nseg_max = (int)std::max(1L, std::min(4096L, (long)sms / ((long)cfg->B * cfg->H)));
+        m->ws_per_unit =
+            std::max(m->ws_per_unit, (size_t)m->nseg_max * titans::linear_scan_slot_floats(cfg->d, cfg->chunk));
+    }
     m->ws_per_unit = (m->ws_per_unit + 255) & ~size_t(255);  // 1 KiB-aligned unit slices
     e = cudaMalloc(&m->ws, m->ws_per_unit * sizeof(float) * (size_t)cfg->B * cfg->H);
     if (e != cudaSuccess) {
@@ -227,6 +241,7 @@ int titans_mem_path(titans_mem_t m, int chunk, int step) {
     if (m->layers > 2) return (!step && chunk >= 1 && chunk <= m->cfg.chunk) ? TITANS_PATH_DEEP_CUDA_CORES : -1;
     if (step) return m->cfg.d_hidden ? TITANS_PATH_STEP_CLUSTER : TITANS_PATH_CUDA_CORES;
     if (chunk < 1 || chunk > m->cfg.chunk) return -1;
+    if (m->cfg.d_hidden == 0 && (m->cfg.flags & TITANS_FLAG_CHUNK_SCAN)) return TITANS_PATH_LINEAR_SCAN;
     if (tc_eligible(m->cfg, chunk)) return TITANS_PATH_TC_MLP64;
     return phased_eligible(m->cfg, chunk) ? TITANS_PATH_TC_PHASED : TITANS_PATH_CUDA_CORES;
 }
@@ -260,6 +275,8 @@ titans_status_t forward_impl(titans_mem_t m, const void* k, const void* q, const
             !encode_tokens(&tv, v, T, a.units, chunk))
             return fail(TITANS_ECUDA, "cuTensorMapEncodeTiled failed");
         e = titans::launch_chunk_tc_mlp64(a, tk, tq, tv, st);
+    } else if (m->cfg.d_hidden == 0 && (m->cfg.flags & TITANS_FLAG_CHUNK_SCAN)) {
+        e = titans::launch_linear_scan(a, m->nseg_max, st);
     } else if (phased_eligible(m->cfg, chunk)) {
         e = titans::launch_chunk_tc_phased(a, m->status + 2, st);
     } else {

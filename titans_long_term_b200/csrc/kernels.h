@@ -42,6 +42,10 @@ size_t chunk_tc_mlp64_smem_bytes();
 size_t deep_ws_floats(int d, int h, int layers, int n);
 __host__ __device__ size_t deep_state_floats(int d, int h, int layers);
 cudaError_t launch_chunk_deep_cuda_cores(const ForwardArgs& a, int layers, cudaStream_t st);
+// Linear memory by the cross-chunk scan: up to nseg_max segments per unit, each needing
+// linear_scan_slot_floats(d, chunk) floats of workspace (a.ws, a.ws_per_unit floats per unit).
+size_t linear_scan_slot_floats(int d, int n);
+cudaError_t launch_linear_scan(const ForwardArgs& a, int nseg_max, cudaStream_t st);
 size_t tc_phased_ws_bytes_per_unit();
 bool tc_phased_supported(int d, int h, int chunk);
 cudaError_t launch_chunk_tc_phased(const ForwardArgs& a, unsigned* sync, cudaStream_t st);

@@ -1,0 +1,259 @@
+// Cross-chunk scan of the linear memory M(x) = W x ("Titans: Learning to Memorize at Test Time":
+// walk-through sec. 3.2; the German summary's "Parallelisiertes Training" and the tencent review
+// name parallel associative scans for the recurrent part).
+//
+// One chunk of the linear memory is an affine map of the row state X = [W | S] (d x 2d):
+//   X' = X M + N,  M = [[A I - 2 K^T C K, -2 K^T D K], [sigma I, E I]],  N = [2 V^T C K, 2 V^T D K],
+// (K, V the chunk's keys and values as rows, C = diag(c), D = diag(d) from the gate scan), so the
+// chunks of a stream combine associatively and a single long stream can use many SMs:
+//   1. compose: each segment of G chunks composes its chunks' maps. Appending a chunk to a composed
+//      map (M, N) multiplies every row of [M; N] by the chunk's map, which is the ordinary chunk
+//      update applied to a 3d-row state whose first 2d rows (M) see v = 0 and last d rows (N) see
+//      v: started from [I; 0], one CTA per (unit, segment);
+//   2. scan: per unit, X_{s+1} = X_s M_s + N_s over the segments, in order (one CTA per unit);
+//   3. run: each segment runs its chunks from X_s, writing y_t = W q_t with the chunk-start W (one
+//      CTA per (unit, segment)); the last segment hands the final W, S back.
+// fp32 arithmetic on CUDA cores; k, q, v, y in fp32 or bf16.
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "kernels.h"
+
+namespace titans {
+
+namespace {
+
+__device__ __forceinline__ float ldx(const float* p) { return *p; }
+__device__ __forceinline__ float ldx(const __nv_bfloat16* p) { return __bfloat162float(*p); }
+__device__ __forceinline__ void stx(float* p, float v) { *p = v; }
+__device__ __forceinline__ void stx(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
+
+constexpr int kScanThreads = 256;
+constexpr int kScanMaxChunk = 128;
+
+// Per (unit, segment) workspace slot, in floats: R [3d][2d], P [3d][n], X [d][2d], G [n][d].
+__host__ __device__ inline size_t slot_floats(int d, int n) {
+    return (size_t)6 * d * d + (size_t)3 * d * n + (size_t)2 * d * d + (size_t)n * d;
+}
+
+// The chunk's gate scan (division-free suffix scan) into shared memory: c, d, and A, E, sigma.
+__device__ void chunk_scan(const float* alpha, const float* eta, const float* theta, long t0, int n, int chunk,
+                           int chunk_gates, float* s_a, float* s_e, float* s_t, float* s_c, float* s_d, float* s_scal) {
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        const long gi = chunk_gates ? t0 / chunk : t0 + i;
+        s_a[i] = alpha[gi];
+        s_e[i] = eta[gi];
+        s_t[i] = theta[gi];
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float Pr = 1.f, Qr = 1.f, r_next = 0.f;
+        for (int j = n - 1; j >= 0; --j) {
+            const float r = Pr + (j + 1 < n ? s_e[j + 1] * r_next : 0.f);
+            s_c[j] = s_t[j] * r;
+            s_d[j] = s_t[j] * Qr;
+            r_next = r;
+            Pr *= 1.f - s_a[j];
+            Qr *= s_e[j];
+        }
+        s_scal[0] = Pr;
+        s_scal[1] = Qr;
+        s_scal[2] = s_e[0] * r_next;
+    }
+    __syncthreads();
+}
+
+}  // namespace
+
+size_t linear_scan_slot_floats(int d, int n) { return slot_floats(d, n); }
+
+// 1. compose the maps of segment s of unit u (blockIdx = u * nseg + s).
+template <typename Tin>
+__global__ void __launch_bounds__(kScanThreads) linear_scan_compose(
+    int d, long T, long gate_ld, int chunk, int chunk_gates, int nseg, int G, const Tin* __restrict__ k,
+    const Tin* __restrict__ v, const float* __restrict__ alpha, const float* __restrict__ eta,
+    const float* __restrict__ theta, float* __restrict__ ws, size_t ws_per_unit) {
+    __shared__ float s_a[kScanMaxChunk], s_e[kScanMaxChunk], s_t[kScanMaxChunk], s_c[kScanMaxChunk],
+        s_d[kScanMaxChunk], s_scal[3];
+    const long u = blockIdx.x / nseg;
+    const int s = blockIdx.x % nseg, tid = threadIdx.x;
+    float* R = ws + u * ws_per_unit + (size_t)s * slot_floats(d, chunk);
+    float* P = R + (size_t)6 * d * d;
+    const int d2 = 2 * d, rows = 3 * d;
+    for (int idx = tid; idx < rows * d2; idx += blockDim.x) {
+        const int r = idx / d2, col = idx % d2;
+        R[idx] = (r < d2 && col == r) ? 1.f : 0.f;
+    }
+    __syncthreads();
+    k += u * T * d;
+    v += u * T * d;
+    alpha += u * gate_ld;
+    eta += u * gate_ld;
+    theta += u * gate_ld;
+    const int nch = (int)((T + chunk - 1) / chunk);
+    const int c1 = min(nch, (s + 1) * G);
+    for (int c = s * G; c < c1; ++c) {
+        const long t0 = (long)c * chunk;
+        const int n = (int)min((long)chunk, T - t0);
+        chunk_scan(alpha, eta, theta, t0, n, chunk, chunk_gates, s_a, s_e, s_t, s_c, s_d, s_scal);
+        const float An = s_scal[0], En = s_scal[1], sig = s_scal[2];
+        const Tin* K = k + t0 * d;
+        const Tin* V = v + t0 * d;
+        // P[r][t] = (row r of the W part) . k_t  - (v_t's component for the N rows)
+        for (int idx = tid; idx < rows * n; idx += blockDim.x) {
+            const int r = idx / n, t = idx % n;
+            float p = 0.f;
+            const float* Rr = R + (size_t)r * d2;
+            for (int m = 0; m < d; ++m) p += Rr[m] * ldx(K + (size_t)t * d + m);
+            if (r >= d2) p -= ldx(V + (size_t)t * d + (r - d2));
+            P[idx] = p;
+        }
+        __syncthreads();
+        for (int idx = tid; idx < rows * d; idx += blockDim.x) {
+            const int r = idx / d, m = idx % d;
+            float uc = 0.f, ud = 0.f;
+            for (int t = 0; t < n; ++t) {
+                const float g = P[(size_t)r * n + t] * ldx(K + (size_t)t * d + m);
+                uc += s_c[t] * g;
+                ud += s_d[t] * g;
+            }
+            float* Rr = R + (size_t)r * d2;
+            const float w = Rr[m], sv = Rr[d + m];
+            Rr[m] = An * w + sig * sv - 2.f * uc;
+            Rr[d + m] = En * sv - 2.f * ud;
+        }
+        __syncthreads();
+    }
+}
+
+// 2. per unit: X_0 = [W | S], X_{s+1} = X_s M_s + N_s (M_s = R_s rows 0..2d-1, N_s = rows 2d..3d-1).
+__global__ void __launch_bounds__(kScanThreads) linear_scan_segments(int d, int chunk, int nseg_used, int nseg,
+                                                                   const float* __restrict__ W,
+                                                                   const float* __restrict__ S,
+                                                                   float* __restrict__ ws, size_t ws_per_unit) {
+    const long u = blockIdx.x;
+    const int d2 = 2 * d;
+    const size_t slot = slot_floats(d, chunk);
+    float* base = ws + u * ws_per_unit;
+    auto Xof = [&](int s) { return base + (size_t)s * slot + (size_t)6 * d * d + (size_t)3 * d * chunk; };
+    float* X0 = Xof(0);
+    for (int idx = threadIdx.x; idx < d * d2; idx += blockDim.x) {
+        const int i = idx / d2, j = idx % d2;
+        X0[idx] = j < d ? W[u * d * d + (size_t)i * d + j] : S[u * d * d + (size_t)i * d + (j - d)];
+    }
+    __syncthreads();
+    for (int s = 0; s + 1 < nseg_used; ++s) {
+        const float* Xs = Xof(s);
+        const float* R = base + (size_t)s * slot;
+        float* Xn = Xof(s + 1);
+        for (int idx = threadIdx.x; idx < d * d2; idx += blockDim.x) {
+            const int i = idx / d2, j = idx % d2;
+            float acc = R[(size_t)(d2 + i) * d2 + j];  // N_s[i][j]
+            for (int r = 0; r < d2; ++r) acc += Xs[(size_t)i * d2 + r] * R[(size_t)r * d2 + j];
+            Xn[idx] = acc;
+        }
+        __syncthreads();
+    }
+    (void)nseg;
+}
+
+// 3. run segment s of unit u from X_s: y for its tokens; the last segment writes the final W, S.
+template <typename Tin>
+__global__ void __launch_bounds__(kScanThreads) linear_scan_run(
+    int d, long T, long gate_ld, int chunk, int chunk_gates, int nseg_used, int G, const Tin* __restrict__ k,
+    const Tin* __restrict__ q, const Tin* __restrict__ v, const float* __restrict__ alpha,
+    const float* __restrict__ eta, const float* __restrict__ theta, float* __restrict__ Wout,
+    float* __restrict__ Sout, Tin* __restrict__ y, const Tin* __restrict__ attn, float* __restrict__ ws,
+    size_t ws_per_unit) {
+    __shared__ float s_a[kScanMaxChunk], s_e[kScanMaxChunk], s_t[kScanMaxChunk], s_c[kScanMaxChunk],
+        s_d[kScanMaxChunk], s_scal[3];
+    const long u = blockIdx.x / nseg_used;
+    const int s = blockIdx.x % nseg_used, tid = threadIdx.x, d2 = 2 * d;
+    float* slotp = ws + u * ws_per_unit + (size_t)s * slot_floats(d, chunk);
+    float* X = slotp + (size_t)6 * d * d + (size_t)3 * d * chunk;  // [d][2d]: W | S, updated in place
+    float* Ge = X + (size_t)2 * d * d;                                // [n][d]
+    k += u * T * d;
+    q += u * T * d;
+    v += u * T * d;
+    y += u * T * d;
+    if (attn) attn += u * T * d;
+    alpha += u * gate_ld;
+    eta += u * gate_ld;
+    theta += u * gate_ld;
+    const int nch = (int)((T + chunk - 1) / chunk);
+    const int c1 = min(nch, (s + 1) * G);
+    for (int c = s * G; c < c1; ++c) {
+        const long t0 = (long)c * chunk;
+        const int n = (int)min((long)chunk, T - t0);
+        chunk_scan(alpha, eta, theta, t0, n, chunk, chunk_gates, s_a, s_e, s_t, s_c, s_d, s_scal);
+        const float An = s_scal[0], En = s_scal[1], sig = s_scal[2];
+        const Tin* K = k + t0 * d;
+        const Tin* Q = q + t0 * d;
+        const Tin* V = v + t0 * d;
+        for (int idx = tid; idx < n * d; idx += blockDim.x) {  // G = 2 (W k - v), y = W q
+            const int t = idx / d, i = idx % d;
+            float yh = 0.f, yq = 0.f;
+            const float* Wr = X + (size_t)i * d2;
+            for (int m = 0; m < d; ++m) {
+                yh += Wr[m] * ldx(K + (size_t)t * d + m);
+                yq += Wr[m] * ldx(Q + (size_t)t * d + m);
+            }
+            Ge[idx] = 2.f * (yh - ldx(V + idx));
+            const long o = (t0 + t) * d + i;
+            stx(y + o, attn ? ldx(attn + o) / (1.f + expf(-yq)) : yq);
+        }
+        __syncthreads();
+        for (int idx = tid; idx < d * d; idx += blockDim.x) {
+            const int i = idx / d, m = idx % d;
+            float uc = 0.f, ud = 0.f;
+            for (int t = 0; t < n; ++t) {
+                const float g = Ge[(size_t)t * d + i] * ldx(K + (size_t)t * d + m);
+                uc += s_c[t] * g;
+                ud += s_d[t] * g;
+            }
+            float* Wr = X + (size_t)i * d2;
+            const float w = Wr[m], sv = Wr[d + m];
+            Wr[m] = An * w + sig * sv - uc;
+            Wr[d + m] = En * sv - ud;
+        }
+        __syncthreads();
+    }
+    if (s == nseg_used - 1) {
+        for (int idx = tid; idx < d * d; idx += blockDim.x) {
+            const int i = idx / d, m = idx % d;
+            Wout[u * d * d + idx] = X[(size_t)i * d2 + m];
+            Sout[u * d * d + idx] = X[(size_t)i * d2 + d + m];
+        }
+    }
+}
+
+template <typename Tin>
+static cudaError_t launch_scan(const ForwardArgs& a, int nseg_max, cudaStream_t st) {
+    const int nch = (int)((a.T + a.chunk - 1) / a.chunk);
+    int nseg = nseg_max < 1 ? 1 : nseg_max;
+    if (nseg > nch) nseg = nch;
+    const int G = (nch + nseg - 1) / nseg;
+    const int used = (nch + G - 1) / G;  // segments that hold chunks
+    const unsigned grid = (unsigned)(a.units * used);
+    linear_scan_compose<Tin><<<grid, kScanThreads, 0, st>>>(a.d, a.T, a.gate_ld, a.chunk, (int)a.chunk_gates, used, G,
+                                                            (const Tin*)a.k, (const Tin*)a.v, a.alpha, a.eta,
+                                                            a.theta, a.ws, a.ws_per_unit);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    linear_scan_segments<<<(unsigned)a.units, kScanThreads, 0, st>>>(a.d, a.chunk, used, used, a.W1, a.S1, a.ws,
+                                                                     a.ws_per_unit);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    linear_scan_run<Tin><<<grid, kScanThreads, 0, st>>>(a.d, a.T, a.gate_ld, a.chunk, (int)a.chunk_gates, used, G,
+                                                        (const Tin*)a.k, (const Tin*)a.q, (const Tin*)a.v, a.alpha,
+                                                        a.eta, a.theta, a.W1, a.S1, (Tin*)a.y, (const Tin*)a.attn,
+                                                        a.ws, a.ws_per_unit);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_linear_scan(const ForwardArgs& a, int nseg_max, cudaStream_t st) {
+    if (a.h != 0 || a.chunk > kScanMaxChunk) return cudaErrorInvalidValue;
+    return a.bf16 ? launch_scan<__nv_bfloat16>(a, nseg_max, st) : launch_scan<float>(a, nseg_max, st);
+}
+
+}  // namespace titans

@@ -20,7 +20,9 @@ OK, EINVAL, EUNSUPPORTED, ECUDA, EDEVICE = 0, 1, 2, 3, 4
 BF16, FP32 = 0, 1
 FLAG_CUDA_CORES = 1
 FLAG_CHUNK_GATES = 2
-PATH_TC_MLP64, PATH_CUDA_CORES, PATH_STEP_CLUSTER, PATH_TC_PHASED, PATH_DEEP_CUDA_CORES = 1, 2, 3, 4, 5
+FLAG_CHUNK_SCAN = 4
+(PATH_TC_MLP64, PATH_CUDA_CORES, PATH_STEP_CLUSTER, PATH_TC_PHASED, PATH_DEEP_CUDA_CORES,
+ PATH_LINEAR_SCAN) = 1, 2, 3, 4, 5, 6
 
 EXPORTED = ["titans_mem_init", "titans_mem_destroy", "titans_mem_forward", "titans_mem_step",
             "titans_mem_path", "titans_mem_sync_status", "titans_last_error_string", "titans_mem_version",
@@ -98,14 +100,15 @@ class Memory:
     2-layer SiLU MLP memory (d_hidden = 4d)."""
 
     def __init__(self, d: int, d_hidden: int, chunk: int, mode: str, B: int, H: int, cuda_cores: bool = False,
-                 layers: Optional[int] = None, chunk_gates: bool = False):
+                 layers: Optional[int] = None, chunk_gates: bool = False, chunk_scan: bool = False):
         self.d, self.h, self.chunk, self.B, self.H = d, d_hidden, chunk, B, H
         self.mode = mode
         self.layers = layers or 2
         self.chunk_gates = chunk_gates
         self.dtype = torch.bfloat16 if mode == "bf16" else torch.float32
         cfg = Config(d, d_hidden, chunk, BF16 if mode == "bf16" else FP32, B, H,
-                     (FLAG_CUDA_CORES if cuda_cores else 0) | (FLAG_CHUNK_GATES if chunk_gates else 0))
+                     (FLAG_CUDA_CORES if cuda_cores else 0) | (FLAG_CHUNK_GATES if chunk_gates else 0) |
+                     (FLAG_CHUNK_SCAN if chunk_scan else 0))
         h = ctypes.c_void_p()
         if layers is None:
             _check(lib().titans_mem_init(ctypes.byref(cfg), ctypes.byref(h)))
