@@ -29,6 +29,12 @@ Two fp64 paths, both from the pages on "Titans: Learning to Memorize at Test Tim
   Training": parallel associative scans; tencent review, the same): segments
   of chunks compose their maps independently, a short scan over the segments
   gives every segment's start state, and each segment then runs its chunks.
+* :func:`backward` -- gradients of a scalar loss on the forward's outputs (y and
+  the final state) with respect to every input (k, q, v, the gates, the initial
+  state), by reverse-mode automatic differentiation in fp64 through the token
+  loop written in plain PyTorch ops (the outer loop of training: walk-through
+  sec. 3.1, W_K and W_V are outer-loop parameters). Pinned by central finite
+  differences of the C token loop.
 * :func:`mag_gate` / :func:`forward_gated` -- the gated output of the
   memory-as-a-gate architecture (walk-through sec. 4.2 "Gated Memory": o = y
   (x) M(x~), y the sliding-window attention branch's output; the tencent review's
@@ -396,3 +402,60 @@ def forward_linear_scan(k, q, v, alpha, eta, theta, state: Dict, chunk: int, seg
             X = X @ Ms + Ns
         W[u], S[u] = X[:, :d], X[:, d:]
     return y, {"W1": W, "S1": S}
+
+
+def _torch_token_loop(k, q, v, alpha, eta, theta, state, chunk):
+    """The defining recurrence in fp64 torch ops (differentiable): the same steps as the C token
+    loop, with the per-token gradient written out (linear: 2 (W k - v) k^T; MLP: the chain rule)."""
+    import torch
+    U, T, d = k.shape
+    linear = "W2" not in state
+    W1, S1 = state["W1"], state["S1"]
+    W2, S2 = (None, None) if linear else (state["W2"], state["S2"])
+    ys = []
+    for t in range(T):
+        if t % chunk == 0:
+            W1b, W2b = W1, W2
+        kt, qt, vt = k[:, t], q[:, t], v[:, t]
+        if linear:
+            ys.append(torch.einsum("uij,uj->ui", W1b, qt))
+            e = 2.0 * (torch.einsum("uij,uj->ui", W1b, kt) - vt)
+            g1 = e[:, :, None] * kt[:, None, :]
+        else:
+            zq = torch.einsum("uij,uj->ui", W1b, qt)
+            ys.append(torch.einsum("uij,uj->ui", W2b, zq * torch.sigmoid(zq)))
+            z = torch.einsum("uij,uj->ui", W1b, kt)
+            s_ = torch.sigmoid(z)
+            a = z * s_
+            e = 2.0 * (torch.einsum("uij,uj->ui", W2b, a) - vt)
+            g2 = e[:, :, None] * a[:, None, :]
+            delta = torch.einsum("uij,ui->uj", W2b, e) * s_ * (1.0 + z * (1.0 - s_))
+            g1 = delta[:, :, None] * kt[:, None, :]
+        at, et_, tt = alpha[:, t, None, None], eta[:, t, None, None], theta[:, t, None, None]
+        S1 = et_ * S1 - tt * g1
+        W1 = (1.0 - at) * W1 + S1
+        if not linear:
+            S2 = et_ * S2 - tt * g2
+            W2 = (1.0 - at) * W2 + S2
+    out = {"W1": W1, "S1": S1}
+    if not linear:
+        out.update(W2=W2, S2=S2)
+    return torch.stack(ys, 1), out
+
+
+def backward(k, q, v, alpha, eta, theta, state: Dict, chunk: int, dy, dstate: Dict):
+    """Gradients of L = <dy, y> + sum_n <dstate[n], final state[n]> with respect to k, q, v, alpha,
+    eta, theta and the initial state, in fp64 (reverse mode through the token loop). Returns a dict
+    with keys k, q, v, alpha, eta, theta and the state's names (W1, S1, W2, S2)."""
+    import torch
+    f64 = lambda x: torch.as_tensor(np.asarray(_np(x, np.float64)), dtype=torch.float64).clone().requires_grad_(True)
+    ins = {n: f64(x) for n, x in (("k", k), ("q", q), ("v", v), ("alpha", alpha), ("eta", eta), ("theta", theta))}
+    st = {n: f64(x) for n, x in state.items()}
+    y, out = _torch_token_loop(ins["k"], ins["q"], ins["v"], ins["alpha"], ins["eta"], ins["theta"], st, chunk)
+    L = (y * torch.as_tensor(_np(dy, np.float64))).sum()
+    for n, g in dstate.items():
+        L = L + (out[n] * torch.as_tensor(_np(g, np.float64))).sum()
+    L.backward()
+    grads = {n: x.grad.numpy() for n, x in ins.items()}
+    grads.update({n: x.grad.numpy() for n, x in st.items()})
+    return grads
