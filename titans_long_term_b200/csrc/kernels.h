@@ -46,6 +46,20 @@ cudaError_t launch_chunk_deep_cuda_cores(const ForwardArgs& a, int layers, cudaS
 // linear_scan_slot_floats(d, chunk) floats of workspace (a.ws, a.ws_per_unit floats per unit).
 size_t linear_scan_slot_floats(int d, int n);
 cudaError_t launch_linear_scan(const ForwardArgs& a, int nseg_max, cudaStream_t st);
+// Backward of the chunked linear memory (see linear_backward.cu).
+struct LinearBackwardArgs {
+    int d, chunk;
+    long units, T;
+    bool bf16;
+    const void *k, *q, *v, *dy;
+    const float *alpha, *eta, *theta, *W0, *S0, *dWT, *dST;  // dWT, dST may be NULL (zero)
+    void *dk, *dq, *dv;
+    float *dalpha, *deta, *dtheta, *dW0, *dS0;
+    float* ws;
+    size_t ws_per_unit;  // floats
+};
+size_t linear_backward_ws_floats(int d, long T, int chunk);
+cudaError_t launch_linear_backward(const LinearBackwardArgs& b, cudaStream_t st);
 size_t tc_phased_ws_bytes_per_unit();
 bool tc_phased_supported(int d, int h, int chunk);
 cudaError_t launch_chunk_tc_phased(const ForwardArgs& a, unsigned* sync, cudaStream_t st);

@@ -27,7 +27,8 @@ FLAG_CHUNK_SCAN = 4
 EXPORTED = ["titans_mem_init", "titans_mem_destroy", "titans_mem_forward", "titans_mem_step",
             "titans_mem_path", "titans_mem_sync_status", "titans_last_error_string", "titans_mem_version",
             "titans_mem_forward_noalloc", "titans_mem_forward_host", "titans_mem_forward_gated",
-            "titans_mem_step_gated", "titans_mem_init_deep", "titans_mem_forward_deep"]
+            "titans_mem_step_gated", "titans_mem_init_deep", "titans_mem_forward_deep", "titans_mem_backward",
+            "titans_mem_backward_workspace_bytes"]
 
 
 class TitansError(RuntimeError):
@@ -70,12 +71,16 @@ def lib():
         L.titans_mem_step_gated.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
         L.titans_mem_init_deep.argtypes = [ctypes.POINTER(Config), i, ctypes.POINTER(vp)]
         L.titans_mem_forward_deep.argtypes = [vp, vp, vp, vp, vp, vp, vp, l, i, vp, vp, vp, vp, vp]
+        L.titans_mem_backward_workspace_bytes.argtypes = [vp, l, i]
+        L.titans_mem_backward_workspace_bytes.restype = ctypes.c_size_t
+        L.titans_mem_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, l, i, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                          vp, vp, vp, vp, ctypes.c_size_t, vp]
         L.titans_mem_sync_status.argtypes = [vp, vp]
         L.titans_last_error_string.restype = ctypes.c_char_p
         for f in ("titans_mem_init", "titans_mem_destroy", "titans_mem_forward", "titans_mem_step",
                   "titans_mem_path", "titans_mem_sync_status", "titans_mem_version", "titans_mem_forward_noalloc",
                   "titans_mem_forward_host", "titans_mem_forward_gated", "titans_mem_step_gated",
-                  "titans_mem_init_deep", "titans_mem_forward_deep"):
+                  "titans_mem_init_deep", "titans_mem_forward_deep", "titans_mem_backward"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -191,6 +196,31 @@ class Memory:
                                              T, chunk or self.chunk, _ptr(state["W"]), _ptr(state["S"]), _ptr(attn),
                                              _ptr(y), _stream(stream)))
         return y
+
+    def backward(self, k, q, v, alpha, eta, theta, state: Dict[str, torch.Tensor], dy: torch.Tensor,
+                 dstate: Optional[Dict[str, torch.Tensor]] = None, chunk: Optional[int] = None,
+                 stream=None) -> Dict[str, torch.Tensor]:
+        """Linear memory: gradients of <dy, y> + <dW, W_T> + <dS, S_T> (dstate {"W1", "S1"}, optional)
+        with respect to k, q, v, the gates and the initial state {"W1", "S1"} (read only). Returns a
+        dict k, q, v, alpha, eta, theta, W1, S1."""
+        T = k.shape[-2]
+        chunk = chunk or self.chunk
+        self._check_tensors({"k": k, "q": q, "v": v, "dy": dy}, {"alpha": alpha, "eta": eta, "theta": theta},
+                            state, torch.empty_like(k), (self.B, self.H, T), chunk)
+        out = {n: torch.empty_like(x) for n, x in (("k", k), ("q", q), ("v", v), ("alpha", alpha), ("eta", eta),
+                                                   ("theta", theta))}
+        out["W1"] = torch.empty_like(state["W1"])
+        out["S1"] = torch.empty_like(state["S1"])
+        nbytes = lib().titans_mem_backward_workspace_bytes(self._h, T, chunk)
+        ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=k.device)
+        dstate = dstate or {}
+        _check(lib().titans_mem_backward(self._h, _ptr(k), _ptr(q), _ptr(v), _ptr(alpha), _ptr(eta), _ptr(theta), T,
+                                         chunk, _ptr(state["W1"]), _ptr(state["S1"]), _ptr(dy),
+                                         _ptr(dstate.get("W1")), _ptr(dstate.get("S1")), _ptr(out["k"]),
+                                         _ptr(out["q"]), _ptr(out["v"]), _ptr(out["alpha"]), _ptr(out["eta"]),
+                                         _ptr(out["theta"]), _ptr(out["W1"]), _ptr(out["S1"]), _ptr(ws), nbytes,
+                                         _stream(stream)))
+        return out
 
     def forward_host(self, k, q, v, alpha, eta, theta, state: Dict[str, torch.Tensor], y: torch.Tensor,
                      staging: Dict[str, torch.Tensor], chunk: Optional[int] = None, t_seg: int = 0,
