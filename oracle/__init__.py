@@ -456,6 +456,9 @@ def backward(k, q, v, alpha, eta, theta, state: Dict, chunk: int, dy, dstate: Di
     for n, g in dstate.items():
         L = L + (out[n] * torch.as_tensor(_np(g, np.float64))).sum()
     L.backward()
-    grads = {n: x.grad.numpy() for n, x in ins.items()}
-    grads.update({n: x.grad.numpy() for n, x in st.items()})
+    # an input the loss does not depend on (e.g. the initial momentum when only the first chunk's y
+    # is scored) has no .grad: its gradient is zero
+    g = lambda x: x.grad.numpy() if x.grad is not None else np.zeros(tuple(x.shape))
+    grads = {n: g(x) for n, x in ins.items()}
+    grads.update({n: g(x) for n, x in st.items()})
     return grads

@@ -61,3 +61,13 @@ def test_backward_of_a_frozen_memory():
     for t in range(T):
         Wc = beta[(t // chunk) * chunk] * st["W1"][0]
         np.testing.assert_allclose(g["q"][0, t], Wc.T @ dy[0, t], rtol=1e-12, atol=1e-14)
+
+
+def test_backward_of_an_input_the_loss_ignores_is_zero():
+    """One chunk, loss on y only: y reads the initial weights, never the initial momentum, so the
+    momentum's gradient is exactly zero (returned as zeros, not missing)."""
+    k, q, v, al, et, th, st = _mk(1, 6, 3, 4, 97)
+    dy = np.random.default_rng(5).standard_normal((1, 6, 3))
+    g = oracle.backward(k, q, v, al, et, th, st, 6, dy, {})
+    assert g["S1"].shape == st["S1"].shape and not g["S1"].any() and not g["S2"].any()
+    assert np.abs(g["W1"]).max() > 0
