@@ -254,27 +254,32 @@ titans_status_t titans_mem_forward_noalloc(const titans_mem_config *cfg, const v
                                            float *S1, float *S2, void *y, void *stream);
 
 /*
- * Backward of the chunk-wise forward of a LINEAR memory (the outer loop of training: the walk-
- * through's sec. 3.1 makes the projections that produce k, v, q outer-loop parameters; the memory's
- * forward is defined by sec. 3.1-3.2). For L = <dy, y> + <dW, W_T> + <dS, S_T>, with y and the final
- * state W_T, S_T those of titans_mem_forward on the same inputs and initial state, it writes
+ * Backward of the chunk-wise forward (the outer loop of training: the walk-through's sec. 3.1
+ * makes the projections that produce k, v, q outer-loop parameters; the memory's forward is
+ * defined by sec. 3.1-3.2), for the linear and the 2-layer MLP memory. For
+ *   L = <dy, y> + <dW1, W1_T> + <dW2, W2_T> + <dS1, S1_T> + <dS2, S2_T>,
+ * with y and the final state those of titans_mem_forward on the same inputs and initial state
+ * (W1, W2, S1, S2 as in titans_mem_forward, read only; W2, S2, dW2, dS2, dW2_0, dS2_0 NULL for
+ * the linear memory), it writes
  *   dk, dq, dv  [B, H, T, d] (dtype of k)      dL/dk, dL/dq, dL/dv
  *   dalpha, deta, dtheta [B, H, T] fp32        dL/d the gates
- *   dW0, dS0 [B, H, d, d] fp32                 dL/d the initial state
- * from k, q, v, the gates and the initial state W, S (read only) and the upstream dy [B, H, T, d]
- * (dtype of k) and dW, dS [B, H, d, d] (NULL = zero). It reruns the forward, keeping every
- * chunk-start state in `workspace` (caller-owned device memory of at least
- * titans_mem_backward_workspace_bytes(m, T, chunk) bytes, 16-byte aligned), then walks the chunks
- * backwards. Per-token gates only. Returns TITANS_EUNSUPPORTED for an MLP or deep memory or with
+ *   dW1_0, dW2_0, dS1_0, dS2_0 (shapes of W1..S2) fp32  dL/d the initial state
+ * from the upstream dy [B, H, T, d] (dtype of k) and dW1, dW2, dS1, dS2 (NULL = zero). It reruns
+ * the forward, keeping every chunk-start state in `workspace` (caller-owned device memory of at
+ * least titans_mem_backward_workspace_bytes(m, T, chunk) bytes, 16-byte aligned), then walks the
+ * chunks backwards (fp32 on CUDA cores; the MLP's adjoint includes the second-order terms of the
+ * inner gradient). Per-token gates only. Returns TITANS_EUNSUPPORTED for a deep memory or with
  * TITANS_FLAG_CHUNK_GATES, TITANS_EINVAL for a NULL or misaligned pointer or a small workspace.
  */
 size_t titans_mem_backward_workspace_bytes(titans_mem_t m, long T, int chunk);
 titans_status_t titans_mem_backward(titans_mem_t m, const void *k, const void *q, const void *v,
                                     const float *alpha, const float *eta, const float *theta, long T,
-                                    int chunk, const float *W, const float *S, const void *dy,
-                                    const float *dW, const float *dS, void *dk, void *dq, void *dv,
-                                    float *dalpha, float *deta, float *dtheta, float *dW0, float *dS0,
-                                    void *workspace, size_t workspace_bytes, void *stream);
+                                    int chunk, const float *W1, const float *W2, const float *S1,
+                                    const float *S2, const void *dy, const float *dW1, const float *dW2,
+                                    const float *dS1, const float *dS2, void *dk, void *dq, void *dv,
+                                    float *dalpha, float *deta, float *dtheta, float *dW1_0,
+                                    float *dW2_0, float *dS1_0, float *dS2_0, void *workspace,
+                                    size_t workspace_bytes, void *stream);
 
 /* Kernel that titans_mem_forward (step = 0) or titans_mem_step (step = 1) would run with
  * this chunk length; negative on an unsupported combination. */

@@ -56,7 +56,49 @@ def test_linear_backward_matches_the_oracle(d, B, H, T, chunk, mode, with_dstate
     print(f"backward d={d} T={T} chunk={chunk} {mode}:", {k: f"{v:.1e}" for k, v in worst.items()})
 
 
-def test_backward_leaves_its_inputs_alone_and_rejects_the_mlp():
+def _mlp_case(B, H, T, chunk, mode, seed, with_dstate, recipe=None):
+    w = synth.WORKLOADS["mlp-d64-b2h4-t2k"]
+    inp = synth.make_inputs(w, units=range(B * H), T=T, dtype=mode, recipe=recipe)
+    U = B * H
+    g = torch.Generator().manual_seed(seed)
+    inp["S1"] = torch.randn(*inp["S1"].shape, generator=g) * 0.01  # a non-zero momentum, every term exercised
+    inp["S2"] = torch.randn(*inp["S2"].shape, generator=g) * 0.01
+    dy = torch.randn(U, T, 64, generator=g).to(inp["k"].dtype)
+    dst = {n: torch.randn(*inp[n].shape, generator=g) for n in ("W1", "W2", "S1", "S2")} if with_dstate else {}
+    return w, inp, dy, dst
+
+
+@pytest.mark.parametrize("B,H,T,chunk,mode,with_dstate,recipe", [
+    (1, 2, 40, 16, "fp32", True, None),       # ragged last chunk
+    (2, 1, 64, 64, "fp32", False, None),      # one chunk, loss on y only
+    (1, 2, 12, 1, "fp32", True, None),        # chunk = 1
+    (1, 2, 64, 32, "fp32", True, "stated"),   # the stated gate ranges
+    (1, 2, 48, 16, "bf16", True, None),       # bf16 token streams
+])
+def test_mlp_backward_matches_the_oracle(B, H, T, chunk, mode, with_dstate, recipe):
+    """The MLP memory's adjoint includes the second-order terms of the inner gradient (its update
+    depends on W through g); against fp64 reverse-mode differentiation of the token loop."""
+    w, inp, dy, dst = _mlp_case(B, H, T, chunk, mode, T + chunk, with_dstate, recipe)
+    U = B * H
+    m = mem.Memory(64, 256, chunk, mode, B, H)
+    dev = lambda x: x.reshape(B, H, *x.shape[1:]).cuda().contiguous()
+    args = [dev(inp[n]) for n in ("k", "q", "v", "alpha", "eta", "theta")]
+    state = {n: dev(inp[n]) for n in ("W1", "W2", "S1", "S2")}
+    out = m.backward(*args, state, dev(dy), {n: dev(x) for n, x in dst.items()}, chunk=chunk)
+    m.sync_status()
+    ref = oracle.backward(inp["k"], inp["q"], inp["v"], inp["alpha"], inp["eta"], inp["theta"],
+                          {n: inp[n] for n in ("W1", "W2", "S1", "S2")}, chunk, dy.float(), dst)
+    worst = {}
+    for n in ("k", "q", "v", "alpha", "eta", "theta", "W1", "W2", "S1", "S2"):
+        x = out[n].reshape(U, -1).float().cpu().numpy()
+        e = rel_err(x, ref[n].reshape(U, -1))
+        worst[n] = float(e.max())
+        assert np.isfinite(x).all(), n
+        assert e.max() <= TOL[mode], f"d{n}: {e.max():.3e} > {TOL[mode]}"
+    print(f"MLP backward T={T} chunk={chunk} {mode} {recipe}:", {k: f"{v:.1e}" for k, v in worst.items()})
+
+
+def test_backward_leaves_its_inputs_alone_and_rejects_a_deep_memory():
     w, inp, dy, dst = _case(64, 1, 1, 32, 16, "fp32", 5, True)
     m = mem.Memory(64, 0, 16, "fp32", 1, 1)
     dev = lambda x, *s: x.reshape(1, 1, *s).cuda().contiguous()
@@ -66,10 +108,10 @@ def test_backward_leaves_its_inputs_alone_and_rejects_the_mlp():
                state, dev(dy, 32, 64), {n: dev(x, 64, 64) for n, x in dst.items()})
     m.sync_status()
     assert all(torch.equal(before[n], state[n]) for n in state)
-    mm = mem.Memory(64, 256, 16, "fp32", 1, 1)
+    deep = mem.Memory(64, 256, 16, "fp32", 1, 1, layers=3)
     with pytest.raises(mem.TitansError) as ei:
         z = torch.zeros(1, 1, 8, 64, device="cuda")
         gz = torch.zeros(1, 1, 8, device="cuda")
-        mm.backward(z, z, z, gz, gz, gz, {"W1": torch.zeros(1, 1, 256, 64, device="cuda"),
-                                          "S1": torch.zeros(1, 1, 256, 64, device="cuda")}, z)
+        deep.backward(z, z, z, gz, gz, gz, {"W1": torch.zeros(1, 1, 256, 64, device="cuda"),
+                                            "S1": torch.zeros(1, 1, 256, 64, device="cuda")}, z)
     assert ei.value.status == mem.EUNSUPPORTED

@@ -102,3 +102,18 @@ def test_deep_forward_rejects_null_handle():
     L = mem.lib()
     rc = L.titans_mem_forward_deep(None, None, None, None, None, None, None, 16, 16, None, None, None, None, None)
     assert rc == mem.EINVAL
+
+
+def test_binding_argument_counts_match_the_header():
+    """Every function the binding declares takes as many arguments as the header says."""
+    src = open(os.path.join(ROOT, "include", "titans_mem.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    L = mem.lib()
+    for name, params in re.findall(r"\b(titans_[a-z_]+)\s*\(([^;{]*?)\)\s*;", src):
+        params = params.strip()
+        n = 0 if params in ("", "void") else params.count(",") + 1
+        argtypes = getattr(L, name).argtypes
+        if argtypes is None:
+            assert n == 0, f"{name}: the header declares {n} parameters, the binding none"
+            continue
+        assert len(argtypes) == n, f"{name}: header {n} parameters, binding {len(argtypes)}"

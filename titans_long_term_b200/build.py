@@ -16,7 +16,7 @@ BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libtitans_mem.so")
 SOURCES = ["api.cu", "chunk_cuda_cores.cu", "chunk_deep_cuda_cores.cu", "chunk_tc_mlp64.cu", "chunk_tc_phased.cu",
            "step_cluster.cu", "forward_noalloc.cu", "linear_scan.cu",
-           "linear_backward.cu"]
+           "linear_backward.cu", "mlp_backward.cu"]
 HEADERS = ["kernels.h", "ptx.cuh"]
 NVCC = os.environ.get("NVCC", "nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -452,29 +452,38 @@ titans_status_t titans_mem_step_gated(titans_mem_t m, const void* k, const void*
 
 size_t titans_mem_backward_workspace_bytes(titans_mem_t m, long T, int chunk) {
     if (!m || T < 1 || chunk < 1) return 0;
-    const size_t per_unit = (titans::linear_backward_ws_floats(m->cfg.d, T, chunk) + 63) & ~size_t(63);
+    const size_t f = m->cfg.d_hidden ? titans::mlp_backward_ws_floats(m->cfg.d, m->cfg.d_hidden, T, chunk)
+                                     : titans::linear_backward_ws_floats(m->cfg.d, T, chunk);
+    const size_t per_unit = (f + 63) & ~size_t(63);
     return per_unit * sizeof(float) * (size_t)m->cfg.B * m->cfg.H;
 }
 
 titans_status_t titans_mem_backward(titans_mem_t m, const void* k, const void* q, const void* v, const float* alpha,
-                                    const float* eta, const float* theta, long T, int chunk, const float* W,
-                                    const float* S, const void* dy, const float* dW, const float* dS, void* dk,
-                                    void* dq, void* dv, float* dalpha, float* deta, float* dtheta, float* dW0,
-                                    float* dS0, void* workspace, size_t workspace_bytes, void* stream) {
+                                    const float* eta, const float* theta, long T, int chunk, const float* W1,
+                                    const float* W2, const float* S1, const float* S2, const void* dy,
+                                    const float* dW1, const float* dW2, const float* dS1, const float* dS2, void* dk,
+                                    void* dq, void* dv, float* dalpha, float* deta, float* dtheta, float* dW1_0,
+                                    float* dW2_0, float* dS1_0, float* dS2_0, void* workspace, size_t workspace_bytes,
+                                    void* stream) {
     if (!m) return fail(TITANS_EINVAL, "handle is NULL");
-    if (m->cfg.d_hidden != 0 || m->layers > 2)
-        return fail(TITANS_EUNSUPPORTED, "the backward is built for the linear memory only");
-    if (m->cfg.flags & TITANS_FLAG_CHUNK_GATES)
-        return fail(TITANS_EUNSUPPORTED, "the backward takes per-token gates");
-    const void* req[] = {k, q, v, W, S, dy, dk, dq, dv, dW0, dS0, workspace};
-    const char* names[] = {"k", "q", "v", "W", "S", "dy", "dk", "dq", "dv", "dW0", "dS0", "workspace"};
+    if (m->layers > 2) return fail(TITANS_EUNSUPPORTED, "the backward is built for the linear and the 2-layer memory");
+    if (m->cfg.flags & TITANS_FLAG_CHUNK_GATES) return fail(TITANS_EUNSUPPORTED, "the backward takes per-token gates");
+    const bool mlp = m->cfg.d_hidden != 0;
+    const void* req[] = {k, q, v, W1, S1, dy, dk, dq, dv, dW1_0, dS1_0, workspace};
+    const char* names[] = {"k", "q", "v", "W1", "S1", "dy", "dk", "dq", "dv", "dW1_0", "dS1_0", "workspace"};
     for (int i = 0; i < 12; ++i) {
         if (!req[i]) return fail(TITANS_EINVAL, std::string(names[i]) + " is NULL");
         if (!aligned16(req[i])) return fail(TITANS_EINVAL, std::string(names[i]) + " is not 16-byte aligned");
     }
+    if (mlp) {
+        const void* req2[] = {W2, S2, dW2_0, dS2_0};
+        for (const void* p : req2)
+            if (!p || !aligned16(p)) return fail(TITANS_EINVAL, "W2, S2, dW2_0, dS2_0 must be non-NULL and 16-byte aligned");
+    }
     const float* g4[] = {alpha, eta, theta, dalpha, deta, dtheta};
     for (const float* p : g4)
-        if (!p || (reinterpret_cast<uintptr_t>(p) & 3u)) return fail(TITANS_EINVAL, "gates and their gradients: NULL or misaligned");
+        if (!p || (reinterpret_cast<uintptr_t>(p) & 3u))
+            return fail(TITANS_EINVAL, "the gates and their gradients must be non-NULL and 4-byte aligned");
     if (T < 1) return fail(TITANS_EINVAL, "T must be >= 1");
     if (T * (long)m->cfg.d >= (1L << 31)) return fail(TITANS_EUNSUPPORTED, "T * d must be below 2^31");
     if (chunk < 1 || chunk > m->cfg.chunk) return fail(TITANS_EUNSUPPORTED, "chunk must be in 1..config.chunk");
@@ -482,34 +491,74 @@ titans_status_t titans_mem_backward(titans_mem_t m, const void* k, const void* q
     if (workspace_bytes < need)
         return fail(TITANS_EINVAL, "workspace smaller than titans_mem_backward_workspace_bytes(): " +
                                        std::to_string(workspace_bytes) + " < " + std::to_string(need));
-    titans::LinearBackwardArgs b{};
-    b.d = m->cfg.d;
-    b.chunk = chunk;
-    b.units = (long)m->cfg.B * m->cfg.H;
-    b.T = T;
-    b.bf16 = m->cfg.mode == TITANS_BF16;
-    b.k = k;
-    b.q = q;
-    b.v = v;
-    b.dy = dy;
-    b.alpha = alpha;
-    b.eta = eta;
-    b.theta = theta;
-    b.W0 = W;
-    b.S0 = S;
-    b.dWT = dW;
-    b.dST = dS;
-    b.dk = dk;
-    b.dq = dq;
-    b.dv = dv;
-    b.dalpha = dalpha;
-    b.deta = deta;
-    b.dtheta = dtheta;
-    b.dW0 = dW0;
-    b.dS0 = dS0;
-    b.ws = static_cast<float*>(workspace);
-    b.ws_per_unit = need / sizeof(float) / (size_t)b.units;
-    cudaError_t e = titans::launch_linear_backward(b, static_cast<cudaStream_t>(stream));
+    const long units = (long)m->cfg.B * m->cfg.H;
+    cudaError_t e;
+    if (mlp) {
+        titans::MlpBackwardArgs b{};
+        b.d = m->cfg.d;
+        b.h = m->cfg.d_hidden;
+        b.chunk = chunk;
+        b.units = units;
+        b.T = T;
+        b.bf16 = m->cfg.mode == TITANS_BF16;
+        b.k = k;
+        b.q = q;
+        b.v = v;
+        b.dy = dy;
+        b.alpha = alpha;
+        b.eta = eta;
+        b.theta = theta;
+        b.W1 = W1;
+        b.W2 = W2;
+        b.S1 = S1;
+        b.S2 = S2;
+        b.dW1 = dW1;
+        b.dW2 = dW2;
+        b.dS1 = dS1;
+        b.dS2 = dS2;
+        b.dk = dk;
+        b.dq = dq;
+        b.dv = dv;
+        b.dalpha = dalpha;
+        b.deta = deta;
+        b.dtheta = dtheta;
+        b.dW1_0 = dW1_0;
+        b.dW2_0 = dW2_0;
+        b.dS1_0 = dS1_0;
+        b.dS2_0 = dS2_0;
+        b.ws = static_cast<float*>(workspace);
+        b.ws_per_unit = need / sizeof(float) / (size_t)units;
+        e = titans::launch_mlp_backward(b, static_cast<cudaStream_t>(stream));
+    } else {
+        titans::LinearBackwardArgs b{};
+        b.d = m->cfg.d;
+        b.chunk = chunk;
+        b.units = units;
+        b.T = T;
+        b.bf16 = m->cfg.mode == TITANS_BF16;
+        b.k = k;
+        b.q = q;
+        b.v = v;
+        b.dy = dy;
+        b.alpha = alpha;
+        b.eta = eta;
+        b.theta = theta;
+        b.W0 = W1;
+        b.S0 = S1;
+        b.dWT = dW1;
+        b.dST = dS1;
+        b.dk = dk;
+        b.dq = dq;
+        b.dv = dv;
+        b.dalpha = dalpha;
+        b.deta = deta;
+        b.dtheta = dtheta;
+        b.dW0 = dW1_0;
+        b.dS0 = dS1_0;
+        b.ws = static_cast<float*>(workspace);
+        b.ws_per_unit = need / sizeof(float) / (size_t)units;
+        e = titans::launch_linear_backward(b, static_cast<cudaStream_t>(stream));
+    }
     if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
     return TITANS_OK;
 }

@@ -59,6 +59,23 @@ struct LinearBackwardArgs {
     size_t ws_per_unit;  // floats
 };
 size_t linear_backward_ws_floats(int d, long T, int chunk);
+// Backward of the chunked 2-layer MLP memory (see mlp_backward.cu).
+struct MlpBackwardArgs {
+    int d, h, chunk;
+    long units, T;
+    bool bf16;
+    const void *k, *q, *v, *dy;
+    const float *alpha, *eta, *theta;
+    const float *W1, *W2, *S1, *S2;       // initial state
+    const float *dW1, *dW2, *dS1, *dS2;   // upstream adjoints of the final state, NULL = zero
+    void *dk, *dq, *dv;
+    float *dalpha, *deta, *dtheta;
+    float *dW1_0, *dW2_0, *dS1_0, *dS2_0;
+    float* ws;
+    size_t ws_per_unit;  // floats
+};
+size_t mlp_backward_ws_floats(int d, int h, long T, int chunk);
+cudaError_t launch_mlp_backward(const MlpBackwardArgs& a, cudaStream_t st);
 cudaError_t launch_linear_backward(const LinearBackwardArgs& b, cudaStream_t st);
 size_t tc_phased_ws_bytes_per_unit();
 bool tc_phased_supported(int d, int h, int chunk);

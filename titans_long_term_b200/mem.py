@@ -73,8 +73,7 @@ def lib():
         L.titans_mem_forward_deep.argtypes = [vp, vp, vp, vp, vp, vp, vp, l, i, vp, vp, vp, vp, vp]
         L.titans_mem_backward_workspace_bytes.argtypes = [vp, l, i]
         L.titans_mem_backward_workspace_bytes.restype = ctypes.c_size_t
-        L.titans_mem_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, l, i, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
-                                          vp, vp, vp, vp, ctypes.c_size_t, vp]
+        L.titans_mem_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, l, i] + [vp] * 20 + [ctypes.c_size_t, vp]
         L.titans_mem_sync_status.argtypes = [vp, vp]
         L.titans_last_error_string.restype = ctypes.c_char_p
         for f in ("titans_mem_init", "titans_mem_destroy", "titans_mem_forward", "titans_mem_step",
@@ -200,26 +199,26 @@ class Memory:
     def backward(self, k, q, v, alpha, eta, theta, state: Dict[str, torch.Tensor], dy: torch.Tensor,
                  dstate: Optional[Dict[str, torch.Tensor]] = None, chunk: Optional[int] = None,
                  stream=None) -> Dict[str, torch.Tensor]:
-        """Linear memory: gradients of <dy, y> + <dW, W_T> + <dS, S_T> (dstate {"W1", "S1"}, optional)
-        with respect to k, q, v, the gates and the initial state {"W1", "S1"} (read only). Returns a
-        dict k, q, v, alpha, eta, theta, W1, S1."""
+        """Gradients of <dy, y> + sum_n <dstate[n], final state[n]> (dstate optional) with respect to
+        k, q, v, the gates and the initial state (read only). Returns a dict with keys k, q, v, alpha,
+        eta, theta and the state's names."""
         T = k.shape[-2]
         chunk = chunk or self.chunk
         self._check_tensors({"k": k, "q": q, "v": v, "dy": dy}, {"alpha": alpha, "eta": eta, "theta": theta},
                             state, torch.empty_like(k), (self.B, self.H, T), chunk)
         out = {n: torch.empty_like(x) for n, x in (("k", k), ("q", q), ("v", v), ("alpha", alpha), ("eta", eta),
                                                    ("theta", theta))}
-        out["W1"] = torch.empty_like(state["W1"])
-        out["S1"] = torch.empty_like(state["S1"])
+        for n in state:
+            out[n] = torch.empty_like(state[n])
         nbytes = lib().titans_mem_backward_workspace_bytes(self._h, T, chunk)
         ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=k.device)
-        dstate = dstate or {}
-        _check(lib().titans_mem_backward(self._h, _ptr(k), _ptr(q), _ptr(v), _ptr(alpha), _ptr(eta), _ptr(theta), T,
-                                         chunk, _ptr(state["W1"]), _ptr(state["S1"]), _ptr(dy),
-                                         _ptr(dstate.get("W1")), _ptr(dstate.get("S1")), _ptr(out["k"]),
-                                         _ptr(out["q"]), _ptr(out["v"]), _ptr(out["alpha"]), _ptr(out["eta"]),
-                                         _ptr(out["theta"]), _ptr(out["W1"]), _ptr(out["S1"]), _ptr(ws), nbytes,
-                                         _stream(stream)))
+        ds = dstate or {}
+        _check(lib().titans_mem_backward(
+            self._h, _ptr(k), _ptr(q), _ptr(v), _ptr(alpha), _ptr(eta), _ptr(theta), T, chunk, _ptr(state["W1"]),
+            _ptr(state.get("W2")), _ptr(state["S1"]), _ptr(state.get("S2")), _ptr(dy), _ptr(ds.get("W1")),
+            _ptr(ds.get("W2")), _ptr(ds.get("S1")), _ptr(ds.get("S2")), _ptr(out["k"]), _ptr(out["q"]), _ptr(out["v"]),
+            _ptr(out["alpha"]), _ptr(out["eta"]), _ptr(out["theta"]), _ptr(out["W1"]), _ptr(out.get("W2")),
+            _ptr(out["S1"]), _ptr(out.get("S2")), _ptr(ws), nbytes, _stream(stream)))
         return out
 
     def forward_host(self, k, q, v, alpha, eta, theta, state: Dict[str, torch.Tensor], y: torch.Tensor,
