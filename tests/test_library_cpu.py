@@ -28,6 +28,16 @@ def test_library_exports_every_declared_symbol():
     assert L.titans_mem_version() == 100
 
 
+def test_debug_library_exports_every_declared_symbol():
+    """The bounds-checked variant (TITANS_DEBUG) has the same C ABI as the release library."""
+    from titans_long_term_b200 import build
+    L = ctypes.CDLL(build.build(debug=True))
+    for name in declared_functions():
+        assert hasattr(L, name), name
+    L.titans_mem_version.restype = ctypes.c_int
+    assert L.titans_mem_version() == 100
+
+
 @pytest.mark.parametrize("d,h,chunk,mode,B,H,status", [
     (96, 0, 16, mem.FP32, 1, 1, mem.EUNSUPPORTED),
     (64, 128, 16, mem.FP32, 1, 1, mem.EUNSUPPORTED),

@@ -1,6 +1,11 @@
 """Build libtitans_mem.so in-tree with nvcc for sm_100a.
 
-    python -m titans_long_term_b200.build [--force] [--verbose-ptxas]
+    python -m titans_long_term_b200.build [--force] [--verbose-ptxas] [--debug]
+
+``--debug`` builds libtitans_mem_debug.so instead, with -DTITANS_DEBUG: the tensor-core kernels then
+check the runtime-dependent coordinates and offsets of their memory accesses and report a failed
+check in the device status word (bit 8) instead of making the access. The binding loads it when the
+environment variable TITANS_DEBUG is 1.
 """
 from __future__ import annotations
 
@@ -14,6 +19,8 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libtitans_mem.so")
+BUILD_DEBUG = os.path.join(HERE, "_build_debug")
+LIB_DEBUG = os.path.join(HERE, "libtitans_mem_debug.so")
 SOURCES = ["api.cu", "chunk_cuda_cores.cu", "chunk_deep_cuda_cores.cu", "chunk_tc_mlp64.cu", "chunk_tc_phased.cu",
            "step_cluster.cu", "forward_noalloc.cu", "linear_scan.cu",
            "linear_backward.cu", "mlp_backward.cu"]
@@ -31,19 +38,21 @@ def _stale(out: str, deps) -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose_ptxas: bool = False) -> str:
-    os.makedirs(BUILD, exist_ok=True)
+def build(force: bool = False, verbose_ptxas: bool = False, debug: bool = False) -> str:
+    build_dir, lib = (BUILD_DEBUG, LIB_DEBUG) if debug else (BUILD, LIB)
+    flags = FLAGS + (["-DTITANS_DEBUG"] if debug else [])
+    os.makedirs(build_dir, exist_ok=True)
     hdrs = [os.path.join(CSRC, h) for h in HEADERS] + [os.path.join(ROOT, "include", "titans_mem.h")]
     jobs = []
     for s in SOURCES:
         src = os.path.join(CSRC, s)
-        obj = os.path.join(BUILD, s.replace(".cu", ".o"))
+        obj = os.path.join(build_dir, s.replace(".cu", ".o"))
         if force or verbose_ptxas or _stale(obj, [src] + hdrs):
-            cmd = [NVCC, *ARCH, *FLAGS, "-c", src, "-o", obj]
+            cmd = [NVCC, *ARCH, *flags, "-c", src, "-o", obj]
             if verbose_ptxas:
                 cmd += ["-Xptxas", "-v"]
             jobs.append(cmd)
-    objs = [os.path.join(BUILD, s.replace(".cu", ".o")) for s in SOURCES]
+    objs = [os.path.join(build_dir, s.replace(".cu", ".o")) for s in SOURCES]
 
     def run(cmd):
         return subprocess.run(cmd, capture_output=True, text=True)
@@ -55,14 +64,15 @@ def build(force: bool = False, verbose_ptxas: bool = False) -> str:
                 raise RuntimeError(f"nvcc failed: {' '.join(cmd)}")
             if verbose_ptxas:
                 sys.stderr.write(res.stderr)
-    if force or jobs or _stale(LIB, objs):
-        cmd = [NVCC, *ARCH, "-shared", "-o", LIB, *objs, "-lcuda"]
+    if force or jobs or _stale(lib, objs):
+        cmd = [NVCC, *ARCH, "-shared", "-o", lib, *objs, "-lcuda"]
         res = subprocess.run(cmd, capture_output=True, text=True)
         if res.returncode != 0:
             sys.stderr.write(res.stdout + res.stderr)
             raise RuntimeError("link failed")
-    return LIB
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose_ptxas="--verbose-ptxas" in sys.argv))
+    print(build(force="--force" in sys.argv, verbose_ptxas="--verbose-ptxas" in sys.argv,
+                debug="--debug" in sys.argv))

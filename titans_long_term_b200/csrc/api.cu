@@ -573,9 +573,10 @@ titans_status_t titans_mem_sync_status(titans_mem_t m, void* stream) {
     if (e == cudaSuccess) e = cudaMemset(m->status, 0, sizeof(unsigned));
     if (e != cudaSuccess) return cuda_fail(e, "reading the status word");
     if (h) {
-        char buf[128];
+        char buf[192];
         snprintf(buf, sizeof buf,
-                 "device status 0x%x (1: TMA wait timed out, 2: MMA wait timed out, 4: grid barrier timed out)", h);
+                 "device status 0x%x (1: TMA wait timed out, 2: MMA wait timed out, 4: grid barrier timed out, "
+                 "8: a bounds check of the debug build failed)", h);
         return fail(TITANS_EDEVICE, buf);
     }
     return TITANS_OK;

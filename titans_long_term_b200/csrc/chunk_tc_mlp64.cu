@@ -237,6 +237,10 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
     tc_fence_after();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sm + TPTR);
 
+#define DBG(cond) TITANS_DBG(cond, status, abort_flag)
+    // TMEM column of an address relative to the allocation, and the byte span of shared memory in use.
+    auto tcol_ok = [&](uint32_t taddr) { return ((taddr & 0xFFFFu) - (tmem & 0xFFFFu)) + 16u <= kTmemCols && (taddr >> 16) <= 96u; };
+    auto smem_ok = [&](uint32_t addr) { return addr >= sb && addr + 16u <= sb + END; };
     // Bounded wait; on a timeout records the fault, raises the abort flag and returns false.
     auto wait = [&](int b, uint32_t parity) -> bool {
         if (mbar_wait(&bars[b], parity)) return true;
@@ -284,9 +288,10 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
                 const int j = lane + 32 * i;
                 const bool ok = j < n;
                 const long g = u * gate_ld + (chunk_gates ? (long)c : t0 + j);  // chunk-shared or per-token
-                ga[i] = ok ? __ldg(alpha + g) : 0.f;
-                ge[i] = ok ? __ldg(eta + g) : 1.f;
-                gt[i] = ok ? __ldg(theta + g) : 0.f;
+                const bool in = ok && DBG(g >= u * gate_ld && g < (u + 1) * gate_ld);
+                ga[i] = in ? __ldg(alpha + g) : 0.f;
+                ge[i] = in ? __ldg(eta + g) : 1.f;
+                gt[i] = in ? __ldg(theta + g) : 0.f;
             }
         };
         float* sg = reinterpret_cast<float*>(sm + GATES);
@@ -322,6 +327,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
                 for (int i = 0; i < 16; ++i) {
                     const uint32_t off = (uint32_t)(lane + 32 * i) * 16u;
                     const int row = (lane + 32 * i) >> 3;
+                    if (!DBG(off + 16u <= 8192u)) continue;
                     const uint4 kv = ld_shared_v4(sb + KQb + off);
                     const float cr = -0.5f * cc[row], dr = -0.5f * dd[row];  // W1, S1 are kept halved
                     const uint32_t in[4] = {kv.x, kv.y, kv.z, kv.w};
@@ -402,6 +408,8 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
         auto issue_tma = [&](int c) {
             const int b = c & 1;
             const uint32_t kq = b ? KQ1 : KQ0, vv = b ? V1 : V0;
+            // coordinates: x = 0 (16-byte aligned), a token row inside the stream, this unit
+            if (!DBG((long)c * chunk < T && u < (long)gridDim.x)) return;
             mbar_arrive_expect_tx(&bars[B_TMA0 + b], tx_bytes);
             tma_load_3d(sm + kq, &tmK, &bars[B_TMA0 + b], 0, c * chunk, (int)u);
             tma_load_3d(sm + kq + 8192, &tmQ, &bars[B_TMA0 + b], 0, c * chunk, (int)u);
@@ -549,6 +557,9 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
 #pragma unroll 1
             for (int blk = 0; blk < 4; ++blk) {  // keys and queries, 16-column blocks
                 uint32_t rk[16], rq[16];
+                if (!DBG(tcol_ok(t_work + 16 * blk) && tcol_ok(t_work + 64 + 16 * blk) &&
+                         smem_ok(sb + AT1 + (uint32_t)hrow * 128u + 112u)))
+                    break;
                 tmem_ld16(t_work + 16 * blk, rk);
                 tmem_ld16(t_work + 64 + 16 * blk, rq);
                 tmem_wait_ld();
@@ -625,6 +636,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
 #pragma unroll
                         for (int ch = 0; ch < 2; ++ch) {
                             const uint32_t off = sw128_off((uint32_t)row, (uint32_t)(col0 + 8 * ch));
+                            if (!DBG(off + 16u <= 8192u)) continue;
                             const uint4 vv = ld_shared_v4(sb + Vb + off);
                             const uint32_t vin[4] = {vv.x, vv.y, vv.z, vv.w};
                             uint32_t og[4], oc[4], od[4];
@@ -659,7 +671,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
                     }
                     tc_fence_before();
                     mbar_arrive(&bars[B_G]);
-                    if (row - kN < n) {
+                    if (row - kN < n && DBG(t0 + (row - kN) < T)) {
                         const long off = (u * T + t0 + (row - kN)) * kD + 32 * tile;
                         uint4* dst = reinterpret_cast<uint4*>(yg + off);
                         if (attn == nullptr) {
@@ -766,6 +778,8 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
         tmem_dealloc(tmem, kTmemCols);
     }
 }
+
+#undef DBG
 
 size_t chunk_tc_mlp64_smem_bytes() { return tc::kSmemBytes; }
 

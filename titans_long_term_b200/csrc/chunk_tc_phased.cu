@@ -224,10 +224,13 @@ __global__ void __launch_bounds__(ph::kThreads, 1) chunk_fwd_tc_phased(const __g
         return all;
     };
     auto unit_ws = [&](int u) { return a.ws + (size_t)u * a.ws_stride; };
+#define DBG(cond) TITANS_DBG(cond, a.status, reinterpret_cast<volatile int*>(&a.sync[1]))
 
     const int units = a.units;
     const long T = a.T;
     const int nchunks = (int)((T + a.chunk - 1) / a.chunk);
+    // every workspace piece of a unit lies inside its stride; a chunk fits the 128-token tiles
+    if (!DBG(a.ws_stride >= kWsBytes && a.chunk >= 1 && a.chunk <= kNmax)) ok = false;
 
     // ---- prologue: bf16 copies of the initial weights
     for (long i = (long)blockIdx.x * kThreads + tid; i < (long)units * kH * kD / 4; i += (long)gridDim.x * kThreads) {
@@ -241,11 +244,12 @@ __global__ void __launch_bounds__(ph::kThreads, 1) chunk_fwd_tc_phased(const __g
         __stcg(d1, make_uint2(pack2(w1.x, w1.y), pack2(w1.z, w1.w)));
         __stcg(d2, make_uint2(pack2(w2.x, w2.y), pack2(w2.z, w2.w)));
     }
-    ok = grid_sync(a, epoch, s_ok);
+    ok = grid_sync(a, epoch, s_ok) && ok;
 
     for (int c = 0; c < nchunks && ok; ++c) {
         const long t0 = (long)c * a.chunk;
         const int n = (int)min((long)a.chunk, T - t0);
+        if (!DBG(n >= 1 && n <= kNmax)) break;  // the same verdict in every CTA
 
         // ================= P1: Z^T tiles (unit, 128 hidden rows, keys | queries) and gate scans
         const int p1_gemm = units * 8;
@@ -260,7 +264,9 @@ __global__ void __launch_bounds__(ph::kThreads, 1) chunk_fwd_tc_phased(const __g
                 for (int i = tid; i < 3 * kNmax; i += kThreads) {
                     const int which = i / kNmax, j = i % kNmax;
                     const float* g = which == 0 ? a.alpha : (which == 1 ? a.eta : a.theta);
-                    s_g[i] = j < n ? __ldg(g + (long)u * a.gate_ld + (a.chunk_gates ? t0 / a.chunk : t0 + j)) : 0.f;
+                    const long gi = (long)u * a.gate_ld + (a.chunk_gates ? t0 / a.chunk : t0 + j);
+                    const bool in = j < n && DBG(gi < (long)(u + 1) * a.gate_ld);
+                    s_g[i] = in ? __ldg(g + gi) : 0.f;
                 }
                 __syncthreads();
                 if (tid == 0) {
@@ -435,7 +441,7 @@ __global__ void __launch_bounds__(ph::kThreads, 1) chunk_fwd_tc_phased(const __g
                     __stcg(reinterpret_cast<uint4*>(w + GC + off) + q4, make_uint4(oc[0], oc[1], oc[2], oc[3]));
                     __stcg(reinterpret_cast<uint4*>(w + GD + off) + q4, make_uint4(od[0], od[1], od[2], od[3]));
                 }
-            } else if (row < n) {
+            } else if (row < n && DBG(t0 + row < T && col0 + 32 <= kD)) {
                 const long off = ((long)u * T + t0 + row) * kD + col0;
                 uint4* dst = reinterpret_cast<uint4*>(a.y + off);
                 const uint4* arow = a.attn ? reinterpret_cast<const uint4*>(a.attn + off) : nullptr;
@@ -643,6 +649,8 @@ __global__ void __launch_bounds__(ph::kThreads, 1) chunk_fwd_tc_phased(const __g
         tmem_dealloc(tmem, kTmemCols);
     }
 }
+
+#undef DBG
 
 size_t tc_phased_ws_bytes_per_unit() { return ph::kWsBytes; }
 

@@ -13,6 +13,22 @@ namespace titans {
 constexpr unsigned kStatusTimeoutTma = 1u;
 constexpr unsigned kStatusTimeoutMma = 2u;
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;  // 1 s
+constexpr unsigned kStatusBounds = 8u;  // a TITANS_DEBUG bounds check failed (the access was skipped)
+
+// TITANS_DEBUG builds check the runtime-dependent addresses and coordinates of the kernels' memory
+// accesses (TMA coordinates, gate and token indices, shared-memory and TMEM offsets): a failed check
+// ORs kStatusBounds into the status word, raises the kernel's abort flag and skips the access. Other
+// builds compile every check to `true`.
+__device__ __forceinline__ bool dbg_fail(unsigned* status, volatile int* abort_flag) {
+    if (status) atomicOr(status, kStatusBounds);
+    if (abort_flag) *abort_flag = 1;
+    return false;
+}
+#ifdef TITANS_DEBUG
+#define TITANS_DBG(cond, status, abort_flag) ((cond) ? true : ::titans::dbg_fail((status), (abort_flag)))
+#else
+#define TITANS_DBG(cond, status, abort_flag) true
+#endif
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));

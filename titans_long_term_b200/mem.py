@@ -3,7 +3,9 @@
 Every computation runs in the CUDA library ``libtitans_mem.so`` built in-tree by
 ``titans_long_term_b200/build.py``; if the library is missing this module raises
 instead of falling back to anything else. PyTorch supplies device memory and the
-current CUDA stream.
+current CUDA stream. With the environment variable ``TITANS_DEBUG=1`` the binding loads
+``libtitans_mem_debug.so`` (``build.py --debug``), whose kernels check the coordinates and
+offsets of their memory accesses and report a failed check in the status word.
 """
 from __future__ import annotations
 
@@ -14,7 +16,8 @@ from typing import Dict, Optional
 import torch
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libtitans_mem.so")
+DEBUG = os.environ.get("TITANS_DEBUG", "0") == "1"
+LIB_PATH = os.path.join(HERE, "libtitans_mem_debug.so" if DEBUG else "libtitans_mem.so")
 
 OK, EINVAL, EUNSUPPORTED, ECUDA, EDEVICE = 0, 1, 2, 3, 4
 BF16, FP32 = 0, 1
@@ -55,7 +58,8 @@ def lib():
     global _lib
     if _lib is None:
         if not os.path.exists(LIB_PATH):
-            raise ImportError(f"{LIB_PATH} is missing: run `python -m titans_long_term_b200.build`")
+            how = " --debug" if DEBUG else ""
+            raise ImportError(f"{LIB_PATH} is missing: run `python -m titans_long_term_b200.build{how}`")
         L = ctypes.CDLL(LIB_PATH)
         vp, i, l = ctypes.c_void_p, ctypes.c_int, ctypes.c_long
         L.titans_mem_init.argtypes = [ctypes.POINTER(Config), ctypes.POINTER(vp)]
