@@ -60,6 +60,12 @@ constexpr uint32_t kSmemOperands = 224 * 1024;
 // P4 stages the fp32 W and S tiles it updates ([128 rows][128 floats] each) after its 96 KB of
 // MMA operands.
 constexpr uint32_t kStageW = 96 * 1024, kStageS = 160 * 1024;
+// Epilogue staging (row-contiguous copies out): in the operand area, free once a tile's MMAs
+// completed, except for inputs staged with the operands.
+constexpr uint32_t kP1At = 0, kP1Sp = 32 * 1024;    // silu(Z)^T [128][256 B], silu'(Z_K)^T [128][512 B]
+constexpr uint32_t kP2G = 0, kP2In = 192 * 1024;    // G, -cG, -dG (or y) [128][128 B] each; v or attn [128][128 B]
+constexpr uint32_t kP3Dt = 0, kP3Sp = 64 * 1024;    // Delta^T [128][256 B]; silu'(Z_K)^T rows [128][512 B]
+constexpr uint32_t kP4Wb = 0;                       // bf16 weight rows [128][256 B]
 constexpr uint32_t BAR = kSmemOperands;       // one mbarrier (MMA completion)
 constexpr uint32_t TPTR = BAR + 8;
 constexpr uint32_t OKF = TPTR + 4;            // the grid barrier's verdict for the CTA
@@ -108,19 +114,38 @@ __device__ __forceinline__ void load_tile(uint32_t tile, const uint8_t* src, siz
     }
 }
 
-// Byte offset of 16-byte chunk c (0..31) of row r in a [128][128] fp32 tile staged in shared memory:
-// the chunk index is XORed with r % 8 within its group of eight, so that the 32 lanes of a warp,
-// one row each, spread their 16-byte accesses over all banks.
-__device__ __forceinline__ uint32_t stage_off(int r, int c) {
-    return (uint32_t)r * 512u + ((uint32_t)((c & ~7) | ((c ^ r) & 7)) << 4);
+// Byte offset of 16-byte chunk c of row r in a tile staged in shared memory with rows of `rb`
+// bytes (a multiple of 128): within each group of eight chunks the index is XORed with r % 8, so
+// that the 32 lanes of a warp, one row each, spread their 16-byte accesses over all banks, while a
+// row's chunks stay inside the row.
+__device__ __forceinline__ uint32_t srow_off(int r, int c, uint32_t rb) {
+    return (uint32_t)r * rb + ((uint32_t)((c & ~7) | ((c ^ r) & 7)) << 4);
+}
+__device__ __forceinline__ uint32_t stage_off(int r, int c) { return srow_off(r, c, 512); }
+
+// Coalesced copy of `rows` rows of rb bytes (row r at src + r * ld bytes) into the staged layout.
+__device__ __forceinline__ void stage_rows_in(uint32_t tile, const void* src, size_t ld, int rows, uint32_t rb) {
+    const int cpr = (int)(rb >> 4);
+    for (int i = threadIdx.x; i < rows * cpr; i += ph::kThreads) {
+        const int r = i / cpr, c = i % cpr;
+        cp_async16(tile + srow_off(r, c, rb), reinterpret_cast<const uint8_t*>(src) + (size_t)r * ld + 16 * c);
+    }
+}
+
+// Coalesced copy of the first `rows` staged rows of rb bytes out to dst + r * ld bytes (L2 only):
+// consecutive threads write consecutive 16-byte pieces of a row.
+__device__ __forceinline__ void stage_rows_out(const uint8_t* tile, void* dst, size_t ld, int rows, uint32_t rb) {
+    const int cpr = (int)(rb >> 4);
+    for (int i = threadIdx.x; i < rows * cpr; i += ph::kThreads) {
+        const int r = i / cpr, c = i % cpr;
+        __stcg(reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(dst) + (size_t)r * ld) + c,
+               *reinterpret_cast<const uint4*>(tile + srow_off(r, c, rb)));
+    }
 }
 
 // Coalesced copy of a [128 rows][128 floats] tile (row r at src + r * ld floats) into the staging layout.
 __device__ __forceinline__ void stage_in(uint32_t tile, const float* src, size_t ld) {
-    for (int i = threadIdx.x; i < 128 * 32; i += ph::kThreads) {
-        const int r = i >> 5, c = i & 31;
-        cp_async16(tile + stage_off(r, c), src + (size_t)r * ld + 4 * c);
-    }
+    stage_rows_in(tile, src, ld * sizeof(float), 128, 512);
 }
 
 // All operand copies of the tile have landed and are visible to the tensor core.
@@ -269,24 +294,81 @@ __global__ void __launch_bounds__(ph::kThreads, 1) chunk_fwd_tc_phased(const __g
                     s_g[i] = in ? __ldg(g + gi) : 0.f;
                 }
                 __syncthreads();
-                if (tid == 0) {
+                if (warp == 0) {
+                    // The suffix scan on one warp, tokens j = 4 lane + i (gates past n are neutral):
+                    //   P_j = prod_{l>j} (1 - alpha_l), Q_j = prod_{l>j} eta_l, r_j = P_j + eta_{j+1} r_{j+1}
+                    // with the chain cut after the last token; products and the affine maps of r are
+                    // combined across lanes with shuffles.
                     const float* al = s_g;
                     const float* et = s_g + kNmax;
                     const float* th = s_g + 2 * kNmax;
-                    float Pr = 1.f, Qr = 1.f, r_next = 0.f;
-                    for (int j = kNmax - 1; j >= n; --j) s_c[j] = s_d[j] = 0.f;
-                    for (int j = n - 1; j >= 0; --j) {
-                        // r_j = P_j + eta_{j+1} r_{j+1}, P_j = prod_{l>j} (1 - alpha_l), Q_j = prod_{l>j} eta_l
-                        const float r = Pr + (j + 1 < n ? et[j + 1] * r_next : 0.f);
-                        s_c[j] = th[j] * r;
-                        s_d[j] = th[j] * Qr;
-                        r_next = r;
-                        Pr *= 1.f - al[j];
-                        Qr *= et[j];
+                    float om[4], e4[4], t4[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int j = 4 * lane + i;
+                        const bool v = j < n;
+                        om[i] = v ? 1.f - al[j] : 1.f;
+                        e4[i] = v ? et[j] : 1.f;
+                        t4[i] = v ? th[j] : 0.f;
                     }
-                    s_c[256] = Pr;                 // A = prod (1 - alpha)
-                    s_c[257] = Qr;                 // E = prod eta
-                    s_c[258] = et[0] * r_next;     // sigma = eta_0 r_0
+                    float ps = om[0] * om[1] * om[2] * om[3], qs = e4[0] * e4[1] * e4[2] * e4[3];
+#pragma unroll
+                    for (int off = 1; off < 32; off <<= 1) {  // inclusive suffix products over lanes
+                        const float p2 = __shfl_down_sync(0xffffffffu, ps, off), q2 = __shfl_down_sync(0xffffffffu, qs, off);
+                        if (lane + off < 32) {
+                            ps *= p2;
+                            qs *= q2;
+                        }
+                    }
+                    float P[4], Q[4];
+                    P[3] = __shfl_down_sync(0xffffffffu, ps, 1);
+                    Q[3] = __shfl_down_sync(0xffffffffu, qs, 1);
+                    if (lane == 31) P[3] = Q[3] = 1.f;
+#pragma unroll
+                    for (int i = 2; i >= 0; --i) {
+                        P[i] = P[i + 1] * om[i + 1];
+                        Q[i] = Q[i + 1] * e4[i + 1];
+                    }
+                    // r_j = a_j r_{j+1} + P_j, a_j = eta_{j+1} while j + 1 < n, else 0
+                    const float e_next = __shfl_down_sync(0xffffffffu, e4[0], 1);
+                    float av[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int j = 4 * lane + i;
+                        av[i] = j + 1 < n ? (i < 3 ? e4[i + 1] : e_next) : 0.f;
+                    }
+                    float A = 1.f, B = 0.f;  // this lane's map r_{4 lane} = A r_{4 lane + 4} + B
+#pragma unroll
+                    for (int i = 3; i >= 0; --i) {
+                        B = fmaf(av[i], B, P[i]);
+                        A *= av[i];
+                    }
+#pragma unroll
+                    for (int off = 1; off < 32; off <<= 1) {
+                        const float A2 = __shfl_down_sync(0xffffffffu, A, off), B2 = __shfl_down_sync(0xffffffffu, B, off);
+                        if (lane + off < 32) {
+                            B = fmaf(A, B2, B);
+                            A *= A2;
+                        }
+                    }
+                    float x = __shfl_down_sync(0xffffffffu, B, 1);  // r of the next lane's first token
+                    if (lane == 31) x = 0.f;
+                    float r[4];
+#pragma unroll
+                    for (int i = 3; i >= 0; --i) {
+                        x = fmaf(av[i], x, P[i]);
+                        r[i] = x;
+                    }
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        s_c[4 * lane + i] = t4[i] * r[i];
+                        s_d[4 * lane + i] = t4[i] * Q[i];
+                    }
+                    if (lane == 0) {
+                        s_c[256] = ps;            // A = prod (1 - alpha)
+                        s_c[257] = qs;            // E = prod eta
+                        s_c[258] = e4[0] * r[0];  // sigma = eta_0 r_0
+                    }
                 }
                 __syncthreads();
                 float* gsc = reinterpret_cast<float*>(w + SC);
@@ -338,10 +420,8 @@ __global__ void __launch_bounds__(ph::kThreads, 1) chunk_fwd_tc_phased(const __g
                 ok = false;
                 break;
             }
-            // Epilogue: hidden row h = mt*128 + row, tokens [64 half, +64).
-            const int h = mt * 128 + row;
-            uint8_t* at_row = w + AT + ((size_t)h * 256 + part * 128 + 64 * half) * 2;
-            float* sp_row = reinterpret_cast<float*>(w + SP) + (size_t)h * kNmax + 64 * half;
+            // Epilogue: hidden row mt*128 + row, tokens [64 half, +64). The outputs are staged in the
+            // operand area (free once the MMAs completed) and copied out row-contiguously.
 #pragma unroll 1
             for (int blk = 0; blk < 4; ++blk) {
                 uint32_t r[16];
@@ -360,16 +440,20 @@ __global__ void __launch_bounds__(ph::kThreads, 1) chunk_fwd_tc_phased(const __g
                     spv[i] = s0 + a0 * (1.f - s0);  // silu'(z) = sigma + silu (1 - sigma)
                     spv[i + 1] = s1 + a1 * (1.f - s1);
                 }
-                uint4* dst = reinterpret_cast<uint4*>(at_row + 32 * blk);
-                __stcg(dst, make_uint4(pk[0], pk[1], pk[2], pk[3]));
-                __stcg(dst + 1, make_uint4(pk[4], pk[5], pk[6], pk[7]));
+                st_shared_v4(sb + kP1At + srow_off(row, 8 * half + 2 * blk, 256), pk[0], pk[1], pk[2], pk[3]);
+                st_shared_v4(sb + kP1At + srow_off(row, 8 * half + 2 * blk + 1, 256), pk[4], pk[5], pk[6], pk[7]);
                 if (part == 0) {
-                    float4* sd = reinterpret_cast<float4*>(sp_row + 16 * blk);
 #pragma unroll
                     for (int q4 = 0; q4 < 4; ++q4)
-                        __stcg(sd + q4, make_float4(spv[4 * q4], spv[4 * q4 + 1], spv[4 * q4 + 2], spv[4 * q4 + 3]));
+                        st_shared_v4(sb + kP1Sp + srow_off(row, 16 * half + 4 * blk + q4, 512),
+                                     __float_as_uint(spv[4 * q4]), __float_as_uint(spv[4 * q4 + 1]),
+                                     __float_as_uint(spv[4 * q4 + 2]), __float_as_uint(spv[4 * q4 + 3]));
                 }
             }
+            __syncthreads();
+            stage_rows_out(sm + kP1At, w + AT + ((size_t)mt * 128 * 256 + part * 128) * 2, 256 * 2, 128, 256);
+            if (part == 0)
+                stage_rows_out(sm + kP1Sp, w + SP + (size_t)mt * 128 * kNmax * 4, kNmax * 4, 128, 512);
         }
         if (!grid_sync(a, epoch, s_ok) || !ok) {
             ok = false;
@@ -390,6 +474,10 @@ __global__ void __launch_bounds__(ph::kThreads, 1) chunk_fwd_tc_phased(const __g
                               256 * 2, 64, 64);
                 load_tile(sb + 131072 + kb * 8192, w + W2B + ((size_t)nh * 64 * kH + kb * 64) * 2, kH * 2, 64, 64);
             }
+            // The epilogue's other input, staged row-contiguously: v (keys) or attn (gated queries),
+            // tokens [t0, t0 + n), columns [nh*64, +64).
+            const __nv_bfloat16* ein = part == 0 ? a.v : a.attn;
+            if (ein) stage_rows_in(sb + kP2In, ein + ((long)u * T + t0) * kD + nh * 64, kD * 2, n, 128);
             operands_ready();
             if (tid == 0) {
                 const uint32_t id = idesc_bf16_f32(128, 64, 1, 0);
@@ -403,7 +491,6 @@ __global__ void __launch_bounds__(ph::kThreads, 1) chunk_fwd_tc_phased(const __g
                 break;
             }
             // Epilogue: token row `row`, output columns nh*64 + 32 half + [0, 32).
-            const int col0 = nh * 64 + 32 * half;
             float yv[32];
 #pragma unroll
             for (int b = 0; b < 2; ++b) {
@@ -417,16 +504,11 @@ __global__ void __launch_bounds__(ph::kThreads, 1) chunk_fwd_tc_phased(const __g
                 const float* gsc = reinterpret_cast<const float*>(w + SC);
                 const float cr = -__ldcg(gsc + row), dr = -__ldcg(gsc + 128 + row);
                 const bool valid = row < n;
-                const uint4* vrow = reinterpret_cast<const uint4*>(a.v + ((long)u * T + t0 + row) * kD + col0);
-                const size_t off = ((size_t)row * kD + col0) * 2;
-                uint4 vq[4];
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) vq[q4] = valid ? __ldg(vrow + q4) : make_uint4(0, 0, 0, 0);
 #pragma unroll
                 for (int q4 = 0; q4 < 4; ++q4) {
                     uint32_t og[4] = {0, 0, 0, 0}, oc[4] = {0, 0, 0, 0}, od[4] = {0, 0, 0, 0};
                     if (valid) {
-                        const uint4 vv = vq[q4];
+                        const uint4 vv = ld_shared_v4(sb + kP2In + srow_off(row, 4 * half + q4, 128));
                         const uint32_t vin[4] = {vv.x, vv.y, vv.z, vv.w};
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
@@ -437,32 +519,39 @@ __global__ void __launch_bounds__(ph::kThreads, 1) chunk_fwd_tc_phased(const __g
                             od[e] = pack2(dr * g0, dr * g1);
                         }
                     }
-                    __stcg(reinterpret_cast<uint4*>(w + GG + off) + q4, make_uint4(og[0], og[1], og[2], og[3]));
-                    __stcg(reinterpret_cast<uint4*>(w + GC + off) + q4, make_uint4(oc[0], oc[1], oc[2], oc[3]));
-                    __stcg(reinterpret_cast<uint4*>(w + GD + off) + q4, make_uint4(od[0], od[1], od[2], od[3]));
+                    const uint32_t o = srow_off(row, 4 * half + q4, 128);
+                    st_shared_v4(sb + kP2G + o, og[0], og[1], og[2], og[3]);
+                    st_shared_v4(sb + kP2G + 16384 + o, oc[0], oc[1], oc[2], oc[3]);
+                    st_shared_v4(sb + kP2G + 32768 + o, od[0], od[1], od[2], od[3]);
                 }
-            } else if (row < n && DBG(t0 + row < T && col0 + 32 <= kD)) {
-                const long off = ((long)u * T + t0 + row) * kD + col0;
-                uint4* dst = reinterpret_cast<uint4*>(a.y + off);
-                const uint4* arow = a.attn ? reinterpret_cast<const uint4*>(a.attn + off) : nullptr;
+                __syncthreads();
+                // rows >= n are zero: they are operands of the next phases
+                stage_rows_out(sm + kP2G, w + GG + nh * 64 * 2, kD * 2, 128, 128);
+                stage_rows_out(sm + kP2G + 16384, w + GC + nh * 64 * 2, kD * 2, 128, 128);
+                stage_rows_out(sm + kP2G + 32768, w + GD + nh * 64 * 2, kD * 2, 128, 128);
+            } else {
+                if (row < n && DBG(t0 + row < T)) {
 #pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    uint32_t o[4];
-                    uint4 av = make_uint4(0, 0, 0, 0);
-                    if (arow) av = __ldg(arow + q4);
-                    const uint32_t aw[4] = {av.x, av.y, av.z, av.w};
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        uint32_t o[4];
+                        uint4 av = make_uint4(0, 0, 0, 0);
+                        if (a.attn) av = ld_shared_v4(sb + kP2In + srow_off(row, 4 * half + q4, 128));
+                        const uint32_t aw[4] = {av.x, av.y, av.z, av.w};
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        float y0 = yv[8 * q4 + 2 * e], y1 = yv[8 * q4 + 2 * e + 1];
-                        if (arow) {  // memory-as-a-gate output attn * sigmoid(y) (walk-through sec. 4.2)
-                            const float2 a2 = unpack_bf16x2(aw[e]);
-                            y0 = a2.x * fmaf(0.5f, tanh_approx(0.5f * y0), 0.5f);
-                            y1 = a2.y * fmaf(0.5f, tanh_approx(0.5f * y1), 0.5f);
+                        for (int e = 0; e < 4; ++e) {
+                            float y0 = yv[8 * q4 + 2 * e], y1 = yv[8 * q4 + 2 * e + 1];
+                            if (a.attn) {  // memory-as-a-gate output attn * sigmoid(y) (walk-through sec. 4.2)
+                                const float2 a2 = unpack_bf16x2(aw[e]);
+                                y0 = a2.x * fmaf(0.5f, tanh_approx(0.5f * y0), 0.5f);
+                                y1 = a2.y * fmaf(0.5f, tanh_approx(0.5f * y1), 0.5f);
+                            }
+                            o[e] = pack2(y0, y1);
                         }
-                        o[e] = pack2(y0, y1);
+                        st_shared_v4(sb + kP2G + srow_off(row, 4 * half + q4, 128), o[0], o[1], o[2], o[3]);
                     }
-                    dst[q4] = make_uint4(o[0], o[1], o[2], o[3]);
                 }
+                __syncthreads();
+                stage_rows_out(sm + kP2G, a.y + ((long)u * T + t0) * kD + nh * 64, kD * 2, n, 128);
             }
         }
         if (!grid_sync(a, epoch, s_ok) || !ok) {
@@ -484,6 +573,7 @@ __global__ void __launch_bounds__(ph::kThreads, 1) chunk_fwd_tc_phased(const __g
                               kH * 2, 64, 64);
                 load_tile(sb + 32768 + kb * 16384, w + GG + (size_t)kb * 64 * 2, kD * 2, 128, 128);
             }
+            stage_rows_in(sb + kP3Sp, w + SP + (size_t)mt * 128 * kNmax * 4, kNmax * 4, 128, 512);  // silu'(Z_K)^T rows
             operands_ready();
             if (tid == 0) {
                 const uint32_t id = idesc_bf16_f32(128, 128, 1, 0);
@@ -496,13 +586,7 @@ __global__ void __launch_bounds__(ph::kThreads, 1) chunk_fwd_tc_phased(const __g
                 ok = false;
                 break;
             }
-            const int h = mt * 128 + row;
-            const float* sp_row = reinterpret_cast<const float*>(w + SP) + (size_t)h * kNmax + 64 * half;
-            uint8_t* dt_row = w + DT + ((size_t)h * kNmax + 64 * half) * 2;
-            float4 spv[16];  // this thread's 64 silu' values, read before any store
-#pragma unroll
-            for (int i = 0; i < 16; ++i) spv[i] = __ldcg(reinterpret_cast<const float4*>(sp_row) + i);
-#pragma unroll
+#pragma unroll 1
             for (int blk = 0; blk < 4; ++blk) {
                 uint32_t r[16];
                 tmem_ld16(tmem + lane_off + 64 * half + 16 * blk, r);
@@ -510,14 +594,17 @@ __global__ void __launch_bounds__(ph::kThreads, 1) chunk_fwd_tc_phased(const __g
                 uint32_t pk[8];
 #pragma unroll
                 for (int q4 = 0; q4 < 4; ++q4) {
-                    const float4 s = spv[4 * blk + q4];
-                    pk[2 * q4] = pack2(__uint_as_float(r[4 * q4]) * s.x, __uint_as_float(r[4 * q4 + 1]) * s.y);
-                    pk[2 * q4 + 1] = pack2(__uint_as_float(r[4 * q4 + 2]) * s.z, __uint_as_float(r[4 * q4 + 3]) * s.w);
+                    const uint4 sp = ld_shared_v4(sb + kP3Sp + srow_off(row, 16 * half + 4 * blk + q4, 512));
+                    pk[2 * q4] = pack2(__uint_as_float(r[4 * q4]) * __uint_as_float(sp.x),
+                                       __uint_as_float(r[4 * q4 + 1]) * __uint_as_float(sp.y));
+                    pk[2 * q4 + 1] = pack2(__uint_as_float(r[4 * q4 + 2]) * __uint_as_float(sp.z),
+                                           __uint_as_float(r[4 * q4 + 3]) * __uint_as_float(sp.w));
                 }
-                uint4* dst = reinterpret_cast<uint4*>(dt_row + 32 * blk);
-                __stcg(dst, make_uint4(pk[0], pk[1], pk[2], pk[3]));
-                __stcg(dst + 1, make_uint4(pk[4], pk[5], pk[6], pk[7]));
+                st_shared_v4(sb + kP3Dt + srow_off(row, 8 * half + 2 * blk, 256), pk[0], pk[1], pk[2], pk[3]);
+                st_shared_v4(sb + kP3Dt + srow_off(row, 8 * half + 2 * blk + 1, 256), pk[4], pk[5], pk[6], pk[7]);
             }
+            __syncthreads();
+            stage_rows_out(sm + kP3Dt, w + DT + (size_t)mt * 128 * kNmax * 2, kNmax * 2, 128, 256);
         }
         if (!grid_sync(a, epoch, s_ok) || !ok) {
             ok = false;
@@ -596,8 +683,6 @@ __global__ void __launch_bounds__(ph::kThreads, 1) chunk_fwd_tc_phased(const __g
             // in place in the staged tiles; then the bf16 copy of the row, and coalesced copies out.
             const float* gsc = reinterpret_cast<const float*>(w + SC);
             const float An = __ldcg(gsc + 256), En = __ldcg(gsc + 257), sig = __ldcg(gsc + 258);
-            uint8_t* Wb = which == 0 ? w + W1B + (((size_t)mt * 128 + row) * kD + 64 * half) * 2
-                                     : w + W2B + ((size_t)row * kH + mt * 128 + 64 * half) * 2;
 #pragma unroll 1
             for (int blk = 0; blk < 4; ++blk) {
                 uint32_t rc[16], rd[16];
@@ -622,11 +707,15 @@ __global__ void __launch_bounds__(ph::kThreads, 1) chunk_fwd_tc_phased(const __g
                     pk[2 * q4] = pack2(wn[0], wn[1]);
                     pk[2 * q4 + 1] = pack2(wn[2], wn[3]);
                 }
-                uint4* dst = reinterpret_cast<uint4*>(Wb + 32 * blk);
-                __stcg(dst, make_uint4(pk[0], pk[1], pk[2], pk[3]));
-                __stcg(dst + 1, make_uint4(pk[4], pk[5], pk[6], pk[7]));
+                st_shared_v4(sb + kP4Wb + srow_off(row, 8 * half + 2 * blk, 256), pk[0], pk[1], pk[2], pk[3]);
+                st_shared_v4(sb + kP4Wb + srow_off(row, 8 * half + 2 * blk + 1, 256), pk[4], pk[5], pk[6], pk[7]);
             }
             __syncthreads();
+            // the bf16 copy of the rows: W1 rows [mt*128, +128) or W2 rows 0..127 at hidden [mt*128, +128)
+            if (which == 0)
+                stage_rows_out(sm + kP4Wb, w + W1B + (size_t)mt * 128 * kD * 2, kD * 2, 128, 256);
+            else
+                stage_rows_out(sm + kP4Wb, w + W2B + (size_t)mt * 128 * 2, kH * 2, 128, 256);
             for (int i = tid; i < 128 * 32; i += kThreads) {
                 const int r = i >> 5, cc = i & 31;
                 const uint32_t o = stage_off(r, cc);
