@@ -470,6 +470,155 @@ def decode_arm(args, w, rank, world, local_rank):
         "roofline": rec["roofline"], "gpu_launches": rec["gpu_launches"]}), flush=True)
 
 
+def _dev_inputs(w, dev, T=None, units=None):
+    """Seeded inputs of a workload on the device, shaped [B, H, ...] (units = B*H)."""
+    T = w.T if T is None else T
+    inp = synth.make_inputs(w, T=T)
+    toks = {n: inp[n].reshape(w.B, w.H, T, w.d).to(dev) for n in ("k", "q", "v")}
+    gates = {n: inp[n].reshape(w.B, w.H, T).to(dev) for n in ("alpha", "eta", "theta")}
+    state = {n: inp[n].reshape(w.B, w.H, *inp[n].shape[1:]).to(dev) for n in inp if n[0] in "WS"}
+    return toks, gates, state
+
+
+def _cuda_core_roofline(flops, avg_ms, kernel, units, note):
+    """Roofline record of a CUDA-core kernel: fp32 FMA work against the nominal fp32 FMA peak
+    (148 SMs x 128 lanes x 2 FLOP x 1.965 GHz) and the SMs its one-CTA-per-unit grid can use."""
+    achieved = flops / (avg_ms / 1e3) / 1e12
+    sms = min(units, 148)
+    return {"bound": "alu", "achieved": achieved, "peak": FP32_FMA_TFLOPS_NOMINAL, "unit": "TFLOP/s",
+            "frac": achieved / FP32_FMA_TFLOPS_NOMINAL, "traffic": None,
+            "peak_source": "fp32 FMA nominal (148 SMs x 128 lanes x 2 FLOP x 1.965 GHz)", "kernel": kernel,
+            "flops_per_launch": flops, "avg_launch_ms": avg_ms, "sms_used": sms,
+            "frac_of_sms_used": achieved / (FP32_FMA_TFLOPS_NOMINAL * sms / 148), "note": note}
+
+
+def deep_flops_per_head_token(d, h, layers) -> float:
+    """Algorithmic FLOPs of a deep memory per head-token, with P = the weights of one state copy:
+    key forward 2P, retrieval 2P, back-propagation to every hidden layer 2(P - d h), and the c- and
+    d-weighted outer products 4P. At 2 layers this is the 2-layer memory's 18 d h."""
+    P = sum(o * i for o, i in synth.deep_shapes(d, h, layers))
+    return 10 * P - 2 * d * h
+
+
+def extension_results(dev, steps: int, warmup: int):
+    """The extension rows, each timed on its own workload: the memory-as-a-gate output and chunk-shared
+    gates on the benchmarked kernel, the linear memory's cross-chunk scan, the deep memory and the
+    backward (outer-loop gradients) of the 2-layer memory."""
+    out = {}
+    peaks, which = load_peaks()
+    # memory-as-a-gate output and chunk-shared gates: the 760M-class workload on the tensor-core kernel
+    w = synth.WORKLOADS["mlp-d64-b8h16-t4k"]
+    toks, gates, state = _dev_inputs(w, dev)
+    attn = synth.make_attn(w).reshape(w.B, w.H, w.T, w.d).to(dev)
+    st0 = {n: t.clone() for n, t in state.items()}
+    flops = flops_per_head_token(w) * w.units * w.T
+    for name, chunk_gates in (("gated_output", False), ("chunk_gates", True)):
+        m = mem.Memory(w.d, w.h, w.chunk, w.dtype, w.B, w.H, chunk_gates=chunk_gates)
+        g = gates if not chunk_gates else {n: t[..., ::w.chunk].contiguous() for n, t in gates.items()}
+        st = {n: t.clone() for n, t in st0.items()}
+        o = torch.empty_like(toks["k"])
+        if name == "gated_output":
+            fn = lambda: m.forward_gated(toks["k"], toks["q"], toks["v"], g["alpha"], g["eta"], g["theta"], attn, st, o=o)
+        else:
+            fn = lambda: m.forward(toks["k"], toks["q"], toks["v"], g["alpha"], g["eta"], g["theta"], st, y=o)
+        total, per = time_launches(fn, torch.cuda.current_stream(dev), steps, warmup)
+        m.sync_status()
+        avg = statistics.mean(per)
+        achieved = flops / (avg / 1e3) / 1e12
+        out[name] = {"workload": w.name, "value": w.B * w.T / (total / steps / 1e3), "unit": "tokens/s",
+                     "ms_per_step": total / steps, "steps": steps,
+                     "config": {"path": KERNEL_NAMES.get(m.path()), "chunk_gates": chunk_gates,
+                                "gated_output": name == "gated_output"},
+                     "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
+                                  "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"], "traffic": None,
+                                  "peak_source": f"bf16_tflops ({which})", "kernel": KERNEL_NAMES.get(m.path()),
+                                  "avg_launch_ms": avg},
+                     "gpu_launches": steps}
+        del m, st, o
+    del toks, gates, state, st0, attn
+    torch.cuda.empty_cache()
+
+    # linear memory, one 65,536-token stream: the three-kernel cross-chunk scan against the chunk loop
+    wl = synth.Workload("linear-d64-t64k", 64, 0, 1, 1, 65536, 16, "fp32", 20250106, recipe="stated")
+    toks, gates, state = _dev_inputs(wl, dev)
+    rec = {}
+    for scan in (False, True):
+        m = mem.Memory(wl.d, 0, wl.chunk, wl.dtype, 1, 1, chunk_scan=scan)
+        st = {n: t.clone() for n, t in state.items()}
+        fn = lambda: m.forward(toks["k"], toks["q"], toks["v"], gates["alpha"], gates["eta"], gates["theta"], st)
+        total, per = time_launches(fn, torch.cuda.current_stream(dev), max(3, steps // 2), warmup)
+        m.sync_status()
+        rec[scan] = (total / max(3, steps // 2), statistics.mean(per))
+        del m, st
+    flops = 8.0 * wl.d * wl.d * wl.T
+    out["linear_scan"] = {
+        "workload": wl.name, "value": wl.T / (rec[True][0] / 1e3), "unit": "tokens/s", "ms_per_step": rec[True][0],
+        "chunk_loop_ms": rec[False][0], "speedup_vs_chunk_loop": rec[False][0] / rec[True][0],
+        "config": {"memory": "linear 64x64", "units": 1, "T": wl.T, "chunk": wl.chunk, "mode": "fp32",
+                   "inputs": synth.describe(wl)},
+        "roofline": _cuda_core_roofline(flops, rec[True][1], "linear_scan_compose/segments/run", 148,
+                                        "fp32 on CUDA cores; FLOPs are the chunk recurrence's 8 d^2 per token, "
+                                        "not the scan's extra composition work"),
+        "gpu_launches": 3 * max(3, steps // 2)}
+    del toks, gates, state
+    torch.cuda.empty_cache()
+
+    # deep memory (4 layers, 64 -> 256 -> 256 -> 256 -> 64) on the 8-unit 2K-token workload
+    w = synth.WORKLOADS["mlp-d64-b2h4-t2k"]
+    L = 4
+    toks, gates, _ = _dev_inputs(w, dev)
+    dst = {n: t.reshape(w.B, w.H, -1).to(dev) for n, t in synth.make_deep_state(w, L).items()}
+    flops = deep_flops_per_head_token(w.d, w.h, L) * w.units * w.T
+    for key, cuda_cores in (("deep_memory", False), ("deep_memory_cuda_cores", True)):
+        m = mem.Memory(w.d, w.h, w.chunk, w.dtype, w.B, w.H, layers=L, cuda_cores=cuda_cores)
+        st = {n: t.clone() for n, t in dst.items()}
+        fn = lambda: m.forward_deep(toks["k"], toks["q"], toks["v"], gates["alpha"], gates["eta"], gates["theta"], st)
+        n_deep = steps if not cuda_cores else 3
+        total, per = time_launches(fn, torch.cuda.current_stream(dev), n_deep, 1 if cuda_cores else warmup)
+        m.sync_status()
+        avg = statistics.mean(per)
+        if cuda_cores:
+            roof = _cuda_core_roofline(flops, avg, "chunk_fwd_deep_cuda_cores", w.units,
+                                       "fp32 on CUDA cores, one CTA per unit (TITANS_FLAG_CUDA_CORES)")
+        else:
+            achieved = flops / (avg / 1e3) / 1e12
+            roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                    "frac": achieved / peaks["bf16_tflops"], "traffic": None,
+                    "peak_source": f"bf16_tflops ({which})", "kernel": "chunk_fwd_tc_deep", "flops_per_launch": flops,
+                    "avg_launch_ms": avg}
+        out[key] = {
+            "workload": f"{w.name} deep L={L}", "value": w.B * w.T / (total / n_deep / 1e3), "unit": "tokens/s",
+            "ms_per_step": total / n_deep, "steps": n_deep,
+            "config": {"memory": f"deep {L}-layer {w.d}-{w.h}-{w.h}-{w.h}-{w.d} SiLU", "units": w.units, "T": w.T,
+                       "chunk": w.chunk, "flops_per_head_token": deep_flops_per_head_token(w.d, w.h, L),
+                       "path": "tensor cores (phased, all SMs)" if not cuda_cores else "CUDA cores"},
+            "roofline": roof, "gpu_launches": n_deep}
+        del m, st
+    del dst, toks, gates
+    torch.cuda.empty_cache()
+
+    # backward of the 2-layer memory (gradients of <dy, y> + <dW, W_T> ...) on the same workload
+    toks, gates, state = _dev_inputs(w, dev)
+    dy = torch.randn(toks["k"].shape, generator=torch.Generator().manual_seed(5)).to(toks["k"].dtype).to(dev)
+    m = mem.Memory(w.d, w.h, w.chunk, w.dtype, w.B, w.H)
+    fn = lambda: m.backward(toks["k"], toks["q"], toks["v"], gates["alpha"], gates["eta"], gates["theta"], state, dy)
+    total, per = time_launches(fn, torch.cuda.current_stream(dev), n_deep, 1)
+    m.sync_status()
+    flops = 2 * flops_per_head_token(w) * w.units * w.T
+    out["backward"] = {
+        "workload": f"{w.name} backward", "value": w.B * w.T / (total / n_deep / 1e3), "unit": "tokens/s",
+        "ms_per_step": total / n_deep, "steps": n_deep,
+        "config": {"memory": f"MLP {w.d}-{w.h}-{w.d} SiLU", "units": w.units, "T": w.T, "chunk": w.chunk,
+                   "flops_per_head_token": 2 * flops_per_head_token(w)},
+        "roofline": _cuda_core_roofline(flops, statistics.mean(per), "mlp_backward_kernel", w.units,
+                                        "fp32 on CUDA cores, one CTA per unit; FLOPs counted as twice the "
+                                        "forward's 18 d h per head-token (the chunk forward is recomputed too)"),
+        "gpu_launches": n_deep}
+    del m, toks, gates, state, dy
+    torch.cuda.empty_cache()
+    return out
+
+
 def extra_results(args, dev):
     """The other workloads' numbers, nested in the one JSON line (rank 0 of a 1-GPU run):
     the 2048-unit decode step (HBM-bound), the 16-unit long stream (occupancy-limited: one
@@ -481,6 +630,7 @@ def extra_results(args, dev):
     out["long_stream"] = forward_measure(synth.WORKLOADS["mlp-d64-b1h16-t1m"], dev, max(3, min(args.steps, 5)),
                                          args.warmup)
     out["wide_prefill"] = forward_measure(wide, dev, max(3, min(args.steps, 5)), args.warmup)
+    out.update(extension_results(dev, max(3, min(args.steps, 10)), args.warmup))
     return out
 
 

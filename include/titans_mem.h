@@ -88,7 +88,8 @@ typedef enum {
     TITANS_PATH_STEP_CLUSTER = 3, /* single-token decode, thread-block-cluster kernel (MLP) */
     TITANS_PATH_TC_PHASED = 4,    /* tcgen05 bf16 chunk kernel over all SMs, d=128, h=512, chunk<=128 */
     TITANS_PATH_DEEP_CUDA_CORES = 5, /* deep memory (titans_mem_init_deep), CUDA-core chunk kernel */
-    TITANS_PATH_LINEAR_SCAN = 6      /* linear memory, cross-chunk scan (TITANS_FLAG_CHUNK_SCAN) */
+    TITANS_PATH_LINEAR_SCAN = 6,     /* linear memory, cross-chunk scan (TITANS_FLAG_CHUNK_SCAN) */
+    TITANS_PATH_TC_DEEP = 7          /* deep memory, tcgen05 bf16 phased kernel over all SMs (L >= 3) */
 } titans_path_t;
 
 /* Validates the configuration and allocates the handle, its device status word and
@@ -160,8 +161,10 @@ titans_status_t titans_mem_forward_gated(titans_mem_t m, const void *k, const vo
  *         overwritten with the state after token T-1.
  *   attn  NULL for y = M(q), or the attention branch's output for the memory-as-a-gate output
  *         y = attn * sigmoid(M(q)) (see titans_mem_forward_gated).
- *   Other arguments as in titans_mem_forward. Runs the CUDA-core chunk kernel (fp32 arithmetic;
- *   k, q, v, y in the handle's dtype).
+ *   Other arguments as in titans_mem_forward. In TITANS_BF16 mode with 3..8 layers, chunk <= 128 and
+ *   no TITANS_FLAG_CUDA_CORES it runs the tensor-core phased kernel (bf16 operands, fp32
+ *   accumulation and state; TITANS_PATH_TC_DEEP); otherwise the CUDA-core chunk kernel (fp32
+ *   arithmetic; k, q, v, y in the handle's dtype).
  */
 titans_status_t titans_mem_forward_deep(titans_mem_t m, const void *k, const void *q, const void *v,
                                         const float *alpha, const float *eta, const float *theta,

@@ -72,6 +72,11 @@ bool tc_eligible(const titans_mem_config& c, int chunk) {
            chunk >= 1 && chunk <= 64;
 }
 
+bool deep_tc_eligible(const titans_mem_config& c, int layers, int chunk) {
+    return c.mode == TITANS_BF16 && !(c.flags & TITANS_FLAG_CUDA_CORES) &&
+           titans::tc_deep_supported(c.d, c.d_hidden, layers, chunk);
+}
+
 bool phased_eligible(const titans_mem_config& c, int chunk) {
     return c.mode == TITANS_BF16 && !(c.flags & TITANS_FLAG_CUDA_CORES) &&
            titans::tc_phased_supported(c.d, c.d_hidden, chunk);
@@ -190,6 +195,9 @@ titans_status_t init_impl(const titans_mem_config* cfg, int layers, titans_mem_t
     m->ws_per_unit = titans::cuda_cores_ws_floats(cfg->d, cfg->d_hidden, cfg->chunk);
     if (cfg->d_hidden)
         m->ws_per_unit = std::max(m->ws_per_unit, titans::deep_ws_floats(cfg->d, cfg->d_hidden, layers, cfg->chunk));
+    if (layers > 2 && deep_tc_eligible(*cfg, layers, cfg->chunk))
+        m->ws_per_unit = std::max(m->ws_per_unit,
+                                  (titans::tc_deep_ws_bytes_per_unit(cfg->d, cfg->d_hidden, layers) + 3) / sizeof(float));
     if (phased_eligible(*cfg, cfg->chunk))
         m->ws_per_unit = std::max(m->ws_per_unit, titans::tc_phased_ws_bytes_per_unit() / sizeof(float));
     if (cfg->d_hidden == 0 && (cfg->flags & TITANS_FLAG_CHUNK_SCAN)) {
@@ -238,7 +246,10 @@ titans_status_t titans_mem_destroy(titans_mem_t m) {
 
 int titans_mem_path(titans_mem_t m, int chunk, int step) {
     if (!m) return -1;
-    if (m->layers > 2) return (!step && chunk >= 1 && chunk <= m->cfg.chunk) ? TITANS_PATH_DEEP_CUDA_CORES : -1;
+    if (m->layers > 2) {
+        if (step || chunk < 1 || chunk > m->cfg.chunk) return -1;
+        return deep_tc_eligible(m->cfg, m->layers, chunk) ? TITANS_PATH_TC_DEEP : TITANS_PATH_DEEP_CUDA_CORES;
+    }
     if (step) return m->cfg.d_hidden ? TITANS_PATH_STEP_CLUSTER : TITANS_PATH_CUDA_CORES;
     if (chunk < 1 || chunk > m->cfg.chunk) return -1;
     if (m->cfg.d_hidden == 0 && (m->cfg.flags & TITANS_FLAG_CHUNK_SCAN)) return TITANS_PATH_LINEAR_SCAN;
@@ -318,7 +329,9 @@ titans_status_t titans_mem_forward_deep(titans_mem_t m, const void* k, const voi
     if (chunk < 1 || chunk > m->cfg.chunk) return fail(TITANS_EUNSUPPORTED, "chunk must be in 1..config.chunk");
     titans::ForwardArgs a = make_args(m, k, q, v, alpha, eta, theta, T, chunk, W, nullptr, S, nullptr, y);
     a.attn = attn;
-    cudaError_t e = titans::launch_chunk_deep_cuda_cores(a, m->layers, static_cast<cudaStream_t>(stream));
+    cudaError_t e = m->layers > 2 && deep_tc_eligible(m->cfg, m->layers, chunk)
+                        ? titans::launch_chunk_tc_deep(a, m->layers, m->status + 2, static_cast<cudaStream_t>(stream))
+                        : titans::launch_chunk_deep_cuda_cores(a, m->layers, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
     return TITANS_OK;
 }

@@ -42,6 +42,12 @@ size_t chunk_tc_mlp64_smem_bytes();
 size_t deep_ws_floats(int d, int h, int layers, int n);
 __host__ __device__ size_t deep_state_floats(int d, int h, int layers);
 cudaError_t launch_chunk_deep_cuda_cores(const ForwardArgs& a, int layers, cudaStream_t st);
+// Tensor-core chunk kernel of the deep memory (bf16, d in {64, 128}, h = 4d, 3..8 layers, chunk <= 128):
+// phased cooperative launch over all SMs like the wide 2-layer kernel; needs
+// tc_deep_ws_bytes_per_unit() bytes of workspace per unit and the two grid-barrier words `sync`.
+size_t tc_deep_ws_bytes_per_unit(int d, int h, int layers);
+bool tc_deep_supported(int d, int h, int layers, int chunk);
+cudaError_t launch_chunk_tc_deep(const ForwardArgs& a, int layers, unsigned* sync, cudaStream_t st);
 // Linear memory by the cross-chunk scan: up to nseg_max segments per unit, each needing
 // linear_scan_slot_floats(d, chunk) floats of workspace (a.ws, a.ws_per_unit floats per unit).
 size_t linear_scan_slot_floats(int d, int n);

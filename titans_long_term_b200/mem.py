@@ -25,7 +25,7 @@ FLAG_CUDA_CORES = 1
 FLAG_CHUNK_GATES = 2
 FLAG_CHUNK_SCAN = 4
 (PATH_TC_MLP64, PATH_CUDA_CORES, PATH_STEP_CLUSTER, PATH_TC_PHASED, PATH_DEEP_CUDA_CORES,
- PATH_LINEAR_SCAN) = 1, 2, 3, 4, 5, 6
+ PATH_LINEAR_SCAN, PATH_TC_DEEP) = 1, 2, 3, 4, 5, 6, 7
 
 EXPORTED = ["titans_mem_init", "titans_mem_destroy", "titans_mem_forward", "titans_mem_step",
             "titans_mem_path", "titans_mem_sync_status", "titans_last_error_string", "titans_mem_version",
