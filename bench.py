@@ -34,7 +34,8 @@ from titans_long_term_b200 import mem, synth  # noqa: E402
 
 METRIC = "memory tokens/sec (update+retrieve) per B200; % bf16 tensor-core peak"
 KERNEL_NAMES = {mem.PATH_TC_MLP64: "chunk_fwd_tc_mlp64", mem.PATH_CUDA_CORES: "chunk_fwd_cuda_cores",
-                mem.PATH_TC_PHASED: "chunk_fwd_tc_phased"}
+                mem.PATH_TC_PHASED: "chunk_fwd_tc_phased", mem.PATH_TC_DEEP: "chunk_fwd_tc_deep",
+                mem.PATH_DEEP_CUDA_CORES: "chunk_fwd_deep_cuda_cores"}
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -563,41 +564,49 @@ def extension_results(dev, steps: int, warmup: int):
     del toks, gates, state
     torch.cuda.empty_cache()
 
-    # deep memory (4 layers, 64 -> 256 -> 256 -> 256 -> 64) on the 8-unit 2K-token workload
-    w = synth.WORKLOADS["mlp-d64-b2h4-t2k"]
+    # deep memory (4 layers, 64 -> 256 -> 256 -> 256 -> 64): the 760M-class layer shape on the tensor-core
+    # kernel, and the 8-unit 2K-token workload on both kernels
     L = 4
-    toks, gates, _ = _dev_inputs(w, dev)
-    dst = {n: t.reshape(w.B, w.H, -1).to(dev) for n, t in synth.make_deep_state(w, L).items()}
-    flops = deep_flops_per_head_token(w.d, w.h, L) * w.units * w.T
-    for key, cuda_cores in (("deep_memory", False), ("deep_memory_cuda_cores", True)):
-        m = mem.Memory(w.d, w.h, w.chunk, w.dtype, w.B, w.H, layers=L, cuda_cores=cuda_cores)
-        st = {n: t.clone() for n, t in dst.items()}
-        fn = lambda: m.forward_deep(toks["k"], toks["q"], toks["v"], gates["alpha"], gates["eta"], gates["theta"], st)
-        n_deep = steps if not cuda_cores else 3
-        total, per = time_launches(fn, torch.cuda.current_stream(dev), n_deep, 1 if cuda_cores else warmup)
-        m.sync_status()
-        avg = statistics.mean(per)
-        if cuda_cores:
-            roof = _cuda_core_roofline(flops, avg, "chunk_fwd_deep_cuda_cores", w.units,
-                                       "fp32 on CUDA cores, one CTA per unit (TITANS_FLAG_CUDA_CORES)")
-        else:
-            achieved = flops / (avg / 1e3) / 1e12
-            roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                    "frac": achieved / peaks["bf16_tflops"], "traffic": None,
-                    "peak_source": f"bf16_tflops ({which})", "kernel": "chunk_fwd_tc_deep", "flops_per_launch": flops,
-                    "avg_launch_ms": avg}
-        out[key] = {
-            "workload": f"{w.name} deep L={L}", "value": w.B * w.T / (total / n_deep / 1e3), "unit": "tokens/s",
-            "ms_per_step": total / n_deep, "steps": n_deep,
-            "config": {"memory": f"deep {L}-layer {w.d}-{w.h}-{w.h}-{w.h}-{w.d} SiLU", "units": w.units, "T": w.T,
-                       "chunk": w.chunk, "flops_per_head_token": deep_flops_per_head_token(w.d, w.h, L),
-                       "path": "tensor cores (phased, all SMs)" if not cuda_cores else "CUDA cores"},
-            "roofline": roof, "gpu_launches": n_deep}
-        del m, st
-    del dst, toks, gates
-    torch.cuda.empty_cache()
+    for key, wname, kernels in (("deep_memory", "mlp-d64-b8h16-t4k", (False,)),
+                                ("deep_memory_8units", "mlp-d64-b2h4-t2k", (False, True))):
+        w = synth.WORKLOADS[wname]
+        toks, gates, _ = _dev_inputs(w, dev)
+        dst = {n: t.reshape(w.B, w.H, -1).to(dev) for n, t in synth.make_deep_state(w, L).items()}
+        flops = deep_flops_per_head_token(w.d, w.h, L) * w.units * w.T
+        rec = None
+        for cuda_cores in kernels:
+            m = mem.Memory(w.d, w.h, w.chunk, w.dtype, w.B, w.H, layers=L, cuda_cores=cuda_cores)
+            st = {n: t.clone() for n, t in dst.items()}
+            fn = lambda: m.forward_deep(toks["k"], toks["q"], toks["v"], gates["alpha"], gates["eta"], gates["theta"], st)
+            n_deep = steps if not cuda_cores else 3
+            total, per = time_launches(fn, torch.cuda.current_stream(dev), n_deep, 1 if cuda_cores else warmup)
+            m.sync_status()
+            avg = statistics.mean(per)
+            if cuda_cores:
+                rec["cuda_cores"] = {"ms_per_step": total / n_deep, "roofline": _cuda_core_roofline(
+                    flops, avg, "chunk_fwd_deep_cuda_cores", w.units, "fp32 on CUDA cores, one CTA per unit")}
+                rec["speedup_vs_cuda_cores"] = (total / n_deep) / rec["ms_per_step"]
+            else:
+                achieved = flops / (avg / 1e3) / 1e12
+                rec = {"workload": f"{w.name} deep L={L}", "value": w.B * w.T / (total / n_deep / 1e3), "unit": "tokens/s",
+                       "ms_per_step": total / n_deep, "steps": n_deep,
+                       "config": {"memory": f"deep {L}-layer {w.d}-{w.h}-{w.h}-{w.h}-{w.d} SiLU", "units": w.units,
+                                  "T": w.T, "chunk": w.chunk,
+                                  "flops_per_head_token": deep_flops_per_head_token(w.d, w.h, L),
+                                  "inputs": synth.describe(w)},
+                       "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
+                                    "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"], "traffic": None,
+                                    "peak_source": f"bf16_tflops ({which})", "kernel": "chunk_fwd_tc_deep",
+                                    "flops_per_launch": flops, "avg_launch_ms": avg},
+                       "gpu_launches": n_deep}
+            del m, st
+        out[key] = rec
+        del dst, toks, gates
+        torch.cuda.empty_cache()
 
-    # backward of the 2-layer memory (gradients of <dy, y> + <dW, W_T> ...) on the same workload
+    # backward of the 2-layer memory (gradients of <dy, y> with respect to every input) on the 8-unit workload
+    w = synth.WORKLOADS["mlp-d64-b2h4-t2k"]
+    n_deep = 3
     toks, gates, state = _dev_inputs(w, dev)
     dy = torch.randn(toks["k"].shape, generator=torch.Generator().manual_seed(5)).to(toks["k"].dtype).to(dev)
     m = mem.Memory(w.d, w.h, w.chunk, w.dtype, w.B, w.H)
@@ -617,6 +626,36 @@ def extension_results(dev, steps: int, warmup: int):
     del m, toks, gates, state, dy
     torch.cuda.empty_cache()
     return out
+
+
+def deep_arm(args, w, rank, world, local_rank):
+    """--phase deep: one JSON line for the deep memory (every rank runs its own B*H units)."""
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    L = args.layers
+    toks, gates, _ = _dev_inputs(w, dev)
+    dst = {n: t.reshape(w.B, w.H, -1).to(dev) for n, t in synth.make_deep_state(w, L).items()}
+    m = mem.Memory(w.d, w.h, w.chunk, w.dtype, w.B, w.H, layers=L)
+    fn = lambda: m.forward_deep(toks["k"], toks["q"], toks["v"], gates["alpha"], gates["eta"], gates["theta"], dst)
+    total, per = time_launches(fn, torch.cuda.current_stream(dev), args.steps, args.warmup)
+    m.sync_status()
+    ms = max_over_ranks(total / args.steps, dev, world)
+    if rank != 0:
+        return
+    peaks, which = load_peaks()
+    flops = deep_flops_per_head_token(w.d, w.h, L) * w.units * w.T
+    achieved = flops / (statistics.mean(per) / 1e3) / 1e12
+    print(json.dumps({
+        "metric": "deep memory tokens/sec (update+retrieve) per B200; % bf16 tensor-core peak",
+        "value": world * w.B * w.T / (ms / 1e3), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": w.dtype, "data": "synthetic (seeded)",
+        "config": {"workload": f"{w.name} deep L={L}", "layers": L, "units": w.units, "T": w.T, "chunk": w.chunk,
+                   "path": KERNEL_NAMES.get(m.path(), m.path())},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": achieved / peaks["bf16_tflops"], "traffic": None, "peak_source": f"bf16_tflops ({which})",
+                     "kernel": "chunk_fwd_tc_deep", "flops_per_launch": flops, "avg_launch_ms": statistics.mean(per)},
+        "gpu_launches": args.steps}), flush=True)
 
 
 def extra_results(args, dev):
@@ -657,8 +696,10 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the nested decode / long-stream / wide-prefill results of a 1-GPU run")
-    ap.add_argument("--phase", choices=["forward", "decode"], default="forward",
-                    help="forward: the chunk-wise update + retrieve (default); decode: titans_mem_step")
+    ap.add_argument("--phase", choices=["forward", "decode", "deep"], default="forward",
+                    help="forward: the chunk-wise update + retrieve (default); decode: titans_mem_step; "
+                         "deep: the deep memory's chunk-wise forward (--layers) on the tensor-core kernel")
+    ap.add_argument("--layers", type=int, default=4, help="depth of the deep memory for --phase deep")
     ap.add_argument("--decode-b", type=int, default=0, help="decode batch (default: the workload's, 256)")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -685,6 +726,8 @@ def main():
     try:
         if args.phase == "decode":
             decode_arm(args, w, rank, world, local_rank)
+        elif args.phase == "deep":
+            deep_arm(args, w, rank, world, local_rank)
         else:
             our_arm(args, w, rank, world, local_rank)
     finally:
