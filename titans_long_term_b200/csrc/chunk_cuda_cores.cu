@@ -31,7 +31,7 @@ __device__ __forceinline__ float gated(float yq, const Tin* attn, long idx) {
     return attn ? ldin(attn + idx) * (1.f / (1.f + expf(-yq))) : yq;
 }
 
-constexpr int kCcThreads = 256;
+constexpr int kCcThreads = 1024;
 constexpr int kCcMaxChunk = 128;
 
 // Workspace floats per unit for chunk length n (MLP: Zk, Ak, Aq, Dl [n][h] and G [n][d];

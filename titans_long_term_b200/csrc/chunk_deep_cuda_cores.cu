@@ -26,7 +26,7 @@ __device__ __forceinline__ float ld_in(const __nv_bfloat16* p) { return __bfloat
 __device__ __forceinline__ void st_out(float* p, float v) { *p = v; }
 __device__ __forceinline__ void st_out(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
 
-constexpr int kDeepThreads = 256;
+constexpr int kDeepThreads = 1024;
 constexpr int kDeepMaxChunk = 128;
 
 __device__ __forceinline__ float sigm(float z) { return 1.f / (1.f + expf(-z)); }

@@ -28,7 +28,7 @@ __device__ __forceinline__ float ldx(const __nv_bfloat16* p) { return __bfloat16
 __device__ __forceinline__ void stx(float* p, float v) { *p = v; }
 __device__ __forceinline__ void stx(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
 
-constexpr int kScanThreads = 256;
+constexpr int kScanThreads = 1024;
 constexpr int kScanMaxChunk = 128;
 
 // Per (unit, segment) workspace slot, in floats: R [3d][2d], P [3d][n], X [d][2d], G [n][d].

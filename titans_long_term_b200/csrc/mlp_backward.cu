@@ -39,16 +39,18 @@ __device__ __forceinline__ void stm(float* p, float v) { *p = v; }
 __device__ __forceinline__ void stm(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
 __device__ __forceinline__ float sgm(float z) { return 1.f / (1.f + expf(-z)); }
 
-constexpr int kMbThreads = 256;
+constexpr int kMbThreads = 1024;
 constexpr int kMbMaxChunk = 128;
 
 }  // namespace
 
 // Workspace floats per unit: every chunk-start state (4 h d each), two adjoint sets (2 x 4 h d), and
-// per-chunk activations: Z, A, B, Delta, dA, dZ, Zq, Aq ([n][h] each), G, dG ([n][d]).
+// per-chunk activations: Z, A, B, Delta, dA, dZ, Zq, Aq ([n][h] each), G, dG ([n][d]), and the terms of
+// dc_j, dd_j ([2][n][d + h]).
 size_t mlp_backward_ws_floats(int d, int h, long T, int chunk) {
     const long nch = (T + chunk - 1) / chunk;
-    return (size_t)nch * 4 * h * d + (size_t)8 * h * d + (size_t)8 * chunk * h + (size_t)2 * chunk * d;
+    return (size_t)nch * 4 * h * d + (size_t)8 * h * d + (size_t)8 * chunk * h + (size_t)2 * chunk * d +
+           (size_t)2 * chunk * (d + h);
 }
 
 template <typename Tin>
@@ -86,6 +88,8 @@ __global__ void __launch_bounds__(kMbThreads) mlp_backward_kernel(MlpBackwardArg
     float* Aq = Zq + nh;
     float* Gb = Aq + nh;                              // [n][d]
     float* dGb = Gb + (size_t)chunk * d;
+    float* Tc = dGb + (size_t)chunk * d;              // terms of dc_j, dd_j: [n][d + h] each
+    float* Td = Tc + (size_t)chunk * (d + h);
 
     auto scan = [&](long t0, int n) {
         for (int i = tid; i < n; i += blockDim.x) {
@@ -235,6 +239,10 @@ __global__ void __launch_bounds__(kMbThreads) mlp_backward_kernel(MlpBackwardArg
                 y2 += dS2e[(size_t)i * h + j] * aj;
             }
             dGb[idx] = -(s_c[t] * x2 + s_d[t] * y2);
+            // dc_j, dd_j terms -g_j . dW2' a_j, -g_j . dS2' a_j (summed per token below)
+            const float g = Gb[idx];
+            Tc[(size_t)t * (d + h) + i] = -g * x2;
+            Td[(size_t)t * (d + h) + i] = -g * y2;
         }
         // da_j = -(c_j dW2'^T + d_j dS2'^T) g_j;  ddelta_j = -(c_j dW1' + d_j dS1') k_j   [n][h]
         for (int idx = tid; idx < n * h; idx += blockDim.x) {
@@ -252,37 +260,32 @@ __global__ void __launch_bounds__(kMbThreads) mlp_backward_kernel(MlpBackwardArg
             }
             dAb[idx] = -(s_c[t] * x2 + s_d[t] * y2);
             const float ddel = -(s_c[t] * x1 + s_d[t] * y1);
+            // dc_j, dd_j terms -delta_j . dW1' k_j, -delta_j . dS1' k_j
+            Tc[(size_t)t * (d + h) + d + j] = -Dl[idx] * x1;
+            Td[(size_t)t * (d + h) + d + j] = -Dl[idx] * y1;
             // db = ddelta * silu'(z); dz = ddelta * b * silu''(z)
             const float z = Zb[idx], s = sgm(z);
             dZb[idx] = ddel * Bb[idx] * s * (1.f - s) * (2.f + z * (1.f - 2.f * s));
             Bb[idx] = ddel * s * (1.f + z * (1.f - s));  // Bb now holds db
         }
         __syncthreads();
-        // dc_j, dd_j
-        for (int t = tid; t < n; t += blockDim.x) {
+        // dc_j, dd_j: one warp per token sums its d + h terms in a fixed order (lane-strided, then
+        // a shuffle tree), so the result does not depend on scheduling.
+        for (int t = tid >> 5; t < n; t += blockDim.x >> 5) {
+            const int lane = tid & 31;
             float sc = 0.f, sd = 0.f;
-            for (int i = 0; i < d; ++i) {  // -g_j . dW2' a_j == g_j . dg_j / c_j when c_j != 0; computed directly
-                float x2 = 0.f, y2 = 0.f;
-                for (int j = 0; j < h; ++j) {
-                    const float aj = Ab[(size_t)t * h + j];
-                    x2 += dW2e[(size_t)i * h + j] * aj;
-                    y2 += dS2e[(size_t)i * h + j] * aj;
-                }
-                sc -= Gb[(size_t)t * d + i] * x2;
-                sd -= Gb[(size_t)t * d + i] * y2;
+            for (int i = lane; i < d + h; i += 32) {
+                sc += Tc[(size_t)t * (d + h) + i];
+                sd += Td[(size_t)t * (d + h) + i];
             }
-            for (int j = 0; j < h; ++j) {
-                float x1 = 0.f, y1 = 0.f;
-                for (int m = 0; m < d; ++m) {
-                    const float km = ldm(k + (t0 + t) * d + m);
-                    x1 += dW1e[(size_t)j * d + m] * km;
-                    y1 += dS1e[(size_t)j * d + m] * km;
-                }
-                sc -= Dl[(size_t)t * h + j] * x1;
-                sd -= Dl[(size_t)t * h + j] * y1;
+            for (int off = 16; off > 0; off >>= 1) {
+                sc += __shfl_xor_sync(0xffffffffu, sc, off);
+                sd += __shfl_xor_sync(0xffffffffu, sd, off);
             }
-            s_dc[t] = sc;
-            s_dd[t] = sd;
+            if (lane == 0) {
+                s_dc[t] = sc;
+                s_dd[t] = sd;
+            }
         }
         // dg_j += W2 db_j;  then dyhat = 2 dg, dv = -2 dg
         for (int idx = tid; idx < n * d; idx += blockDim.x) {
