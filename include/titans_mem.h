@@ -89,7 +89,8 @@ typedef enum {
     TITANS_PATH_TC_PHASED = 4,    /* tcgen05 bf16 chunk kernel over all SMs, d=128, h=512, chunk<=128 */
     TITANS_PATH_DEEP_CUDA_CORES = 5, /* deep memory (titans_mem_init_deep), CUDA-core chunk kernel */
     TITANS_PATH_LINEAR_SCAN = 6,     /* linear memory, cross-chunk scan (TITANS_FLAG_CHUNK_SCAN) */
-    TITANS_PATH_TC_DEEP = 7          /* deep memory, tcgen05 bf16 phased kernel over all SMs (L >= 3) */
+    TITANS_PATH_TC_DEEP = 7,         /* deep memory, tcgen05 bf16 phased kernel over all SMs (L >= 3) */
+    TITANS_PATH_TC_BACKWARD = 8      /* backward, tcgen05 bf16, one CTA per unit (d=64, h=256, chunk<=64) */
 } titans_path_t;
 
 /* Validates the configuration and allocates the handle, its device status word and
@@ -284,8 +285,8 @@ titans_status_t titans_mem_backward(titans_mem_t m, const void *k, const void *q
                                     float *dW2_0, float *dS1_0, float *dS2_0, void *workspace,
                                     size_t workspace_bytes, void *stream);
 
-/* Kernel that titans_mem_forward (step = 0) or titans_mem_step (step = 1) would run with
- * this chunk length; negative on an unsupported combination. */
+/* Kernel that titans_mem_forward (step = 0), titans_mem_step (step = 1) or titans_mem_backward
+ * (step = 2) would run with this chunk length; negative on an unsupported combination. */
 int titans_mem_path(titans_mem_t m, int chunk, int step);
 
 /* Synchronises the stream, then reads and clears the handle's device status word.

@@ -73,7 +73,11 @@ def _mlp_case(B, H, T, chunk, mode, seed, with_dstate, recipe=None):
     (2, 1, 64, 64, "fp32", False, None),      # one chunk, loss on y only
     (1, 2, 12, 1, "fp32", True, None),        # chunk = 1
     (1, 2, 64, 32, "fp32", True, "stated"),   # the stated gate ranges
-    (1, 2, 48, 16, "bf16", True, None),       # bf16 token streams
+    (1, 2, 48, 16, "bf16", True, None),       # bf16 token streams (the tensor-core backward from here on)
+    (2, 2, 200, 64, "bf16", True, None),      # several chunks, ragged last chunk
+    (1, 2, 64, 64, "bf16", False, None),      # one chunk, loss on y only
+    (1, 2, 9, 1, "bf16", True, None),         # chunk = 1
+    (1, 2, 64, 32, "bf16", True, "stated"),   # the stated gate ranges, over the two chunks the memory stays bounded
 ])
 def test_mlp_backward_matches_the_oracle(B, H, T, chunk, mode, with_dstate, recipe):
     """The MLP memory's adjoint includes the second-order terms of the inner gradient (its update
@@ -81,6 +85,7 @@ def test_mlp_backward_matches_the_oracle(B, H, T, chunk, mode, with_dstate, reci
     w, inp, dy, dst = _mlp_case(B, H, T, chunk, mode, T + chunk, with_dstate, recipe)
     U = B * H
     m = mem.Memory(64, 256, chunk, mode, B, H)
+    assert m.backward_path(chunk) == (mem.PATH_TC_BACKWARD if mode == "bf16" else mem.PATH_CUDA_CORES)
     dev = lambda x: x.reshape(B, H, *x.shape[1:]).cuda().contiguous()
     args = [dev(inp[n]) for n in ("k", "q", "v", "alpha", "eta", "theta")]
     state = {n: dev(inp[n]) for n in ("W1", "W2", "S1", "S2")}
@@ -115,3 +120,22 @@ def test_backward_leaves_its_inputs_alone_and_rejects_a_deep_memory():
         deep.backward(z, z, z, gz, gz, gz, {"W1": torch.zeros(1, 1, 256, 64, device="cuda"),
                                             "S1": torch.zeros(1, 1, 256, 64, device="cuda")}, z)
     assert ei.value.status == mem.EUNSUPPORTED
+
+
+def test_mlp_backward_tensor_cores_against_cuda_cores():
+    """The bf16 tensor-core backward and the fp32 CUDA-core one (TITANS_FLAG_CUDA_CORES) on the same
+    inputs: each within the bf16 bar of the oracle's gradients."""
+    B, H, T, chunk = 2, 2, 256, 64
+    w, inp, dy, dst = _mlp_case(B, H, T, chunk, "bf16", 3, True)
+    dev = lambda x: x.reshape(B, H, *x.shape[1:]).cuda().contiguous()
+    args = [dev(inp[n]) for n in ("k", "q", "v", "alpha", "eta", "theta")]
+    state = {n: dev(inp[n]) for n in ("W1", "W2", "S1", "S2")}
+    ref = oracle.backward(inp["k"], inp["q"], inp["v"], inp["alpha"], inp["eta"], inp["theta"],
+                          {n: inp[n] for n in ("W1", "W2", "S1", "S2")}, chunk, dy.float(), dst)
+    for cuda_cores in (False, True):
+        m = mem.Memory(64, 256, chunk, "bf16", B, H, cuda_cores=cuda_cores)
+        out = m.backward(*args, state, dev(dy), {n: dev(x) for n, x in dst.items()}, chunk=chunk)
+        m.sync_status()
+        for n in ("k", "q", "v", "alpha", "eta", "theta", "W1", "W2", "S1", "S2"):
+            e = rel_err(out[n].reshape(B * H, -1).float().cpu().numpy(), ref[n].reshape(B * H, -1))
+            assert e.max() <= TOL["bf16"], f"{'CUDA cores' if cuda_cores else 'tensor cores'} d{n}: {e.max():.3e}"

@@ -23,7 +23,7 @@ BUILD_DEBUG = os.path.join(HERE, "_build_debug")
 LIB_DEBUG = os.path.join(HERE, "libtitans_mem_debug.so")
 SOURCES = ["api.cu", "chunk_cuda_cores.cu", "chunk_deep_cuda_cores.cu", "chunk_tc_mlp64.cu", "chunk_tc_phased.cu",
            "chunk_tc_deep.cu", "step_cluster.cu", "forward_noalloc.cu", "linear_scan.cu",
-           "linear_backward.cu", "mlp_backward.cu"]
+           "linear_backward.cu", "mlp_backward.cu", "mlp_backward_tc.cu"]
 HEADERS = ["kernels.h", "ptx.cuh", "phased_common.cuh"]
 NVCC = os.environ.get("NVCC", "nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

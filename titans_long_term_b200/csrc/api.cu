@@ -77,6 +77,11 @@ bool deep_tc_eligible(const titans_mem_config& c, int layers, int chunk) {
            titans::tc_deep_supported(c.d, c.d_hidden, layers, chunk);
 }
 
+bool backward_tc_eligible(const titans_mem_config& c, int chunk) {
+    return c.mode == TITANS_BF16 && !(c.flags & TITANS_FLAG_CUDA_CORES) && c.d_hidden != 0 &&
+           titans::mlp_backward_tc_supported(c.d, c.d_hidden, chunk);
+}
+
 bool phased_eligible(const titans_mem_config& c, int chunk) {
     return c.mode == TITANS_BF16 && !(c.flags & TITANS_FLAG_CUDA_CORES) &&
            titans::tc_phased_supported(c.d, c.d_hidden, chunk);
@@ -246,6 +251,10 @@ titans_status_t titans_mem_destroy(titans_mem_t m) {
 
 int titans_mem_path(titans_mem_t m, int chunk, int step) {
     if (!m) return -1;
+    if (step == 2) {  // titans_mem_backward
+        if (m->layers > 2 || (m->cfg.flags & TITANS_FLAG_CHUNK_GATES) || chunk < 1 || chunk > m->cfg.chunk) return -1;
+        return backward_tc_eligible(m->cfg, chunk) ? TITANS_PATH_TC_BACKWARD : TITANS_PATH_CUDA_CORES;
+    }
     if (m->layers > 2) {
         if (step || chunk < 1 || chunk > m->cfg.chunk) return -1;
         return deep_tc_eligible(m->cfg, m->layers, chunk) ? TITANS_PATH_TC_DEEP : TITANS_PATH_DEEP_CUDA_CORES;
@@ -465,8 +474,10 @@ titans_status_t titans_mem_step_gated(titans_mem_t m, const void* k, const void*
 
 size_t titans_mem_backward_workspace_bytes(titans_mem_t m, long T, int chunk) {
     if (!m || T < 1 || chunk < 1) return 0;
-    const size_t f = m->cfg.d_hidden ? titans::mlp_backward_ws_floats(m->cfg.d, m->cfg.d_hidden, T, chunk)
-                                     : titans::linear_backward_ws_floats(m->cfg.d, T, chunk);
+    size_t f = m->cfg.d_hidden ? titans::mlp_backward_ws_floats(m->cfg.d, m->cfg.d_hidden, T, chunk)
+                               : titans::linear_backward_ws_floats(m->cfg.d, T, chunk);
+    if (backward_tc_eligible(m->cfg, chunk))
+        f = std::max(f, (titans::mlp_backward_tc_ws_bytes(T, chunk) + sizeof(float) - 1) / sizeof(float));
     const size_t per_unit = (f + 63) & ~size_t(63);
     return per_unit * sizeof(float) * (size_t)m->cfg.B * m->cfg.H;
 }
@@ -541,7 +552,9 @@ titans_status_t titans_mem_backward(titans_mem_t m, const void* k, const void* q
         b.dS2_0 = dS2_0;
         b.ws = static_cast<float*>(workspace);
         b.ws_per_unit = need / sizeof(float) / (size_t)units;
-        e = titans::launch_mlp_backward(b, static_cast<cudaStream_t>(stream));
+        b.status = m->status;
+        e = backward_tc_eligible(m->cfg, chunk) ? titans::launch_mlp_backward_tc(b, static_cast<cudaStream_t>(stream))
+                                                : titans::launch_mlp_backward(b, static_cast<cudaStream_t>(stream));
     } else {
         titans::LinearBackwardArgs b{};
         b.d = m->cfg.d;

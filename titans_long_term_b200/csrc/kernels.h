@@ -79,9 +79,15 @@ struct MlpBackwardArgs {
     float *dW1_0, *dW2_0, *dS1_0, *dS2_0;
     float* ws;
     size_t ws_per_unit;  // floats
+    unsigned* status;    // device status word (the tensor-core backward's bounded waits)
 };
 size_t mlp_backward_ws_floats(int d, int h, long T, int chunk);
 cudaError_t launch_mlp_backward(const MlpBackwardArgs& a, cudaStream_t st);
+// Tensor-core backward of the 2-layer memory (bf16, d = 64, h = 256, chunk <= 64): one CTA per unit,
+// mlp_backward_tc_ws_bytes() of workspace per unit (MlpBackwardArgs::ws_per_unit floats apart).
+bool mlp_backward_tc_supported(int d, int h, int chunk);
+size_t mlp_backward_tc_ws_bytes(long T, int chunk);
+cudaError_t launch_mlp_backward_tc(const MlpBackwardArgs& a, cudaStream_t st);
 cudaError_t launch_linear_backward(const LinearBackwardArgs& b, cudaStream_t st);
 size_t tc_phased_ws_bytes_per_unit();
 bool tc_phased_supported(int d, int h, int chunk);

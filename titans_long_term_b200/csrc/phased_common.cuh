@@ -125,5 +125,40 @@ __device__ __forceinline__ bool grid_sync(unsigned* sync, unsigned* status, unsi
     return *s_ok != 0;
 }
 
+// Operand copies into the 128-byte-swizzled layouts the MMA descriptors describe.
+//   K-major: element (r, k) at src[r * ld + k]; per 64-element K block kb a [R][64] tile at
+//            dst + kb * R * 128; rows r >= valid_r are zero.
+//   MN-major: element (r, k) at src[k * ld + r]; per 64-element K block kb and 64-element R block rb
+//            a [64 k][64 r] tile at dst + (kb * R / 64 + rb) * 8192; K rows k >= valid_k are zero.
+__device__ __forceinline__ void load_kmajor(uint32_t dst, const __nv_bfloat16* src, size_t ld, int R, int valid_r,
+                                            int k0, int kc) {
+    for (int kb = 0; kb < kc / 64; ++kb)
+        load_tile(dst + (uint32_t)(kb * R * 128), reinterpret_cast<const uint8_t*>(src + k0 + kb * 64), ld * 2, R,
+                  valid_r);
+}
+__device__ __forceinline__ void load_mnmajor(uint32_t dst, const __nv_bfloat16* src, size_t ld, int R, int k0,
+                                             int kc, int valid_k) {
+    for (int kb = 0; kb < kc / 64; ++kb)
+        for (int rb = 0; rb < R / 64; ++rb)
+            load_tile(dst + (uint32_t)((kb * (R / 64) + rb) * 8192),
+                      reinterpret_cast<const uint8_t*>(src + (size_t)(k0 + kb * 64) * ld + rb * 64), ld * 2, 64,
+                      valid_k - (k0 + kb * 64));
+}
+// Descriptor of K-step ks (16 elements) of an operand loaded by the functions above.
+__device__ __forceinline__ uint64_t desc_k(uint32_t base, int R, int ks) {
+    return sdesc_sw128(base + (uint32_t)((ks >> 2) * R * 128 + (ks & 3) * 32), 16, 1024);
+}
+__device__ __forceinline__ uint64_t desc_mn(uint32_t base, int R, int ks) {
+    return sdesc_sw128(base + (uint32_t)((ks >> 2) * (R / 64) * 8192 + (ks & 3) * 2048), 8192, 1024);
+}
+
+__device__ __forceinline__ void mma_steps(uint32_t d_tmem, uint32_t a, bool a_mn, uint32_t b, bool b_mn, int N,
+                                          int ksteps, bool acc) {
+    const uint32_t id = idesc_bf16_f32(128, N, a_mn ? 1 : 0, b_mn ? 1 : 0);
+    for (int ks = 0; ks < ksteps; ++ks)
+        umma_bf16(d_tmem, a_mn ? desc_mn(a, 128, ks) : desc_k(a, 128, ks), b_mn ? desc_mn(b, N, ks) : desc_k(b, N, ks),
+                  id, (acc || ks > 0) ? 1u : 0u);
+}
+
 }  // namespace phc
 }  // namespace titans

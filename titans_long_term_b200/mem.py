@@ -25,7 +25,7 @@ FLAG_CUDA_CORES = 1
 FLAG_CHUNK_GATES = 2
 FLAG_CHUNK_SCAN = 4
 (PATH_TC_MLP64, PATH_CUDA_CORES, PATH_STEP_CLUSTER, PATH_TC_PHASED, PATH_DEEP_CUDA_CORES,
- PATH_LINEAR_SCAN, PATH_TC_DEEP) = 1, 2, 3, 4, 5, 6, 7
+ PATH_LINEAR_SCAN, PATH_TC_DEEP, PATH_TC_BACKWARD) = 1, 2, 3, 4, 5, 6, 7, 8
 
 EXPORTED = ["titans_mem_init", "titans_mem_destroy", "titans_mem_forward", "titans_mem_step",
             "titans_mem_path", "titans_mem_sync_status", "titans_last_error_string", "titans_mem_version",
@@ -137,6 +137,10 @@ class Memory:
 
     def path(self, chunk: Optional[int] = None, step: bool = False) -> int:
         return lib().titans_mem_path(self._h, chunk or self.chunk, int(step))
+
+    def backward_path(self, chunk: Optional[int] = None) -> int:
+        """Kernel titans_mem_backward runs with this chunk length."""
+        return lib().titans_mem_path(self._h, chunk or self.chunk, 2)
 
     def _gate_lead(self, lead, chunk):
         """Shape of a gate array: one value per token, or per chunk with chunk-shared gates."""
