@@ -604,27 +604,48 @@ def extension_results(dev, steps: int, warmup: int):
         del dst, toks, gates
         torch.cuda.empty_cache()
 
-    # backward of the 2-layer memory (gradients of <dy, y> with respect to every input) on the 8-unit workload
-    w = synth.WORKLOADS["mlp-d64-b2h4-t2k"]
-    n_deep = 3
-    toks, gates, state = _dev_inputs(w, dev)
-    dy = torch.randn(toks["k"].shape, generator=torch.Generator().manual_seed(5)).to(toks["k"].dtype).to(dev)
-    m = mem.Memory(w.d, w.h, w.chunk, w.dtype, w.B, w.H)
-    fn = lambda: m.backward(toks["k"], toks["q"], toks["v"], gates["alpha"], gates["eta"], gates["theta"], state, dy)
-    total, per = time_launches(fn, torch.cuda.current_stream(dev), n_deep, 1)
-    m.sync_status()
-    flops = 2 * flops_per_head_token(w) * w.units * w.T
-    out["backward"] = {
-        "workload": f"{w.name} backward", "value": w.B * w.T / (total / n_deep / 1e3), "unit": "tokens/s",
-        "ms_per_step": total / n_deep, "steps": n_deep,
-        "config": {"memory": f"MLP {w.d}-{w.h}-{w.d} SiLU", "units": w.units, "T": w.T, "chunk": w.chunk,
-                   "flops_per_head_token": 2 * flops_per_head_token(w)},
-        "roofline": _cuda_core_roofline(flops, statistics.mean(per), "mlp_backward_kernel", w.units,
-                                        "fp32 on CUDA cores, one CTA per unit; FLOPs counted as twice the "
-                                        "forward's 18 d h per head-token (the chunk forward is recomputed too)"),
-        "gpu_launches": n_deep}
-    del m, toks, gates, state, dy
-    torch.cuda.empty_cache()
+    # backward of the 2-layer memory (gradients of <dy, y> with respect to every input): the 760M-class
+    # workload on the tensor-core backward, and the 8-unit 2K-token workload on both backward kernels
+    for key, wname, kernels in (("backward", "mlp-d64-b8h16-t4k", (False,)),
+                                ("backward_8units", "mlp-d64-b2h4-t2k", (False, True))):
+        w = synth.WORKLOADS[wname]
+        toks, gates, state = _dev_inputs(w, dev)
+        dy = torch.randn(toks["k"].shape, generator=torch.Generator().manual_seed(5)).to(toks["k"].dtype).to(dev)
+        flops = 2 * flops_per_head_token(w) * w.units * w.T
+        rec = None
+        for cuda_cores in kernels:
+            m = mem.Memory(w.d, w.h, w.chunk, w.dtype, w.B, w.H, cuda_cores=cuda_cores)
+            fn = lambda: m.backward(toks["k"], toks["q"], toks["v"], gates["alpha"], gates["eta"], gates["theta"],
+                                    state, dy)
+            nb = 3
+            total, per = time_launches(fn, torch.cuda.current_stream(dev), nb, 1)
+            m.sync_status()
+            avg = statistics.mean(per)
+            if cuda_cores:
+                rec["cuda_cores"] = {"ms_per_step": total / nb, "roofline": _cuda_core_roofline(
+                    flops, avg, "mlp_backward_kernel", w.units,
+                    "fp32 on CUDA cores, one CTA per unit (TITANS_FLAG_CUDA_CORES)")}
+                rec["speedup_vs_cuda_cores"] = (total / nb) / rec["ms_per_step"]
+            else:
+                achieved = flops / (avg / 1e3) / 1e12
+                sms = min(w.units, 148)
+                rec = {"workload": f"{w.name} backward", "value": w.B * w.T / (total / nb / 1e3), "unit": "tokens/s",
+                       "ms_per_step": total / nb, "steps": nb,
+                       "config": {"memory": f"MLP {w.d}-{w.h}-{w.d} SiLU", "units": w.units, "T": w.T,
+                                  "chunk": w.chunk, "flops_per_head_token": 2 * flops_per_head_token(w),
+                                  "inputs": synth.describe(w)},
+                       "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
+                                    "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"], "traffic": None,
+                                    "peak_source": f"bf16_tflops ({which})", "kernel": "mlp_backward_tc_kernel",
+                                    "flops_per_launch": flops, "avg_launch_ms": avg, "sms_used": sms,
+                                    "frac_of_sms_used": achieved / (peaks["bf16_tflops"] * sms / 148),
+                                    "note": "FLOPs counted as twice the forward's 18 d h per head-token; the "
+                                            "kernel also reruns the forward once to keep the chunk-start states"},
+                       "gpu_launches": nb}
+            del m
+        out[key] = rec
+        del toks, gates, state, dy
+        torch.cuda.empty_cache()
     return out
 
 

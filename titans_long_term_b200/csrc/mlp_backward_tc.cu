@@ -108,21 +108,15 @@ __device__ __forceinline__ void ld16_bf16(const __nv_bfloat16* src, float (&x)[1
         x[2 * i + 1] = f.y;
     }
 }
-__device__ __forceinline__ void st16_f32(float* dst, const float (&x)[16]) {
-    float4* p = reinterpret_cast<float4*>(dst);
+// fp32 per-token scratch is stored token-contiguous ([column][64 tokens]) so that the 32 lanes of a
+// warp, one token row each, read and write 128 contiguous bytes per column.
+__device__ __forceinline__ void ldcol16(const float* base, int col, int t, float (&x)[16]) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) p[i] = make_float4(x[4 * i], x[4 * i + 1], x[4 * i + 2], x[4 * i + 3]);
+    for (int e = 0; e < 16; ++e) x[e] = base[(size_t)(col + e) * 64 + t];
 }
-__device__ __forceinline__ void ld16_f32(const float* src, float (&x)[16]) {
-    const float4* p = reinterpret_cast<const float4*>(src);
+__device__ __forceinline__ void stcol16(float* base, int col, int t, const float (&x)[16]) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const float4 v = p[i];
-        x[4 * i] = v.x;
-        x[4 * i + 1] = v.y;
-        x[4 * i + 2] = v.z;
-        x[4 * i + 3] = v.w;
-    }
+    for (int e = 0; e < 16; ++e) base[(size_t)(col + e) * 64 + t] = x[e];
 }
 __device__ __forceinline__ void tmem16(uint32_t taddr, float (&x)[16]) {
     uint32_t r[16];
@@ -332,11 +326,11 @@ __global__ void __launch_bounds__(mbt::kThreads, 1) mlp_backward_tc_kernel(const
             }
             if (row < 64) {
                 st16_bf16(PQ + (size_t)(128 + row) * kH + col, o1);
-                st16_f32(SP + (size_t)row * kH + col, o2);
-                if (pass2) st16_f32(SPP + (size_t)row * kH + col, o3);
+                stcol16(SP, col, row, o2);
+                if (pass2) stcol16(SPP, col, row, o3);
             } else {
                 st16_bf16(PQ + (size_t)row * kH + col, o1);
-                st16_f32(SPQ + (size_t)(row - 64) * kH + col, o2);
+                stcol16(SPQ, col, row - 64, o2);
             }
         }
         gemm(256, PQ + (size_t)64 * kH, kH, false, W2b, kH, false, kD, kH);  // [A_q; A] W2^T
@@ -356,7 +350,7 @@ __global__ void __launch_bounds__(mbt::kThreads, 1) mlp_backward_tc_kernel(const
                     gc[e] = cr * g[e];
                     gd[e] = dr * g[e];
                 }
-                st16_f32(GF + (size_t)t * kD + col, g);
+                stcol16(GF, col, t, g);
                 st16_bf16(GQ + (size_t)t * kD + col, g);
                 st16_bf16(CG + (size_t)t * 2 * kD + col, gc);
                 st16_bf16(CG + (size_t)t * 2 * kD + kD + col, gd);
@@ -370,13 +364,13 @@ __global__ void __launch_bounds__(mbt::kThreads, 1) mlp_backward_tc_kernel(const
             float b[16], s[16], o[16];
             tmem16(tmem + lane_off + col, b);
             if (row < 64) {
-                ld16_f32(SP + (size_t)row * kH + col, s);
+                ldcol16(SP, col, row, s);
 #pragma unroll
                 for (int e = 0; e < 16; ++e) o[e] = b[e] * s[e];
                 st16_bf16(DL + (size_t)row * kH + col, o);
-                if (pass2) st16_f32(BM + (size_t)row * kH + col, b);
+                if (pass2) stcol16(BM, col, row, b);
             } else if (pass2) {
-                ld16_f32(SPQ + (size_t)(row - 64) * kH + col, s);
+                ldcol16(SPQ, col, row - 64, s);
 #pragma unroll
                 for (int e = 0; e < 16; ++e) o[e] = b[e] * s[e];
                 st16_bf16(DZ + (size_t)row * kH + col, o);
@@ -416,29 +410,44 @@ __global__ void __launch_bounds__(mbt::kThreads, 1) mlp_backward_tc_kernel(const
         }
         if (!ok) break;
         const float An = s_scal[0], En = s_scal[1], sig = s_scal[2];
-        for (int mt = 0; mt < 2; ++mt) {
-            const int j = 128 * mt + row;
+        // The accumulators go through shared memory (rows of 65 floats) so that the state update
+        // reads and writes W, S with consecutive threads on consecutive elements. W1 and S1 first
+        // (TMEM columns 128 mt: c part, + 64: d part), then W2 and S2 (columns 256 + 128 mt).
+        float* st_c = reinterpret_cast<float*>(sm);
+        float* st_d = st_c + 256 * 65;
+        for (int part = 0; part < 2; ++part) {
+            tc_fence_before();
+            __syncthreads();
+            tc_fence_after();
+            for (int mt = 0; mt < 2; ++mt) {
+                const int j = 128 * mt + row;
 #pragma unroll 1
-            for (int blk = 0; blk < 2; ++blk) {
-                const int col = 32 * half + 16 * blk;
-                float ac[16], ad[16];
-                tmem16(tmem + lane_off + 128 * mt + col, ac);
-                tmem16(tmem + lane_off + 128 * mt + kD + col, ad);
+                for (int blk = 0; blk < 2; ++blk) {
+                    const int col = 32 * half + 16 * blk;
+                    float ac[16], ad[16];
+                    tmem16(tmem + lane_off + 256 * part + 128 * mt + col, ac);
+                    tmem16(tmem + lane_off + 256 * part + 128 * mt + kD + col, ad);
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {  // W1, S1 row j
-                    const size_t x = (size_t)j * kD + col + e;
-                    const float w = X[x], s = X[2 * kHD + x];
-                    Xn[x] = fmaf(An, w, sig * s) - ac[e];
-                    Xn[2 * kHD + x] = En * s - ad[e];
+                    for (int e = 0; e < 16; ++e) {
+                        st_c[j * 65 + col + e] = ac[e];
+                        st_d[j * 65 + col + e] = ad[e];
+                    }
                 }
-                tmem16(tmem + lane_off + 256 + 128 * mt + col, ac);
-                tmem16(tmem + lane_off + 256 + 128 * mt + kD + col, ad);
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {  // W2, S2 column j
-                    const size_t x = (size_t)(col + e) * kH + j;
-                    const float w = X[kHD + x], s = X[3 * kHD + x];
-                    Xn[kHD + x] = fmaf(An, w, sig * s) - ac[e];
-                    Xn[3 * kHD + x] = En * s - ad[e];
+            }
+            __syncthreads();
+            if (part == 0) {
+                for (size_t i = tid; i < kHD; i += kThreads) {  // W1, S1 [h][d]
+                    const size_t j = i / kD, m = i % kD;
+                    const float w = X[i], sv = X[2 * kHD + i];
+                    Xn[i] = fmaf(An, w, sig * sv) - st_c[j * 65 + m];
+                    Xn[2 * kHD + i] = En * sv - st_d[j * 65 + m];
+                }
+            } else {
+                for (size_t i = tid; i < kHD; i += kThreads) {  // W2, S2 [d][h]
+                    const size_t r = i / kH, j = i % kH;
+                    const float w = X[kHD + i], sv = X[3 * kHD + i];
+                    Xn[kHD + i] = fmaf(An, w, sig * sv) - st_c[j * 65 + r];
+                    Xn[3 * kHD + i] = En * sv - st_d[j * 65 + r];
                 }
             }
         }
@@ -484,14 +493,14 @@ __global__ void __launch_bounds__(mbt::kThreads, 1) mlp_backward_tc_kernel(const
                     float x2[16], y2[16], g[16], o[16];
                     tmem16(tmem + lane_off + 256 + col, x2);
                     tmem16(tmem + lane_off + 256 + kD + col, y2);
-                    ld16_f32(GF + (size_t)t * kD + col, g);
+                    ldcol16(GF, col, t, g);
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
                         o[e] = -(s_c[t] * x2[e] + s_d[t] * y2[e]);
                         pc -= g[e] * x2[e];
                         pd -= g[e] * y2[e];
                     }
-                    st16_f32(DG0 + (size_t)t * kD + col, o);
+                    stcol16(DG0, col, t, o);
                 }
             }
             s_part[half * 128 + row] = pc;
@@ -515,11 +524,11 @@ __global__ void __launch_bounds__(mbt::kThreads, 1) mlp_backward_tc_kernel(const
                 tmem16(tmem + lane_off + col, x);
 #pragma unroll
                 for (int e = 0; e < 16; ++e) o[e] = -x[e];
-                st16_f32(DA0 + (size_t)t * kH + col, o);
+                stcol16(DA0, col, t, o);
                 tmem16(tmem + lane_off + 256 + col, y);
-                ld16_f32(SP + (size_t)t * kH + col, s);
-                ld16_f32(BM + (size_t)t * kH + col, b);
-                ld16_f32(SPP + (size_t)t * kH + col, s2);
+                ldcol16(SP, col, t, s);
+                ldcol16(BM, col, t, b);
+                ldcol16(SPP, col, t, s2);
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
                     const float ddel = -y[e];
@@ -527,7 +536,7 @@ __global__ void __launch_bounds__(mbt::kThreads, 1) mlp_backward_tc_kernel(const
                     x[e] = ddel * b[e] * s2[e];  // dz0
                 }
                 st16_bf16(PQ + (size_t)t * kH + col, o);
-                st16_f32(DZ0 + (size_t)t * kH + col, x);
+                stcol16(DZ0, col, t, x);
             }
         }
         // dG = dG0 + db W2^T; dyhat = 2 dG, dv = -2 dG
@@ -540,7 +549,7 @@ __global__ void __launch_bounds__(mbt::kThreads, 1) mlp_backward_tc_kernel(const
                 const int col = 32 * half + 16 * blk;
                 float x[16], g0[16], o[16], ov[16];
                 tmem16(tmem + lane_off + col, x);
-                ld16_f32(DG0 + (size_t)t * kD + col, g0);
+                ldcol16(DG0, col, t, g0);
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
                     const float g = g0[e] + x[e];
@@ -561,9 +570,9 @@ __global__ void __launch_bounds__(mbt::kThreads, 1) mlp_backward_tc_kernel(const
                 const int col = 128 * half + 16 * blk;
                 float x[16], a0[16], s[16], z0[16], o[16];
                 tmem16(tmem + lane_off + col, x);
-                ld16_f32(DA0 + (size_t)t * kH + col, a0);
-                ld16_f32(SP + (size_t)t * kH + col, s);
-                ld16_f32(DZ0 + (size_t)t * kH + col, z0);
+                ldcol16(DA0, col, t, a0);
+                ldcol16(SP, col, t, s);
+                ldcol16(DZ0, col, t, z0);
 #pragma unroll
                 for (int e = 0; e < 16; ++e) o[e] = z0[e] + (a0[e] + x[e]) * s[e];
                 st16_bf16(DZ + (size_t)t * kH + col, o);
@@ -614,42 +623,54 @@ __global__ void __launch_bounds__(mbt::kThreads, 1) mlp_backward_tc_kernel(const
         if (!ok) break;
         {
             const float An = s_scal[0], En = s_scal[1], sig = s_scal[2];
-            float pa = 0.f, ps = 0.f, pe = 0.f;
+            // The accumulators (dW1 tiles at TMEM columns 64 mt, dW2^T tiles at 128 + 64 mt) go through
+            // shared memory (rows of 65 floats); the adjoint update then runs with consecutive threads
+            // on consecutive elements.
+            float* st1 = reinterpret_cast<float*>(sm);
+            float* st2 = st1 + 256 * 65;
+            tc_fence_before();
+            __syncthreads();
+            tc_fence_after();
             for (int mt = 0; mt < 2; ++mt) {
                 const int j = 128 * mt + row;
 #pragma unroll 1
                 for (int blk = 0; blk < 2; ++blk) {
                     const int col = 32 * half + 16 * blk;
-                    float x[16];
-                    tmem16(tmem + lane_off + kD * mt + col, x);
+                    float x1[16], x2[16];
+                    tmem16(tmem + lane_off + kD * mt + col, x1);
+                    tmem16(tmem + lane_off + 2 * kD + kD * mt + col, x2);
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {  // W1, S1 row j
-                        const size_t i1 = (size_t)j * kD + col + e;
-                        const float dw = dcur[i1], ds = dcur[2 * kHD + i1];
-                        const float nw = fmaf(An, dw, x[e]), ns = fmaf(sig, dw, En * ds);
-                        pa += dw * X[i1];
-                        ps += dw * X[2 * kHD + i1];
-                        pe += ds * X[2 * kHD + i1];
-                        dnext[i1] = nw;
-                        dnext[2 * kHD + i1] = ns;
-                        dW1b[(size_t)j * 2 * kD + col + e] = __float2bfloat16_rn(nw);
-                        dW1b[(size_t)j * 2 * kD + kD + col + e] = __float2bfloat16_rn(ns);
-                    }
-                    tmem16(tmem + lane_off + 2 * kD + kD * mt + col, x);
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) {  // W2, S2 column j
-                        const size_t i2 = (size_t)(col + e) * kH + j;
-                        const float dw = dcur[kHD + i2], ds = dcur[3 * kHD + i2];
-                        const float nw = fmaf(An, dw, x[e]), ns = fmaf(sig, dw, En * ds);
-                        pa += dw * X[kHD + i2];
-                        ps += dw * X[3 * kHD + i2];
-                        pe += ds * X[3 * kHD + i2];
-                        dnext[kHD + i2] = nw;
-                        dnext[3 * kHD + i2] = ns;
-                        dW2b[i2] = __float2bfloat16_rn(nw);
-                        dW2b[kHD + i2] = __float2bfloat16_rn(ns);
+                    for (int e = 0; e < 16; ++e) {
+                        st1[j * 65 + col + e] = x1[e];
+                        st2[j * 65 + col + e] = x2[e];
                     }
                 }
+            }
+            __syncthreads();
+            float pa = 0.f, ps = 0.f, pe = 0.f;
+            for (size_t i = tid; i < kHD; i += kThreads) {  // W1, S1 [h][d]
+                const size_t j = i / kD, m = i % kD;
+                const float dw = dcur[i], ds = dcur[2 * kHD + i];
+                const float nw = fmaf(An, dw, st1[j * 65 + m]), ns = fmaf(sig, dw, En * ds);
+                pa += dw * X[i];
+                ps += dw * X[2 * kHD + i];
+                pe += ds * X[2 * kHD + i];
+                dnext[i] = nw;
+                dnext[2 * kHD + i] = ns;
+                dW1b[j * 2 * kD + m] = __float2bfloat16_rn(nw);
+                dW1b[j * 2 * kD + kD + m] = __float2bfloat16_rn(ns);
+            }
+            for (size_t i = tid; i < kHD; i += kThreads) {  // W2, S2 [d][h]
+                const size_t r = i / kH, j = i % kH;
+                const float dw = dcur[kHD + i], ds = dcur[3 * kHD + i];
+                const float nw = fmaf(An, dw, st2[j * 65 + r]), ns = fmaf(sig, dw, En * ds);
+                pa += dw * X[kHD + i];
+                ps += dw * X[3 * kHD + i];
+                pe += ds * X[3 * kHD + i];
+                dnext[kHD + i] = nw;
+                dnext[3 * kHD + i] = ns;
+                dW2b[i] = __float2bfloat16_rn(nw);
+                dW2b[kHD + i] = __float2bfloat16_rn(ns);
             }
 #pragma unroll
             for (int off = 16; off > 0; off >>= 1) {
