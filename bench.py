@@ -679,6 +679,35 @@ def deep_arm(args, w, rank, world, local_rank):
         "gpu_launches": args.steps}), flush=True)
 
 
+def backward_arm(args, w, rank, world, local_rank):
+    """--phase backward: one JSON line for titans_mem_backward (every rank runs its own B*H units)."""
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    toks, gates, state = _dev_inputs(w, dev)
+    dy = torch.randn(toks["k"].shape, generator=torch.Generator().manual_seed(5)).to(toks["k"].dtype).to(dev)
+    m = mem.Memory(w.d, w.h, w.chunk, w.dtype, w.B, w.H)
+    fn = lambda: m.backward(toks["k"], toks["q"], toks["v"], gates["alpha"], gates["eta"], gates["theta"], state, dy)
+    total, per = time_launches(fn, torch.cuda.current_stream(dev), args.steps, args.warmup)
+    m.sync_status()
+    ms = max_over_ranks(total / args.steps, dev, world)
+    if rank != 0:
+        return
+    peaks, which = load_peaks()
+    flops = 2 * flops_per_head_token(w) * w.units * w.T
+    achieved = flops / (statistics.mean(per) / 1e3) / 1e12
+    kernel = "mlp_backward_tc_kernel" if m.backward_path() == mem.PATH_TC_BACKWARD else "mlp_backward_kernel"
+    print(json.dumps({
+        "metric": "backward tokens/sec (gradients of every input) per B200; % bf16 tensor-core peak",
+        "value": world * w.B * w.T / (ms / 1e3), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": w.dtype, "data": "synthetic (seeded)",
+        "config": {"workload": f"{w.name} backward", "units": w.units, "T": w.T, "chunk": w.chunk, "kernel": kernel},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": achieved / peaks["bf16_tflops"], "traffic": None, "peak_source": f"bf16_tflops ({which})",
+                     "kernel": kernel, "flops_per_launch": flops, "avg_launch_ms": statistics.mean(per)},
+        "gpu_launches": args.steps}), flush=True)
+
+
 def extra_results(args, dev):
     """The other workloads' numbers, nested in the one JSON line (rank 0 of a 1-GPU run):
     the 2048-unit decode step (HBM-bound), the 16-unit long stream (occupancy-limited: one
@@ -717,9 +746,10 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the nested decode / long-stream / wide-prefill results of a 1-GPU run")
-    ap.add_argument("--phase", choices=["forward", "decode", "deep"], default="forward",
+    ap.add_argument("--phase", choices=["forward", "decode", "deep", "backward"], default="forward",
                     help="forward: the chunk-wise update + retrieve (default); decode: titans_mem_step; "
-                         "deep: the deep memory's chunk-wise forward (--layers) on the tensor-core kernel")
+                         "deep: the deep memory's chunk-wise forward (--layers) on the tensor-core kernel; "
+                         "backward: titans_mem_backward of the 2-layer memory")
     ap.add_argument("--layers", type=int, default=4, help="depth of the deep memory for --phase deep")
     ap.add_argument("--decode-b", type=int, default=0, help="decode batch (default: the workload's, 256)")
     args = ap.parse_args()
@@ -749,6 +779,8 @@ def main():
             decode_arm(args, w, rank, world, local_rank)
         elif args.phase == "deep":
             deep_arm(args, w, rank, world, local_rank)
+        elif args.phase == "backward":
+            backward_arm(args, w, rank, world, local_rank)
         else:
             our_arm(args, w, rank, world, local_rank)
     finally:
