@@ -297,6 +297,7 @@ __global__ void __launch_bounds__(mbt::kThreads, 1) mlp_backward_tc_kernel(const
             }
     };
     auto state_bf16 = [&](const float* X) {
+#pragma unroll 4
         for (size_t i = tid; i < kHD / 4; i += kThreads) {
             const float4 w1 = reinterpret_cast<const float4*>(X)[i];
             const float4 w2 = reinterpret_cast<const float4*>(X + kHD)[i];
@@ -435,20 +436,25 @@ __global__ void __launch_bounds__(mbt::kThreads, 1) mlp_backward_tc_kernel(const
                 }
             }
             __syncthreads();
-            if (part == 0) {
-                for (size_t i = tid; i < kHD; i += kThreads) {  // W1, S1 [h][d]
-                    const size_t j = i / kD, m = i % kD;
-                    const float w = X[i], sv = X[2 * kHD + i];
-                    Xn[i] = fmaf(An, w, sig * sv) - st_c[j * 65 + m];
-                    Xn[2 * kHD + i] = En * sv - st_d[j * 65 + m];
+            // four consecutive elements per thread and step (float4 global accesses)
+            const size_t o = part == 0 ? 0 : kHD;
+#pragma unroll 4
+            for (size_t i = 4 * tid; i < kHD; i += 4 * kThreads) {
+                const float4 w = *reinterpret_cast<const float4*>(X + o + i);
+                const float4 sv = *reinterpret_cast<const float4*>(X + 2 * kHD + o + i);
+                float ac[4], ad[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    // W1, S1 [h][d]: element (j, m) = (i / d, i % d); W2, S2 [d][h]: (r, j) = (i / h, i % h)
+                    const size_t at = part == 0 ? (i / kD) * 65 + (i % kD) + e : ((i % kH) + e) * 65 + i / kH;
+                    ac[e] = st_c[at];
+                    ad[e] = st_d[at];
                 }
-            } else {
-                for (size_t i = tid; i < kHD; i += kThreads) {  // W2, S2 [d][h]
-                    const size_t r = i / kH, j = i % kH;
-                    const float w = X[kHD + i], sv = X[3 * kHD + i];
-                    Xn[kHD + i] = fmaf(An, w, sig * sv) - st_c[j * 65 + r];
-                    Xn[3 * kHD + i] = En * sv - st_d[j * 65 + r];
-                }
+                *reinterpret_cast<float4*>(Xn + o + i) =
+                    make_float4(fmaf(An, w.x, sig * sv.x) - ac[0], fmaf(An, w.y, sig * sv.y) - ac[1],
+                                fmaf(An, w.z, sig * sv.z) - ac[2], fmaf(An, w.w, sig * sv.w) - ac[3]);
+                *reinterpret_cast<float4*>(Xn + 2 * kHD + o + i) =
+                    make_float4(En * sv.x - ad[0], En * sv.y - ad[1], En * sv.z - ad[2], En * sv.w - ad[3]);
             }
         }
         __syncthreads();
@@ -648,29 +654,40 @@ __global__ void __launch_bounds__(mbt::kThreads, 1) mlp_backward_tc_kernel(const
             }
             __syncthreads();
             float pa = 0.f, ps = 0.f, pe = 0.f;
-            for (size_t i = tid; i < kHD; i += kThreads) {  // W1, S1 [h][d]
-                const size_t j = i / kD, m = i % kD;
-                const float dw = dcur[i], ds = dcur[2 * kHD + i];
-                const float nw = fmaf(An, dw, st1[j * 65 + m]), ns = fmaf(sig, dw, En * ds);
-                pa += dw * X[i];
-                ps += dw * X[2 * kHD + i];
-                pe += ds * X[2 * kHD + i];
-                dnext[i] = nw;
-                dnext[2 * kHD + i] = ns;
-                dW1b[j * 2 * kD + m] = __float2bfloat16_rn(nw);
-                dW1b[j * 2 * kD + kD + m] = __float2bfloat16_rn(ns);
-            }
-            for (size_t i = tid; i < kHD; i += kThreads) {  // W2, S2 [d][h]
-                const size_t r = i / kH, j = i % kH;
-                const float dw = dcur[kHD + i], ds = dcur[3 * kHD + i];
-                const float nw = fmaf(An, dw, st2[j * 65 + r]), ns = fmaf(sig, dw, En * ds);
-                pa += dw * X[kHD + i];
-                ps += dw * X[3 * kHD + i];
-                pe += ds * X[3 * kHD + i];
-                dnext[kHD + i] = nw;
-                dnext[3 * kHD + i] = ns;
-                dW2b[i] = __float2bfloat16_rn(nw);
-                dW2b[kHD + i] = __float2bfloat16_rn(ns);
+            // four consecutive elements per thread and step (float4 global accesses)
+            for (int part = 0; part < 2; ++part) {
+                const size_t o = part == 0 ? 0 : kHD;
+                const float* st = part == 0 ? st1 : st2;
+#pragma unroll 4
+                for (size_t i = 4 * tid; i < kHD; i += 4 * kThreads) {
+                    const float4 dw = *reinterpret_cast<const float4*>(dcur + o + i);
+                    const float4 ds = *reinterpret_cast<const float4*>(dcur + 2 * kHD + o + i);
+                    const float4 w = *reinterpret_cast<const float4*>(X + o + i);
+                    const float4 sv = *reinterpret_cast<const float4*>(X + 2 * kHD + o + i);
+                    const float dwv[4] = {dw.x, dw.y, dw.z, dw.w}, dsv[4] = {ds.x, ds.y, ds.z, ds.w};
+                    const float wv[4] = {w.x, w.y, w.z, w.w}, svv[4] = {sv.x, sv.y, sv.z, sv.w};
+                    float nw[4], ns[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const size_t at = part == 0 ? (i / kD) * 65 + (i % kD) + e : ((i % kH) + e) * 65 + i / kH;
+                        nw[e] = fmaf(An, dwv[e], st[at]);
+                        ns[e] = fmaf(sig, dwv[e], En * dsv[e]);
+                        pa += dwv[e] * wv[e];
+                        ps += dwv[e] * svv[e];
+                        pe += dsv[e] * svv[e];
+                    }
+                    *reinterpret_cast<float4*>(dnext + o + i) = make_float4(nw[0], nw[1], nw[2], nw[3]);
+                    *reinterpret_cast<float4*>(dnext + 2 * kHD + o + i) = make_float4(ns[0], ns[1], ns[2], ns[3]);
+                    const uint2 bw = make_uint2(pack2(nw[0], nw[1]), pack2(nw[2], nw[3]));
+                    const uint2 bs = make_uint2(pack2(ns[0], ns[1]), pack2(ns[2], ns[3]));
+                    if (part == 0) {  // [h][dW1' | dS1'], row j = i / d
+                        *reinterpret_cast<uint2*>(dW1b + (i / kD) * 2 * kD + (i % kD)) = bw;
+                        *reinterpret_cast<uint2*>(dW1b + (i / kD) * 2 * kD + kD + (i % kD)) = bs;
+                    } else {          // [dW2'; dS2']
+                        *reinterpret_cast<uint2*>(dW2b + i) = bw;
+                        *reinterpret_cast<uint2*>(dW2b + kHD + i) = bs;
+                    }
+                }
             }
 #pragma unroll
             for (int off = 16; off > 0; off >>= 1) {
