@@ -15,6 +15,8 @@
 //      CTA per (unit, segment)); the last segment hands the final W, S back.
 // fp32 arithmetic on CUDA cores; k, q, v, y in fp32 or bf16.
 #include <cuda_bf16.h>
+
+#include <atomic>
 #include <cstdint>
 
 #include "kernels.h"
@@ -157,6 +159,68 @@ __global__ void __launch_bounds__(kScanThreads) linear_scan_segments(int d, int 
     (void)nseg;
 }
 
+// 2'. The same scan with the state and each segment's map in shared memory (d = 64: the map R_s
+// [3d][2d] and two state buffers [d][2d], 160 KB): every step reads its operands from shared memory
+// instead of L2, and the next segment's map is copied in while nothing else waits on it.
+constexpr int kSegSmemD = 64;
+constexpr size_t kSegSmemBytes = (size_t)(6 * kSegSmemD * kSegSmemD + 4 * kSegSmemD * kSegSmemD) * sizeof(float);
+
+static_assert(kScanThreads == 1024, "the shared-memory segment scan maps 1024 threads onto d x 2d = 64 x 128");
+__global__ void __launch_bounds__(kScanThreads) linear_scan_segments_smem(int chunk, int nseg_used,
+                                                                        const float* __restrict__ W,
+                                                                        const float* __restrict__ S,
+                                                                        float* __restrict__ ws, size_t ws_per_unit) {
+    constexpr int d = kSegSmemD, d2 = 2 * kSegSmemD;
+    extern __shared__ float smf[];
+    float* sR = smf;               // [3d][2d]: M_s rows 0..2d-1, N_s rows 2d..3d-1
+    float* sX0 = sR + 3 * d * d2;  // [d][2d] state buffers
+    float* sX1 = sX0 + d * d2;
+    const long u = blockIdx.x;
+    const size_t slot = slot_floats(d, chunk);
+    float* base = ws + u * ws_per_unit;
+    auto Xof = [&](int s) { return base + (size_t)s * slot + (size_t)6 * d * d + (size_t)3 * d * chunk; };
+    float* X0 = Xof(0);
+    for (int idx = threadIdx.x; idx < d * d2; idx += blockDim.x) {
+        const int i = idx / d2, j = idx % d2;
+        const float x = j < d ? W[u * d * d + (size_t)i * d + j] : S[u * d * d + (size_t)i * d + (j - d)];
+        X0[idx] = x;
+        sX0[idx] = x;
+    }
+    float* cur = sX0;
+    float* nxt = sX1;
+    for (int s = 0; s + 1 < nseg_used; ++s) {
+        __syncthreads();  // the previous step's reads of sR are done
+        const float4* R4 = reinterpret_cast<const float4*>(base + (size_t)s * slot);
+        for (int i = threadIdx.x; i < 3 * d * d2 / 4; i += blockDim.x) reinterpret_cast<float4*>(sR)[i] = R4[i];
+        __syncthreads();
+        float* Xn = Xof(s + 1);
+        // thread: rows i0 and i0 + 32, columns 4 j4 .. 4 j4 + 3 (1024 threads x 8 outputs = d x 2d)
+        const int i0 = threadIdx.x >> 5, j4 = threadIdx.x & 31;
+        float4 a0 = *reinterpret_cast<const float4*>(sR + (d2 + i0) * d2 + 4 * j4);  // N_s rows
+        float4 a1 = *reinterpret_cast<const float4*>(sR + (d2 + i0 + 32) * d2 + 4 * j4);
+#pragma unroll 8
+        for (int r = 0; r < d2; ++r) {
+            const float x0 = cur[i0 * d2 + r], x1 = cur[(i0 + 32) * d2 + r];
+            const float4 m = *reinterpret_cast<const float4*>(sR + r * d2 + 4 * j4);
+            a0.x = fmaf(x0, m.x, a0.x);
+            a0.y = fmaf(x0, m.y, a0.y);
+            a0.z = fmaf(x0, m.z, a0.z);
+            a0.w = fmaf(x0, m.w, a0.w);
+            a1.x = fmaf(x1, m.x, a1.x);
+            a1.y = fmaf(x1, m.y, a1.y);
+            a1.z = fmaf(x1, m.z, a1.z);
+            a1.w = fmaf(x1, m.w, a1.w);
+        }
+        *reinterpret_cast<float4*>(nxt + i0 * d2 + 4 * j4) = a0;
+        *reinterpret_cast<float4*>(nxt + (i0 + 32) * d2 + 4 * j4) = a1;
+        *reinterpret_cast<float4*>(Xn + i0 * d2 + 4 * j4) = a0;
+        *reinterpret_cast<float4*>(Xn + (i0 + 32) * d2 + 4 * j4) = a1;
+        float* t = cur;
+        cur = nxt;
+        nxt = t;
+    }
+}
+
 // 3. run segment s of unit u from X_s: y for its tokens; the last segment writes the final W, S.
 template <typename Tin>
 __global__ void __launch_bounds__(kScanThreads) linear_scan_run(
@@ -240,8 +304,24 @@ static cudaError_t launch_scan(const ForwardArgs& a, int nseg_max, cudaStream_t 
                                                             a.theta, a.ws, a.ws_per_unit);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    linear_scan_segments<<<(unsigned)a.units, kScanThreads, 0, st>>>(a.d, a.chunk, used, used, a.W1, a.S1, a.ws,
-                                                                     a.ws_per_unit);
+    if (a.d == kSegSmemD) {
+        static std::atomic<unsigned> attr_set{0};  // per device: set before the first launch there
+        int dev = 0;
+        e = cudaGetDevice(&dev);
+        if (e != cudaSuccess) return e;
+        if (dev < 0 || dev >= 32) return cudaErrorInvalidDevice;
+        if (!(attr_set.load() & (1u << dev))) {
+            e = cudaFuncSetAttribute(linear_scan_segments_smem, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)kSegSmemBytes);
+            if (e != cudaSuccess) return e;
+            attr_set.fetch_or(1u << dev);
+        }
+        linear_scan_segments_smem<<<(unsigned)a.units, kScanThreads, kSegSmemBytes, st>>>(a.chunk, used, a.W1, a.S1,
+                                                                                           a.ws, a.ws_per_unit);
+    } else {
+        linear_scan_segments<<<(unsigned)a.units, kScanThreads, 0, st>>>(a.d, a.chunk, used, used, a.W1, a.S1, a.ws,
+                                                                         a.ws_per_unit);
+    }
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     linear_scan_run<Tin><<<grid, kScanThreads, 0, st>>>(a.d, a.T, a.gate_ld, a.chunk, (int)a.chunk_gates, used, G,
