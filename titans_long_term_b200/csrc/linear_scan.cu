@@ -128,6 +128,81 @@ __global__ void __launch_bounds__(kScanThreads) linear_scan_compose(
     }
 }
 
+// 1'. The same composition with the map, the chunk's keys and the products in shared memory (d = 64):
+// R [3d][2d], P [3d][n], the keys [n][d + 1] (one padding column so that a warp reading one column
+// of 16 or more key rows does not hit one bank), 96 KB + about 1 KB per token of the chunk.
+constexpr int kComposeSmemMaxChunk = 64;  // chunks up to 64 tokens: 160 KB of shared memory at most
+__host__ __device__ inline size_t compose_smem_bytes(int chunk) {
+    constexpr int d = 64;
+    return ((size_t)6 * d * d + (size_t)3 * d * chunk + (size_t)chunk * (d + 1)) * sizeof(float);
+}
+
+template <typename Tin>
+__global__ void __launch_bounds__(kScanThreads) linear_scan_compose_smem(
+    long T, long gate_ld, int chunk, int chunk_gates, int nseg, int G, const Tin* __restrict__ k,
+    const Tin* __restrict__ v, const float* __restrict__ alpha, const float* __restrict__ eta,
+    const float* __restrict__ theta, float* __restrict__ ws, size_t ws_per_unit) {
+    constexpr int d = 64, d2 = 128, rows = 192;
+    __shared__ float s_a[kScanMaxChunk], s_e[kScanMaxChunk], s_t[kScanMaxChunk], s_c[kScanMaxChunk],
+        s_d[kScanMaxChunk], s_scal[3];
+    extern __shared__ float smf[];
+    float* sR = smf;                         // [3d][2d]
+    float* sP = sR + rows * d2;              // [3d][n]
+    float* sK = sP + (size_t)rows * chunk;   // [n][d + 1]
+    const long u = blockIdx.x / nseg;
+    const int s = blockIdx.x % nseg, tid = threadIdx.x;
+    float* R = ws + u * ws_per_unit + (size_t)s * slot_floats(d, chunk);
+    for (int idx = tid; idx < rows * d2; idx += blockDim.x) {
+        const int r = idx / d2, col = idx % d2;
+        sR[idx] = (r < d2 && col == r) ? 1.f : 0.f;
+    }
+    k += u * T * d;
+    v += u * T * d;
+    alpha += u * gate_ld;
+    eta += u * gate_ld;
+    theta += u * gate_ld;
+    const int nch = (int)((T + chunk - 1) / chunk);
+    const int c1 = min(nch, (s + 1) * G);
+    for (int c = s * G; c < c1; ++c) {
+        const long t0 = (long)c * chunk;
+        const int n = (int)min((long)chunk, T - t0);
+        chunk_scan(alpha, eta, theta, t0, n, chunk, chunk_gates, s_a, s_e, s_t, s_c, s_d, s_scal);
+        const float An = s_scal[0], En = s_scal[1], sig = s_scal[2];
+        const Tin* K = k + t0 * d;
+        const Tin* V = v + t0 * d;
+        for (int idx = tid; idx < n * d; idx += blockDim.x) sK[(idx / d) * (d + 1) + idx % d] = ldx(K + idx);
+        __syncthreads();
+        // P[r][t] = (row r of the W part) . k_t  - (v_t's component for the N rows)
+        for (int idx = tid; idx < rows * n; idx += blockDim.x) {
+            const int r = idx / n, t = idx % n;
+            float p = 0.f;
+            const float* Rr = sR + r * d2;
+            const float* Kt = sK + t * (d + 1);
+#pragma unroll 8
+            for (int m = 0; m < d; ++m) p = fmaf(Rr[m], Kt[m], p);
+            if (r >= d2) p -= ldx(V + (size_t)t * d + (r - d2));
+            sP[r * n + t] = p;
+        }
+        __syncthreads();
+        for (int idx = tid; idx < rows * d; idx += blockDim.x) {
+            const int r = idx / d, m = idx % d;
+            float uc = 0.f, ud = 0.f;
+            for (int t = 0; t < n; ++t) {
+                const float g = sP[r * n + t] * sK[t * (d + 1) + m];
+                uc = fmaf(s_c[t], g, uc);
+                ud = fmaf(s_d[t], g, ud);
+            }
+            float* Rr = sR + r * d2;
+            const float w = Rr[m], sv = Rr[d + m];
+            Rr[m] = An * w + sig * sv - 2.f * uc;
+            Rr[d + m] = En * sv - 2.f * ud;
+        }
+        __syncthreads();
+    }
+    for (int i = tid; i < rows * d2 / 4; i += blockDim.x)
+        reinterpret_cast<float4*>(R)[i] = reinterpret_cast<const float4*>(sR)[i];
+}
+
 // 2. per unit: X_0 = [W | S], X_{s+1} = X_s M_s + N_s (M_s = R_s rows 0..2d-1, N_s = rows 2d..3d-1).
 __global__ void __launch_bounds__(kScanThreads) linear_scan_segments(int d, int chunk, int nseg_used, int nseg,
                                                                    const float* __restrict__ W,
@@ -291,6 +366,97 @@ __global__ void __launch_bounds__(kScanThreads) linear_scan_run(
     }
 }
 
+// 3'. The same run with the state, the chunk's keys and queries and G in shared memory (d = 64,
+// chunks up to 64 tokens): X [d][2d], K and Q [n][d + 1] (one padding column), G [d][n].
+__host__ __device__ inline size_t run_smem_bytes(int chunk) {
+    constexpr int d = 64;
+    return ((size_t)2 * d * d + (size_t)2 * chunk * (d + 1) + (size_t)chunk * d) * sizeof(float);
+}
+
+template <typename Tin>
+__global__ void __launch_bounds__(kScanThreads) linear_scan_run_smem(
+    long T, long gate_ld, int chunk, int chunk_gates, int nseg_used, int G, const Tin* __restrict__ k,
+    const Tin* __restrict__ q, const Tin* __restrict__ v, const float* __restrict__ alpha,
+    const float* __restrict__ eta, const float* __restrict__ theta, float* __restrict__ Wout,
+    float* __restrict__ Sout, Tin* __restrict__ y, const Tin* __restrict__ attn, float* __restrict__ ws,
+    size_t ws_per_unit) {
+    constexpr int d = 64, d2 = 128;
+    __shared__ float s_a[kScanMaxChunk], s_e[kScanMaxChunk], s_t[kScanMaxChunk], s_c[kScanMaxChunk],
+        s_d[kScanMaxChunk], s_scal[3];
+    extern __shared__ float smf[];
+    float* sX = smf;                          // [d][2d]: W | S
+    float* sK = sX + d * d2;                  // [n][d + 1]
+    float* sQ = sK + (size_t)chunk * (d + 1);
+    float* sG = sQ + (size_t)chunk * (d + 1);  // [d][n]
+    const long u = blockIdx.x / nseg_used;
+    const int s = blockIdx.x % nseg_used, tid = threadIdx.x;
+    const float* X0 = ws + u * ws_per_unit + (size_t)s * slot_floats(d, chunk) + (size_t)6 * d * d +
+                      (size_t)3 * d * chunk;
+    for (int i = tid; i < d * d2 / 4; i += blockDim.x)
+        reinterpret_cast<float4*>(sX)[i] = reinterpret_cast<const float4*>(X0)[i];
+    k += u * T * d;
+    q += u * T * d;
+    v += u * T * d;
+    y += u * T * d;
+    if (attn) attn += u * T * d;
+    alpha += u * gate_ld;
+    eta += u * gate_ld;
+    theta += u * gate_ld;
+    const int nch = (int)((T + chunk - 1) / chunk);
+    const int c1 = min(nch, (s + 1) * G);
+    for (int c = s * G; c < c1; ++c) {
+        const long t0 = (long)c * chunk;
+        const int n = (int)min((long)chunk, T - t0);
+        chunk_scan(alpha, eta, theta, t0, n, chunk, chunk_gates, s_a, s_e, s_t, s_c, s_d, s_scal);
+        const float An = s_scal[0], En = s_scal[1], sig = s_scal[2];
+        for (int idx = tid; idx < n * d; idx += blockDim.x) {
+            const int t = idx / d, m = idx % d;
+            sK[t * (d + 1) + m] = ldx(k + t0 * d + idx);
+            sQ[t * (d + 1) + m] = ldx(q + t0 * d + idx);
+        }
+        __syncthreads();
+        // G = 2 (W k - v), y = W q; the lanes of a warp take consecutive tokens of one output row i,
+        // so the row of W is a broadcast and the key rows (padded) hit distinct banks. G is [d][n].
+        for (int idx = tid; idx < n * d; idx += blockDim.x) {
+            const int i = idx / n, t = idx % n;
+            float yh = 0.f, yq = 0.f;
+            const float* Wr = sX + i * d2;
+            const float* Kt = sK + t * (d + 1);
+            const float* Qt = sQ + t * (d + 1);
+#pragma unroll 8
+            for (int m = 0; m < d; ++m) {
+                yh = fmaf(Wr[m], Kt[m], yh);
+                yq = fmaf(Wr[m], Qt[m], yq);
+            }
+            const long o = (t0 + t) * d + i;
+            sG[i * n + t] = 2.f * (yh - ldx(v + o));
+            stx(y + o, attn ? ldx(attn + o) / (1.f + expf(-yq)) : yq);
+        }
+        __syncthreads();
+        for (int idx = tid; idx < d * d; idx += blockDim.x) {
+            const int i = idx / d, m = idx % d;
+            float uc = 0.f, ud = 0.f;
+            for (int t = 0; t < n; ++t) {
+                const float g = sG[i * n + t] * sK[t * (d + 1) + m];
+                uc = fmaf(s_c[t], g, uc);
+                ud = fmaf(s_d[t], g, ud);
+            }
+            float* Wr = sX + i * d2;
+            const float w = Wr[m], sv = Wr[d + m];
+            Wr[m] = An * w + sig * sv - uc;
+            Wr[d + m] = En * sv - ud;
+        }
+        __syncthreads();
+    }
+    if (s == nseg_used - 1) {
+        for (int idx = tid; idx < d * d; idx += blockDim.x) {
+            const int i = idx / d, m = idx % d;
+            Wout[u * d * d + idx] = sX[i * d2 + m];
+            Sout[u * d * d + idx] = sX[i * d2 + d + m];
+        }
+    }
+}
+
 template <typename Tin>
 static cudaError_t launch_scan(const ForwardArgs& a, int nseg_max, cudaStream_t st) {
     const int nch = (int)((a.T + a.chunk - 1) / a.chunk);
@@ -299,10 +465,28 @@ static cudaError_t launch_scan(const ForwardArgs& a, int nseg_max, cudaStream_t 
     const int G = (nch + nseg - 1) / nseg;
     const int used = (nch + G - 1) / G;  // segments that hold chunks
     const unsigned grid = (unsigned)(a.units * used);
-    linear_scan_compose<Tin><<<grid, kScanThreads, 0, st>>>(a.d, a.T, a.gate_ld, a.chunk, (int)a.chunk_gates, used, G,
-                                                            (const Tin*)a.k, (const Tin*)a.v, a.alpha, a.eta,
-                                                            a.theta, a.ws, a.ws_per_unit);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = cudaSuccess;
+    if (a.d == kSegSmemD && a.chunk <= kComposeSmemMaxChunk) {
+        static std::atomic<unsigned> attr_set{0};  // per device: set before the first launch there
+        int dev = 0;
+        e = cudaGetDevice(&dev);
+        if (e != cudaSuccess) return e;
+        if (dev < 0 || dev >= 32) return cudaErrorInvalidDevice;
+        if (!(attr_set.load() & (1u << dev))) {
+            e = cudaFuncSetAttribute(linear_scan_compose_smem<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)compose_smem_bytes(kComposeSmemMaxChunk));
+            if (e != cudaSuccess) return e;
+            attr_set.fetch_or(1u << dev);
+        }
+        linear_scan_compose_smem<Tin><<<grid, kScanThreads, compose_smem_bytes(a.chunk), st>>>(
+            a.T, a.gate_ld, a.chunk, (int)a.chunk_gates, used, G, (const Tin*)a.k, (const Tin*)a.v, a.alpha, a.eta,
+            a.theta, a.ws, a.ws_per_unit);
+    } else {
+        linear_scan_compose<Tin><<<grid, kScanThreads, 0, st>>>(a.d, a.T, a.gate_ld, a.chunk, (int)a.chunk_gates,
+                                                                used, G, (const Tin*)a.k, (const Tin*)a.v, a.alpha,
+                                                                a.eta, a.theta, a.ws, a.ws_per_unit);
+    }
+    e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     if (a.d == kSegSmemD) {
         static std::atomic<unsigned> attr_set{0};  // per device: set before the first launch there
@@ -324,10 +508,27 @@ static cudaError_t launch_scan(const ForwardArgs& a, int nseg_max, cudaStream_t 
     }
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    linear_scan_run<Tin><<<grid, kScanThreads, 0, st>>>(a.d, a.T, a.gate_ld, a.chunk, (int)a.chunk_gates, used, G,
-                                                        (const Tin*)a.k, (const Tin*)a.q, (const Tin*)a.v, a.alpha,
-                                                        a.eta, a.theta, a.W1, a.S1, (Tin*)a.y, (const Tin*)a.attn,
-                                                        a.ws, a.ws_per_unit);
+    if (a.d == kSegSmemD && a.chunk <= kComposeSmemMaxChunk) {
+        static std::atomic<unsigned> attr_set{0};  // per device: set before the first launch there
+        int dev = 0;
+        e = cudaGetDevice(&dev);
+        if (e != cudaSuccess) return e;
+        if (dev < 0 || dev >= 32) return cudaErrorInvalidDevice;
+        if (!(attr_set.load() & (1u << dev))) {
+            e = cudaFuncSetAttribute(linear_scan_run_smem<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)run_smem_bytes(kComposeSmemMaxChunk));
+            if (e != cudaSuccess) return e;
+            attr_set.fetch_or(1u << dev);
+        }
+        linear_scan_run_smem<Tin><<<grid, kScanThreads, run_smem_bytes(a.chunk), st>>>(
+            a.T, a.gate_ld, a.chunk, (int)a.chunk_gates, used, G, (const Tin*)a.k, (const Tin*)a.q, (const Tin*)a.v,
+            a.alpha, a.eta, a.theta, a.W1, a.S1, (Tin*)a.y, (const Tin*)a.attn, a.ws, a.ws_per_unit);
+    } else {
+        linear_scan_run<Tin><<<grid, kScanThreads, 0, st>>>(a.d, a.T, a.gate_ld, a.chunk, (int)a.chunk_gates, used,
+                                                            G, (const Tin*)a.k, (const Tin*)a.q, (const Tin*)a.v,
+                                                            a.alpha, a.eta, a.theta, a.W1, a.S1, (Tin*)a.y,
+                                                            (const Tin*)a.attn, a.ws, a.ws_per_unit);
+    }
     return cudaGetLastError();
 }
 
