@@ -33,8 +33,12 @@ __device__ __forceinline__ void stx(__nv_bfloat16* p, float v) { *p = __float2bf
 constexpr int kScanThreads = 1024;
 constexpr int kScanMaxChunk = 128;
 
-// Per (unit, segment) workspace slot, in floats: R [3d][2d], P [3d][n], X [d][2d], G [n][d].
+// Per (unit, segment) workspace slot, in floats: R [3d][2d], P [3d][n], X [d][2d], G [n][d], and a
+// second map buffer R2 [3d][2d] for the tree scan over segments.
 __host__ __device__ inline size_t slot_floats(int d, int n) {
+    return (size_t)6 * d * d + (size_t)3 * d * n + (size_t)2 * d * d + (size_t)n * d + (size_t)6 * d * d;
+}
+__host__ __device__ inline size_t slot_r2(int d, int n) {
     return (size_t)6 * d * d + (size_t)3 * d * n + (size_t)2 * d * d + (size_t)n * d;
 }
 
@@ -238,6 +242,7 @@ __global__ void __launch_bounds__(kScanThreads) linear_scan_segments(int d, int 
 // [3d][2d] and two state buffers [d][2d], 160 KB): every step reads its operands from shared memory
 // instead of L2, and the next segment's map is copied in while nothing else waits on it.
 constexpr int kSegSmemD = 64;
+constexpr int kTreeMinSegments = 16;  // below this the sequential scan (one CTA per unit) is as fast
 constexpr size_t kSegSmemBytes = (size_t)(6 * kSegSmemD * kSegSmemD + 4 * kSegSmemD * kSegSmemD) * sizeof(float);
 
 static_assert(kScanThreads == 1024, "the shared-memory segment scan maps 1024 threads onto d x 2d = 64 x 128");
@@ -294,6 +299,106 @@ __global__ void __launch_bounds__(kScanThreads) linear_scan_segments_smem(int ch
         cur = nxt;
         nxt = t;
     }
+}
+
+// 2''. The scan over segments as a tree (d = 64): Hillis-Steele levels, each composing every map
+// with the one 2^level segments before it, so that after ceil(log2 S) levels map s is
+// F_s o ... o F_0; then X_{s+1} = X_0 M + N for every segment at once. Composition, X -> (X M_a +
+// N_a) M_b + N_b: R_out = R_a M_b + [0; N_b] with R = [M; N] ([3d][2d]); one CTA per (unit,
+// segment), both maps in shared memory (160 KB), 6 x 4 outputs per thread.
+constexpr size_t kTreeSmemBytes = (size_t)(6 * 64 * 64 + 4 * 64 * 64) * sizeof(float);
+
+__global__ void __launch_bounds__(kScanThreads) linear_scan_tree_level(int chunk, int nseg_used, int step, int src2,
+                                                                     float* __restrict__ ws, size_t ws_per_unit) {
+    constexpr int d = 64, d2 = 128, rows = 192;
+    extern __shared__ float smf[];
+    float* sA = smf;              // R_a [3d][2d]
+    float* sM = sA + rows * d2;   // M_b [2d][2d]
+    const long u = blockIdx.x / nseg_used;
+    const int s = blockIdx.x % nseg_used, tid = threadIdx.x;
+    const size_t slot = slot_floats(d, chunk), r2 = slot_r2(d, chunk);
+    float* base = ws + u * ws_per_unit;
+    auto map_in = [&](int seg) { return base + (size_t)seg * slot + (src2 ? r2 : 0); };
+    float* out = base + (size_t)s * slot + (src2 ? 0 : r2);
+    const float* Rb = map_in(s);
+    if (s < step) {  // nothing 2^level segments back: the map carries over
+        for (int i = tid; i < rows * d2 / 4; i += blockDim.x)
+            reinterpret_cast<float4*>(out)[i] = reinterpret_cast<const float4*>(Rb)[i];
+        return;
+    }
+    const float* Ra = map_in(s - step);
+    for (int i = tid; i < rows * d2 / 4; i += blockDim.x)
+        reinterpret_cast<float4*>(sA)[i] = reinterpret_cast<const float4*>(Ra)[i];
+    for (int i = tid; i < d2 * d2 / 4; i += blockDim.x)
+        reinterpret_cast<float4*>(sM)[i] = reinterpret_cast<const float4*>(Rb)[i];
+    __syncthreads();
+    const int i0 = tid >> 5, j4 = tid & 31;  // rows i0 + 32 q (q < 6), columns 4 j4 .. 4 j4 + 3
+    float4 acc[6];
+#pragma unroll
+    for (int qr = 0; qr < 6; ++qr) {
+        const int r = i0 + 32 * qr;  // N_b joins the N rows (r >= 2d)
+        acc[qr] = r >= d2 ? *reinterpret_cast<const float4*>(Rb + (size_t)r * d2 + 4 * j4) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll 4
+    for (int k = 0; k < d2; ++k) {
+        const float4 m = *reinterpret_cast<const float4*>(sM + k * d2 + 4 * j4);
+#pragma unroll
+        for (int qr = 0; qr < 6; ++qr) {
+            const float a = sA[(i0 + 32 * qr) * d2 + k];
+            acc[qr].x = fmaf(a, m.x, acc[qr].x);
+            acc[qr].y = fmaf(a, m.y, acc[qr].y);
+            acc[qr].z = fmaf(a, m.z, acc[qr].z);
+            acc[qr].w = fmaf(a, m.w, acc[qr].w);
+        }
+    }
+#pragma unroll
+    for (int qr = 0; qr < 6; ++qr) *reinterpret_cast<float4*>(out + (size_t)(i0 + 32 * qr) * d2 + 4 * j4) = acc[qr];
+}
+
+// X_0 = [W | S] into slot 0; X_{s+1} = X_0 M + N with the composed map s, for s < S - 1.
+__global__ void __launch_bounds__(kScanThreads) linear_scan_tree_apply(int chunk, int nseg_used, int src2,
+                                                                     const float* __restrict__ W,
+                                                                     const float* __restrict__ S,
+                                                                     float* __restrict__ ws, size_t ws_per_unit) {
+    constexpr int d = 64, d2 = 128;
+    extern __shared__ float smf[];
+    float* sX = smf;             // X_0 [d][2d]
+    float* sM = sX + d * d2;     // M [2d][2d]
+    const long u = blockIdx.x / nseg_used;
+    const int s = blockIdx.x % nseg_used, tid = threadIdx.x;
+    const size_t slot = slot_floats(d, chunk);
+    float* base = ws + u * ws_per_unit;
+    auto Xof = [&](int seg) { return base + (size_t)seg * slot + (size_t)6 * d * d + (size_t)3 * d * chunk; };
+    for (int idx = tid; idx < d * d2; idx += blockDim.x) {
+        const int i = idx / d2, j = idx % d2;
+        sX[idx] = j < d ? W[u * d * d + (size_t)i * d + j] : S[u * d * d + (size_t)i * d + (j - d)];
+    }
+    if (s == 0)
+        for (int idx = tid; idx < d * d2; idx += blockDim.x) Xof(0)[idx] = sX[idx];
+    if (s + 1 >= nseg_used) return;
+    const float* R = base + (size_t)s * slot + (src2 ? slot_r2(d, chunk) : 0);
+    for (int i = tid; i < d2 * d2 / 4; i += blockDim.x)
+        reinterpret_cast<float4*>(sM)[i] = reinterpret_cast<const float4*>(R)[i];
+    __syncthreads();
+    const int i0 = tid >> 5, j4 = tid & 31;
+    float4 a0 = *reinterpret_cast<const float4*>(R + (size_t)(d2 + i0) * d2 + 4 * j4);
+    float4 a1 = *reinterpret_cast<const float4*>(R + (size_t)(d2 + i0 + 32) * d2 + 4 * j4);
+#pragma unroll 8
+    for (int r = 0; r < d2; ++r) {
+        const float x0 = sX[i0 * d2 + r], x1 = sX[(i0 + 32) * d2 + r];
+        const float4 m = *reinterpret_cast<const float4*>(sM + r * d2 + 4 * j4);
+        a0.x = fmaf(x0, m.x, a0.x);
+        a0.y = fmaf(x0, m.y, a0.y);
+        a0.z = fmaf(x0, m.z, a0.z);
+        a0.w = fmaf(x0, m.w, a0.w);
+        a1.x = fmaf(x1, m.x, a1.x);
+        a1.y = fmaf(x1, m.y, a1.y);
+        a1.z = fmaf(x1, m.z, a1.z);
+        a1.w = fmaf(x1, m.w, a1.w);
+    }
+    float* Xn = Xof(s + 1);
+    *reinterpret_cast<float4*>(Xn + i0 * d2 + 4 * j4) = a0;
+    *reinterpret_cast<float4*>(Xn + (i0 + 32) * d2 + 4 * j4) = a1;
 }
 
 // 3. run segment s of unit u from X_s: y for its tokens; the last segment writes the final W, S.
@@ -497,11 +602,32 @@ static cudaError_t launch_scan(const ForwardArgs& a, int nseg_max, cudaStream_t 
         if (!(attr_set.load() & (1u << dev))) {
             e = cudaFuncSetAttribute(linear_scan_segments_smem, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      (int)kSegSmemBytes);
+            if (e == cudaSuccess)
+                e = cudaFuncSetAttribute(linear_scan_tree_level, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kTreeSmemBytes);
+            if (e == cudaSuccess)
+                e = cudaFuncSetAttribute(linear_scan_tree_apply, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kTreeSmemBytes);
             if (e != cudaSuccess) return e;
             attr_set.fetch_or(1u << dev);
         }
-        linear_scan_segments_smem<<<(unsigned)a.units, kScanThreads, kSegSmemBytes, st>>>(a.chunk, used, a.W1, a.S1,
-                                                                                           a.ws, a.ws_per_unit);
+        if (used >= kTreeMinSegments) {
+            // tree over the segments: ceil(log2 used) composition levels, then every start state at once
+            int src2 = 0;
+            for (int step = 1; step < used; step <<= 1) {
+                linear_scan_tree_level<<<grid, kScanThreads, kTreeSmemBytes, st>>>(a.chunk, used, step, src2, a.ws,
+                                                                                   a.ws_per_unit);
+                e = cudaGetLastError();
+                if (e != cudaSuccess) return e;
+                src2 ^= 1;
+            }
+            linear_scan_tree_apply<<<grid, kScanThreads, kTreeSmemBytes, st>>>(a.chunk, used, src2, a.W1, a.S1, a.ws,
+                                                                               a.ws_per_unit);
+        } else {
+            linear_scan_segments_smem<<<(unsigned)a.units, kScanThreads, kSegSmemBytes, st>>>(a.chunk, used, a.W1,
+                                                                                               a.S1, a.ws,
+                                                                                               a.ws_per_unit);
+        }
     } else {
         linear_scan_segments<<<(unsigned)a.units, kScanThreads, 0, st>>>(a.d, a.chunk, used, used, a.W1, a.S1, a.ws,
                                                                          a.ws_per_unit);
