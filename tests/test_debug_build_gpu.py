@@ -1,5 +1,5 @@
 """The bounds-checked build (libtitans_mem_debug.so, compiled with -DTITANS_DEBUG) passes the
-tensor-core parity suites (the deep memory's included) with a clean status word: none of its checks on TMA coordinates, gate and
+tensor-core parity suites (the deep memory's and the backward's included) with a clean status word: none of its checks on TMA coordinates, gate and
 token indices, shared-memory and TMEM offsets fires on any parity case, and its results still match
 the oracle. The suites run in a child process with TITANS_DEBUG=1, which makes the binding load the
 debug library; the child also confirms from its own memory map that this library is the one loaded."""
@@ -15,7 +15,8 @@ pytestmark = pytest.mark.gpu
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 SUITES = ["tests/test_parity_gpu.py", "tests/test_phased_gpu.py", "tests/test_chunk_gates_gpu.py",
-          "tests/test_gated_gpu.py", "tests/test_stated_inputs_gpu.py", "tests/test_deep_gpu.py"]
+          "tests/test_gated_gpu.py", "tests/test_stated_inputs_gpu.py", "tests/test_deep_gpu.py",
+          "tests/test_backward_gpu.py"]
 
 CHILD = r"""
 import sys, pytest

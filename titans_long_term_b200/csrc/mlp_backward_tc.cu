@@ -167,6 +167,7 @@ __global__ void __launch_bounds__(mbt::kThreads, 1) mlp_backward_tc_kernel(const
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sm + TPTR);
     uint32_t mma_phase = 0;
     bool ok = true;
+#define DBG(cond) TITANS_DBG(cond, a.status, static_cast<volatile int*>(nullptr))
 
     const long u = blockIdx.x, T = a.T;
     const int chunk = a.chunk;
@@ -399,6 +400,7 @@ __global__ void __launch_bounds__(mbt::kThreads, 1) mlp_backward_tc_kernel(const
         const int n = (int)min((long)chunk, T - t0);
         const float* X = ckpt + (size_t)c * 4 * kHD;
         float* Xn = ckpt + (size_t)(c + 1) * 4 * kHD;
+        if (!DBG(n >= 1 && n <= kN)) break;  // the same verdict in every thread
         scan(t0, n);
         load_chunk(t0, n, false);
         state_bf16(X);
@@ -480,6 +482,7 @@ __global__ void __launch_bounds__(mbt::kThreads, 1) mlp_backward_tc_kernel(const
         const long t0 = c * chunk;
         const int n = (int)min((long)chunk, T - t0);
         const float* X = ckpt + (size_t)c * 4 * kHD;
+        if (!DBG(n >= 1 && n <= kN)) break;
         scan(t0, n);
         load_chunk(t0, n, true);
         state_bf16(X);
@@ -563,7 +566,7 @@ __global__ void __launch_bounds__(mbt::kThreads, 1) mlp_backward_tc_kernel(const
                     ov[e] = -2.f * g;
                 }
                 st16_bf16(GQ + (size_t)(128 + t) * kD + col, o);
-                if (t < n) st16_bf16(dv + (t0 + t) * kD + col, ov);
+                if (t < n && DBG(t0 + t < T)) st16_bf16(dv + (t0 + t) * kD + col, ov);
             }
         }
         // dA = dA0 + dyhat W2;  dz = dz0 + dA * silu'(Z)
@@ -607,8 +610,8 @@ __global__ void __launch_bounds__(mbt::kThreads, 1) mlp_backward_tc_kernel(const
                         pc -= km[e] * x0[e];
                         pd -= km[e] * x1[e];
                     }
-                    if (t < n) st16_bf16(dk + (t0 + t) * kD + col, o);
-                } else if (t < n) {
+                    if (t < n && DBG(t0 + t < T)) st16_bf16(dk + (t0 + t) * kD + col, o);
+                } else if (t < n && DBG(t0 + t < T)) {
                     st16_bf16(dq + (t0 + t) * kD + col, x2);
                 }
             }
@@ -738,6 +741,8 @@ __global__ void __launch_bounds__(mbt::kThreads, 1) mlp_backward_tc_kernel(const
         tmem_dealloc(tmem, kTmemCols);
     }
 }
+
+#undef DBG
 
 bool mlp_backward_tc_supported(int d, int h, int chunk) {
     return d == mbt::kD && h == mbt::kH && chunk >= 1 && chunk <= mbt::kN;
