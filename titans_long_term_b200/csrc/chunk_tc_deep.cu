@@ -273,7 +273,7 @@ __global__ void __launch_bounds__(dp::kThreads, 1) chunk_fwd_tc_deep(const __gri
     for (int c = 0; c < nchunks && ok; ++c) {
         const long t0 = (long)c * a.chunk;
         const int n = (int)min((long)a.chunk, T - t0);
-        if (!DBG(n >= 1 && n <= kNmax)) break;  // the same verdict in every CTA
+        if (!DBG(n >= 1 && n <= kNmax)) break;  // the same outcome in every CTA
 
         // ================= forward layers (F_1 also runs the gate scan of every unit)
         for (int l = 1; l < L && ok; ++l) {

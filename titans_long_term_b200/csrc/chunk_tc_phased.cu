@@ -69,7 +69,7 @@ constexpr uint32_t kP3Dt = 0, kP3Sp = 64 * 1024;    // Delta^T [128][256 B]; sil
 constexpr uint32_t kP4Wb = 0;                       // bf16 weight rows [128][256 B]
 constexpr uint32_t BAR = kSmemOperands;       // one mbarrier (MMA completion)
 constexpr uint32_t TPTR = BAR + 8;
-constexpr uint32_t OKF = TPTR + 4;            // the grid barrier's verdict for the CTA
+constexpr uint32_t OKF = TPTR + 4;            // the grid barrier's outcome for the CTA
 constexpr uint32_t END = OKF + 4;
 constexpr size_t kSmemBytes = END + 1024;
 constexpr uint32_t kTmemCols = 256;
@@ -138,7 +138,7 @@ __global__ void __launch_bounds__(ph::kThreads, 1) chunk_fwd_tc_phased(const __g
     bool ok = true;
 
     // Issue on one thread, wait on all: the tile's MMAs are complete and TMEM is readable. The
-    // verdict is the same for every thread of the CTA (a timeout anywhere counts for all).
+    // outcome is the same for every thread of the CTA (a timeout anywhere counts for all).
     auto mma_done = [&]() -> bool {
         if (tid == 0) umma_commit(bar);
         const bool done = mbar_wait(bar, mma_phase);
@@ -177,7 +177,7 @@ __global__ void __launch_bounds__(ph::kThreads, 1) chunk_fwd_tc_phased(const __g
     for (int c = 0; c < nchunks && ok; ++c) {
         const long t0 = (long)c * a.chunk;
         const int n = (int)min((long)a.chunk, T - t0);
-        if (!DBG(n >= 1 && n <= kNmax)) break;  // the same verdict in every CTA
+        if (!DBG(n >= 1 && n <= kNmax)) break;  // the same outcome in every CTA
 
         // ================= P1: Z^T tiles (unit, 128 hidden rows, keys | queries) and gate scans
         const int p1_gemm = units * 8;

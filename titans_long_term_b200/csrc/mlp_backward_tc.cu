@@ -400,7 +400,7 @@ __global__ void __launch_bounds__(mbt::kThreads, 1) mlp_backward_tc_kernel(const
         const int n = (int)min((long)chunk, T - t0);
         const float* X = ckpt + (size_t)c * 4 * kHD;
         float* Xn = ckpt + (size_t)(c + 1) * 4 * kHD;
-        if (!DBG(n >= 1 && n <= kN)) break;  // the same verdict in every thread
+        if (!DBG(n >= 1 && n <= kN)) break;  // the same outcome in every thread
         scan(t0, n);
         load_chunk(t0, n, false);
         state_bf16(X);
