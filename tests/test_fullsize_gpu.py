@@ -9,7 +9,9 @@ minutes per unit, and the oracle's chunk closed form (pinned to the token loop a
 small shapes) stands in. The wide memory (128-512-128) is compared
 on the whole prefill and on sampled decode units over 1024 steps that start from the
 oracle's own prefill state. fp32 reference mode is held to 1e-4 on the prefixes the
-library claims it for.
+library claims it for. The deep memory (4 layers) and the backward run the 760M-class shape in
+the launch configurations `bench.py --phase deep` and `--phase backward` time, with sampled
+units against the oracle's token loop.
 """
 import functools
 
@@ -147,3 +149,52 @@ def test_wide_memory_decode(mode, steps):
     ry, rs = oracle.forward(seq["k"], seq["q"], seq["v"], seq["alpha"], seq["eta"], seq["theta"],
                             {nm: x[sample] for nm, x in state0.items()}, 1)
     compare(gy, gst, ry, rs, TOL[mode], what=f"decode {mode} x{steps}")
+
+
+def test_deep_memory_760m_class_sampled_units():
+    """The deep memory (4 layers) on the 760M-class shape in the launch configuration
+    `bench.py --phase deep` times: all 128 units on the tensor-core deep kernel, two units (the
+    first and the last) against the oracle's deep token loop over the whole 4096 tokens."""
+    w = synth.WORKLOADS["mlp-d64-b8h16-t4k"]
+    L = 4
+    inp = synth.make_inputs(w)
+    st = synth.make_deep_state(w, L)
+    m = mem.Memory(w.d, w.h, w.chunk, w.dtype, w.B, w.H, layers=L)
+    assert m.path() == mem.PATH_TC_DEEP
+    dev = lambda x, *s: x.reshape(w.B, w.H, *s).cuda().contiguous()
+    toks = {n: dev(inp[n], w.T, w.d) for n in ("k", "q", "v")}
+    gates = {n: dev(inp[n], w.T) for n in ("alpha", "eta", "theta")}
+    state = {n: dev(st[n], st[n].shape[-1]) for n in ("W", "S")}
+    y = m.forward_deep(toks["k"], toks["q"], toks["v"], gates["alpha"], gates["eta"], gates["theta"], state)
+    m.sync_status()
+    sample = [0, w.units - 1]
+    gy = y.reshape(w.units, w.T, w.d)[sample].float().cpu().numpy()
+    gst = {n: t.reshape(w.units, -1)[sample].cpu().numpy() for n, t in state.items()}
+    ry, rst = oracle.forward_deep(*(inp[n][sample] for n in ("k", "q", "v", "alpha", "eta", "theta")),
+                                  {n: st[n][sample] for n in ("W", "S")}, w.chunk, L)
+    compare(gy, gst, ry, rst, TOL["bf16"], what="deep L=4 760M-class, sampled units")
+
+
+def test_backward_760m_class_sampled_unit():
+    """The tensor-core backward on the 760M-class shape in the launch configuration
+    `bench.py --phase backward` times (all 128 units, 4096 tokens); one unit's gradients of
+    <dy, y> against the oracle's fp64 reverse-mode gradients through the token loop."""
+    from parity import rel_err
+    w = synth.WORKLOADS["mlp-d64-b8h16-t4k"]
+    inp = synth.make_inputs(w)
+    dev = lambda x: x.reshape(w.B, w.H, *x.shape[1:]).cuda().contiguous()
+    dy = torch.randn(w.units, w.T, w.d, generator=torch.Generator().manual_seed(5)).to(torch.bfloat16)
+    m = mem.Memory(w.d, w.h, w.chunk, w.dtype, w.B, w.H)
+    assert m.backward_path() == mem.PATH_TC_BACKWARD
+    out = m.backward(*[dev(inp[n]) for n in ("k", "q", "v", "alpha", "eta", "theta")],
+                     {n: dev(inp[n]) for n in ("W1", "W2", "S1", "S2")}, dev(dy))
+    m.sync_status()
+    u = w.units - 1
+    one = lambda x: x[u:u + 1]
+    ref = oracle.backward(*(one(inp[n]) for n in ("k", "q", "v", "alpha", "eta", "theta")),
+                          {n: one(inp[n]) for n in ("W1", "W2", "S1", "S2")}, w.chunk, one(dy).float(), {})
+    for n in ("k", "q", "v", "alpha", "eta", "theta", "W1", "W2", "S1", "S2"):
+        x = out[n].reshape(w.units, -1)[u:u + 1].float().cpu().numpy()
+        e = rel_err(x, np.asarray(ref[n], np.float64).reshape(1, -1))
+        assert np.isfinite(x).all(), n
+        assert e.max() <= TOL["bf16"], f"d{n}: {e.max():.3e}"
