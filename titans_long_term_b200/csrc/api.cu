@@ -479,7 +479,13 @@ size_t titans_mem_backward_workspace_bytes(titans_mem_t m, long T, int chunk) {
     if (backward_tc_eligible(m->cfg, chunk))
         f = std::max(f, (titans::mlp_backward_tc_ws_bytes(T, chunk) + sizeof(float) - 1) / sizeof(float));
     const size_t per_unit = (f + 63) & ~size_t(63);
-    return per_unit * sizeof(float) * (size_t)m->cfg.B * m->cfg.H;
+    const size_t units = (size_t)m->cfg.B * m->cfg.H;
+    // the tensor-core backward runs the forward once on a copy of the initial state, kept after
+    // the units' slices: W1, W2, S1, S2 [units][h * d] each
+    const size_t fwd_state = backward_tc_eligible(m->cfg, chunk)
+                                 ? 4 * units * (size_t)m->cfg.d * m->cfg.d_hidden * sizeof(float)
+                                 : 0;
+    return per_unit * sizeof(float) * units + fwd_state;
 }
 
 titans_status_t titans_mem_backward(titans_mem_t m, const void* k, const void* q, const void* v, const float* alpha,
@@ -516,7 +522,7 @@ titans_status_t titans_mem_backward(titans_mem_t m, const void* k, const void* q
         return fail(TITANS_EINVAL, "workspace smaller than titans_mem_backward_workspace_bytes(): " +
                                        std::to_string(workspace_bytes) + " < " + std::to_string(need));
     const long units = (long)m->cfg.B * m->cfg.H;
-    cudaError_t e;
+    cudaError_t e = cudaSuccess;
     if (mlp) {
         titans::MlpBackwardArgs b{};
         b.d = m->cfg.d;
@@ -551,10 +557,36 @@ titans_status_t titans_mem_backward(titans_mem_t m, const void* k, const void* q
         b.dS1_0 = dS1_0;
         b.dS2_0 = dS2_0;
         b.ws = static_cast<float*>(workspace);
-        b.ws_per_unit = need / sizeof(float) / (size_t)units;
         b.status = m->status;
-        e = backward_tc_eligible(m->cfg, chunk) ? titans::launch_mlp_backward_tc(b, static_cast<cudaStream_t>(stream))
-                                                : titans::launch_mlp_backward(b, static_cast<cudaStream_t>(stream));
+        cudaStream_t st = static_cast<cudaStream_t>(stream);
+        if (backward_tc_eligible(m->cfg, chunk)) {
+            // The forward with checkpoints: the tensor-core chunk kernel runs on a copy of the initial
+            // state and writes every chunk-start state into the units' workspace slices (y goes to
+            // dk, which the backward overwrites).
+            const size_t hd = (size_t)m->cfg.d * m->cfg.d_hidden;
+            const size_t fwd_state = 4 * (size_t)units * hd * sizeof(float);
+            b.ws_per_unit = (need - fwd_state) / sizeof(float) / (size_t)units;
+            float* sw = reinterpret_cast<float*>(static_cast<char*>(workspace) + (need - fwd_state));
+            float* sW[4] = {sw, sw + units * hd, sw + 2 * units * hd, sw + 3 * units * hd};
+            const float* src[4] = {W1, W2, S1, S2};
+            for (int i = 0; i < 4 && e == cudaSuccess; ++i)
+                e = cudaMemcpyAsync(sW[i], src[i], (size_t)units * hd * sizeof(float), cudaMemcpyDeviceToDevice, st);
+            if (e != cudaSuccess) return cuda_fail(e, "copying the initial state");
+            CUtensorMap tk, tq, tv;
+            if (!encode_tokens(&tk, k, T, units, chunk) || !encode_tokens(&tq, q, T, units, chunk) ||
+                !encode_tokens(&tv, v, T, units, chunk))
+                return fail(TITANS_ECUDA, "cuTensorMapEncodeTiled failed");
+            titans::ForwardArgs a = make_args(m, k, q, v, alpha, eta, theta, T, chunk, sW[0], sW[1], sW[2], sW[3], dk);
+            a.ckpt = reinterpret_cast<float*>(static_cast<char*>(workspace) + titans::mlp_backward_tc_ckpt_offset());
+            a.ckpt_unit_stride = b.ws_per_unit;
+            e = titans::launch_chunk_tc_mlp64(a, tk, tq, tv, st);
+            if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
+            b.ckpt_ready = true;
+            e = titans::launch_mlp_backward_tc(b, st);
+        } else {
+            b.ws_per_unit = need / sizeof(float) / (size_t)units;
+            e = titans::launch_mlp_backward(b, st);
+        }
     } else {
         titans::LinearBackwardArgs b{};
         b.d = m->cfg.d;

@@ -186,12 +186,13 @@ __device__ __forceinline__ float tanh_approx(float x) {
     return y;
 }
 
+template <bool kCkpt>  // kCkpt: also write every chunk-start state to ckpt (the backward's first pass)
 __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ,
     const __grid_constant__ CUtensorMap tmV, const float* __restrict__ alpha, const float* __restrict__ eta,
     const float* __restrict__ theta, float* __restrict__ W1g, float* __restrict__ W2g, float* __restrict__ S1g,
     float* __restrict__ S2g, __nv_bfloat16* __restrict__ yg, const __nv_bfloat16* __restrict__ attn, long T,
-    long gate_ld, int chunk, int chunk_gates, unsigned* status) {
+    long gate_ld, int chunk, int chunk_gates, unsigned* status, float* __restrict__ ckpt, long ckpt_stride) {
     using namespace tc;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -597,12 +598,31 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
             if (!wait(B_SC0 + p, (uint32_t)(c >> 1) & 1u)) break;
             {
                 const float An = s_scal[4 * p], sig = s_scal[4 * p + 2];
+                // Optional checkpoint of the chunk-start state (W in registers, S in TMEM), for the
+                // backward's first pass: W1, S1 rows and W2, S2 columns of this thread's hidden row.
+                float* ck = kCkpt ? ckpt + u * ckpt_stride + (long)c * 4 * kH * kD : nullptr;
 #pragma unroll
                 for (int blk = 0; blk < 4; ++blk) {
                     uint32_t r1[16], r2[16];
                     tmem_ld16(t_s + 16 * blk, r1);
                     tmem_ld16(t_s + 64 + 16 * blk, r2);
                     tmem_wait_ld();
+                    if (kCkpt) {
+                        float4* c1 = reinterpret_cast<float4*>(ck + (size_t)hrow * kD + 16 * blk);
+                        float4* s1 = reinterpret_cast<float4*>(ck + 2 * kH * kD + (size_t)hrow * kD + 16 * blk);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            c1[i] = make_float4(2.f * w1[16 * blk + 4 * i], 2.f * w1[16 * blk + 4 * i + 1],
+                                                2.f * w1[16 * blk + 4 * i + 2], 2.f * w1[16 * blk + 4 * i + 3]);
+                            s1[i] = make_float4(2.f * __uint_as_float(r1[4 * i]), 2.f * __uint_as_float(r1[4 * i + 1]),
+                                                2.f * __uint_as_float(r1[4 * i + 2]), 2.f * __uint_as_float(r1[4 * i + 3]));
+                        }
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            ck[kH * kD + (size_t)(16 * blk + i) * kH + hrow] = w2[16 * blk + i];
+                            ck[3 * kH * kD + (size_t)(16 * blk + i) * kH + hrow] = __uint_as_float(r2[i]);
+                        }
+                    }
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
                         w1[16 * blk + i] = fmaf(An, w1[16 * blk + i], sig * __uint_as_float(r1[i]));
@@ -792,14 +812,19 @@ cudaError_t launch_chunk_tc_mlp64(const ForwardArgs& a, const CUtensorMap& tk, c
     if (e0 != cudaSuccess) return e0;
     const unsigned long long bit = 1ull << (dev & 63);
     if (!(attr_set.load() & bit)) {
-        cudaError_t e = cudaFuncSetAttribute(chunk_fwd_tc_mlp64, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t e = cudaFuncSetAttribute(chunk_fwd_tc_mlp64<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)tc::kSmemBytes);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(chunk_fwd_tc_mlp64<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)tc::kSmemBytes);
         if (e != cudaSuccess) return e;
         attr_set.fetch_or(bit);
     }
-    chunk_fwd_tc_mlp64<<<(unsigned)a.units, tc::kThreads, tc::kSmemBytes, st>>>(
+    auto kernel = a.ckpt ? chunk_fwd_tc_mlp64<true> : chunk_fwd_tc_mlp64<false>;
+    kernel<<<(unsigned)a.units, tc::kThreads, tc::kSmemBytes, st>>>(
         tk, tq, tv, a.alpha, a.eta, a.theta, a.W1, a.W2, a.S1, a.S2, (__nv_bfloat16*)a.y,
-        (const __nv_bfloat16*)a.attn, a.T, a.gate_ld, a.chunk, (int)a.chunk_gates, a.status);
+        (const __nv_bfloat16*)a.attn, a.T, a.gate_ld, a.chunk, (int)a.chunk_gates, a.status, a.ckpt,
+        (long)a.ckpt_unit_stride);
     return cudaGetLastError();
 }
 

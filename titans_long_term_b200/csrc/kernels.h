@@ -21,6 +21,10 @@ struct ForwardArgs {
     float* ws;         // CUDA-core path workspace
     size_t ws_per_unit;
     unsigned* status;  // device status word
+    // Tensor-core chunk kernel only: when set, every chunk's start state [W1 | W2 | S1 | S2] (fp32,
+    // 4 h d floats) is also written to ckpt + unit * ckpt_unit_stride + chunk * 4 h d.
+    float* ckpt = nullptr;
+    size_t ckpt_unit_stride = 0;
 };
 
 size_t cuda_cores_ws_floats(int d, int h, int n);
@@ -80,6 +84,7 @@ struct MlpBackwardArgs {
     float* ws;
     size_t ws_per_unit;  // floats
     unsigned* status;    // device status word (the tensor-core backward's bounded waits)
+    bool ckpt_ready = false;  // tensor-core backward: the chunk-start states are already in the workspace
 };
 size_t mlp_backward_ws_floats(int d, int h, long T, int chunk);
 cudaError_t launch_mlp_backward(const MlpBackwardArgs& a, cudaStream_t st);
@@ -87,6 +92,7 @@ cudaError_t launch_mlp_backward(const MlpBackwardArgs& a, cudaStream_t st);
 // mlp_backward_tc_ws_bytes() of workspace per unit (MlpBackwardArgs::ws_per_unit floats apart).
 bool mlp_backward_tc_supported(int d, int h, int chunk);
 size_t mlp_backward_tc_ws_bytes(long T, int chunk);
+size_t mlp_backward_tc_ckpt_offset();  // byte offset of the chunk-start states in a unit's workspace
 cudaError_t launch_mlp_backward_tc(const MlpBackwardArgs& a, cudaStream_t st);
 cudaError_t launch_linear_backward(const LinearBackwardArgs& b, cudaStream_t st);
 size_t tc_phased_ws_bytes_per_unit();

@@ -388,14 +388,16 @@ __global__ void __launch_bounds__(mbt::kThreads, 1) mlp_backward_tc_kernel(const
     zero(CG, (size_t)128 * 2 * kD * 2);
     zero(DZ, (size_t)128 * kH * 2);
     zero(DL, (size_t)128 * kH * 2);
-    for (size_t i = tid; i < 4 * kHD; i += kThreads) {
-        const float* src = i < kHD ? a.W1 : (i < 2 * kHD ? a.W2 : (i < 3 * kHD ? a.S1 : a.S2));
-        ckpt[i] = src[u * kHD + (i % kHD)];
-    }
+    if (!a.ckpt_ready)
+        for (size_t i = tid; i < 4 * kHD; i += kThreads) {
+            const float* src = i < kHD ? a.W1 : (i < 2 * kHD ? a.W2 : (i < 3 * kHD ? a.S1 : a.S2));
+            ckpt[i] = src[u * kHD + (i % kHD)];
+        }
     __syncthreads();
 
-    // ---- pass 1: the forward, keeping each chunk-start state
-    for (long c = 0; c + 1 < nch && ok; ++c) {
+    // ---- pass 1: the forward, keeping each chunk-start state (unless the chunk kernel already
+    //      wrote them into the workspace)
+    for (long c = 0; c + 1 < nch && ok && !a.ckpt_ready; ++c) {
         const long t0 = c * chunk;
         const int n = (int)min((long)chunk, T - t0);
         const float* X = ckpt + (size_t)c * 4 * kHD;
@@ -747,6 +749,8 @@ __global__ void __launch_bounds__(mbt::kThreads, 1) mlp_backward_tc_kernel(const
 bool mlp_backward_tc_supported(int d, int h, int chunk) {
     return d == mbt::kD && h == mbt::kH && chunk >= 1 && chunk <= mbt::kN;
 }
+
+size_t mlp_backward_tc_ckpt_offset() { return mbt::layout(1).ckpt; }
 
 size_t mlp_backward_tc_ws_bytes(long T, int chunk) {
     if (chunk < 1) return 0;
