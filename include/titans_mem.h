@@ -271,8 +271,12 @@ titans_status_t titans_mem_forward_noalloc(const titans_mem_config *cfg, const v
  * from the upstream dy [B, H, T, d] (dtype of k) and dW1, dW2, dS1, dS2 (NULL = zero). It reruns
  * the forward, keeping every chunk-start state in `workspace` (caller-owned device memory of at
  * least titans_mem_backward_workspace_bytes(m, T, chunk) bytes, 16-byte aligned), then walks the
- * chunks backwards (fp32 on CUDA cores; the MLP's adjoint includes the second-order terms of the
- * inner gradient). Per-token gates only. Returns TITANS_EUNSUPPORTED for a deep memory or with
+ * chunks backwards; the MLP's adjoint includes the second-order terms of the inner gradient.
+ * In TITANS_BF16 mode with d = 64, h = 256, chunk <= 64 and no TITANS_FLAG_CUDA_CORES it runs on
+ * tensor cores (titans_mem_path(m, chunk, 2) == TITANS_PATH_TC_BACKWARD): the forward is the
+ * tensor-core chunk kernel writing checkpoints (its y goes to dk, which is then overwritten), and
+ * the backward pass is bf16 tcgen05 GEMMs with fp32 accumulation. Otherwise fp32 on CUDA cores.
+ * Per-token gates only. Returns TITANS_EUNSUPPORTED for a deep memory or with
  * TITANS_FLAG_CHUNK_GATES, TITANS_EINVAL for a NULL or misaligned pointer or a small workspace.
  */
 size_t titans_mem_backward_workspace_bytes(titans_mem_t m, long T, int chunk);
