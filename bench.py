@@ -636,12 +636,14 @@ def extension_results(dev, steps: int, warmup: int):
                                   "inputs": synth.describe(w)},
                        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
                                     "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"], "traffic": None,
-                                    "peak_source": f"bf16_tflops ({which})", "kernel": "mlp_backward_tc_kernel",
+                                    "peak_source": f"bf16_tflops ({which})",
+                                    "kernel": "chunk_fwd_tc_mlp64<true> + mlp_backward_tc_kernel",
                                     "flops_per_launch": flops, "avg_launch_ms": avg, "sms_used": sms,
                                     "frac_of_sms_used": achieved / (peaks["bf16_tflops"] * sms / 148),
-                                    "note": "FLOPs counted as twice the forward's 18 d h per head-token; the "
-                                            "kernel also reruns the forward once to keep the chunk-start states"},
-                       "gpu_launches": nb}
+                                    "note": "one titans_mem_backward call: the forward with chunk-start "
+                                            "checkpoints, then the backward pass; FLOPs counted as twice the "
+                                            "forward's 18 d h per head-token"},
+                       "gpu_launches": 2 * nb}
             del m
         out[key] = rec
         del toks, gates, state, dy
@@ -695,7 +697,8 @@ def backward_arm(args, w, rank, world, local_rank):
     peaks, which = load_peaks()
     flops = 2 * flops_per_head_token(w) * w.units * w.T
     achieved = flops / (statistics.mean(per) / 1e3) / 1e12
-    kernel = "mlp_backward_tc_kernel" if m.backward_path() == mem.PATH_TC_BACKWARD else "mlp_backward_kernel"
+    tc = m.backward_path() == mem.PATH_TC_BACKWARD
+    kernel = "chunk_fwd_tc_mlp64<true> + mlp_backward_tc_kernel" if tc else "mlp_backward_kernel"
     print(json.dumps({
         "metric": "backward tokens/sec (gradients of every input) per B200; % bf16 tensor-core peak",
         "value": world * w.B * w.T / (ms / 1e3), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
@@ -705,7 +708,7 @@ def backward_arm(args, w, rank, world, local_rank):
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": achieved / peaks["bf16_tflops"], "traffic": None, "peak_source": f"bf16_tflops ({which})",
                      "kernel": kernel, "flops_per_launch": flops, "avg_launch_ms": statistics.mean(per)},
-        "gpu_launches": args.steps}), flush=True)
+        "gpu_launches": (2 if tc else 1) * args.steps}), flush=True)
 
 
 def extra_results(args, dev):
