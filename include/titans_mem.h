@@ -303,6 +303,15 @@ const char *titans_last_error_string(void);
 /* Library version: major * 10000 + minor * 100 + patch. */
 int titans_mem_version(void);
 
+/* Diagnostic: the two evaluations of the MLP memory's activation that the tensor-core chunk kernel
+ * uses, silu(z) = h (1 + tanh h) with h = z / 2 ("Titans", walk-through sec. 3.1: the memory is an
+ * MLP; hotdry blog sec. 3.1: memory(x) = W2 sigma(W1 x) with SiLU). For each of the n fp32 values h
+ * (device memory), silu_fma[i] takes tanh from fp32 arithmetic on the FMA pipe (Chebyshev
+ * interpolants, absolute error on tanh below 1.1e-4) and silu_mufu[i] from the hardware's
+ * tanh.approx. All three arrays are caller-owned device memory of n floats, asynchronous on
+ * `stream`. TITANS_EINVAL for n < 0 or a NULL pointer, TITANS_ECUDA for a failed launch. */
+titans_status_t titans_silu_routes(const float *h, float *silu_fma, float *silu_mufu, long n, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

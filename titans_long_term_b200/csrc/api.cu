@@ -171,6 +171,14 @@ extern "C" {
 
 int titans_mem_version(void) { return 100; }
 
+titans_status_t titans_silu_routes(const float* h, float* silu_fma, float* silu_mufu, long n, void* stream) {
+    if (n < 0) return fail(TITANS_EINVAL, "titans_silu_routes: n < 0");
+    if (n > 0 && (!h || !silu_fma || !silu_mufu)) return fail(TITANS_EINVAL, "titans_silu_routes: NULL pointer");
+    const cudaError_t e = titans::launch_silu_routes(h, silu_fma, silu_mufu, n, (cudaStream_t)stream);
+    if (e != cudaSuccess) return fail(TITANS_ECUDA, std::string("titans_silu_routes: ") + cudaGetErrorString(e));
+    return TITANS_OK;
+}
+
 const char* titans_last_error_string(void) { return g_err.c_str(); }
 
 }  // extern "C"

@@ -39,6 +39,7 @@
 //     warpgroups (setmaxnreg).
 // Hand-offs go through mbarriers only; every wait is bounded.
 #include <cuda_bf16.h>
+#include <algorithm>
 #include <atomic>
 #include <cstdint>
 
@@ -56,6 +57,12 @@ constexpr int kThreads = 384;  // 3 warpgroups: tile 0, tile 1, producer (warp 8
 constexpr int kRegsLaunch = 168, kRegsProducer = 88, kRegsEpilogue = 208;
 static_assert(128 * kRegsProducer + 256 * kRegsEpilogue <= 384 * kRegsLaunch, "register split");
 constexpr int kD = 64, kH = 256, kN = 64;
+// SiLU split between the special-function unit and the FMA pipe: of each 16-column block of the
+// queries, the first kQueryFma columns take the FMA-pipe tanh (about 15 instructions instead of
+// one MUFU op). Measured on the 128-unit, 4096-token workload, shares of 4, 6 and 8 columns take
+// a launch from 0.409 ms to 0.419, 0.424 and 0.440 ms: the phase is not bound by the MUFU's
+// throughput, so every evaluation stays on it (0 compiles to the MUFU-only loop).
+constexpr int kQueryFma = 0;
 // Shared-memory map (byte offsets from a 1024-aligned base). Every tile is
 // [rows][64] bf16 with the 128-byte swizzle: 128 B per row, 1024-B atoms of 8 rows.
 constexpr uint32_t W1 = 0;             // [256 h][64 d]      A of Z^T (K-major)
@@ -185,6 +192,31 @@ __device__ __forceinline__ float tanh_approx(float x) {
     asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
+
+// tanh|h| on the FMA and integer pipes only, so that part of the SiLU's evaluations leave the
+// special-function unit, the bound of the SiLU phase, to run beside it. With e = exp(-2|h|) = 2^-y:
+// 2^-y = 2^-n 2^-f (n = round(y) by the 1.5 * 2^23 rounding constant, f in [-1/2, 1/2], 2^-f a cubic,
+// 2^-n subtracted from the exponent field), then tanh|h| = (1 - e) / (1 + e) as a quintic in
+// e in [0, 1]. Both polynomials are Chebyshev interpolants generated by the fit script of this
+// package (titans_long_term_b200/silu_fit.py); the absolute error is below 1.1e-4 (2^-13.2) for
+// every fp32 h.
+namespace tanh_fma {
+constexpr float kP0 = 9.999245405e-01f, kP1 = -6.931367517e-01f, kP2 = 2.426394820e-01f, kP3 = -5.583828315e-02f;
+constexpr float kQ0 = 9.998979568e-01f, kQ1 = -1.992551446e+00f, kQ2 = 1.906841516e+00f, kQ3 = -1.541145802e+00f, kQ4 = 8.358757496e-01f, kQ5 = -2.089689374e-01f;
+constexpr float kLog2eX2 = 2.885390082f, kYMax = 64.f, kRound = 12582912.f;
+}  // namespace tanh_fma
+__device__ __forceinline__ float tanh_abs_fma(float h) {
+    using namespace tanh_fma;
+    const float y = fminf(fabsf(h) * kLog2eX2, kYMax);
+    const float r = y + kRound;
+    const float f = y - (r - kRound);
+    const float p = fmaf(fmaf(fmaf(kP3, f, kP2), f, kP1), f, kP0);
+    // 0 <= n <= 64 sits in the low bits of r; (bits(r) << 23) mod 2^32 = n << 23.
+    const float e = __uint_as_float(__float_as_uint(p) - (__float_as_uint(r) << 23));
+    return fmaf(fmaf(fmaf(fmaf(fmaf(kQ5, e, kQ4), e, kQ3), e, kQ2), e, kQ1), e, kQ0);
+}
+// silu(2h) = h (1 + tanh h) = h + |h| tanh|h| on that route.
+__device__ __forceinline__ float silu_half_fma(float h) { return fmaf(fabsf(h), tanh_abs_fma(h), h); }
 
 template <bool kCkpt>  // kCkpt: also write every chunk-start state to ckpt (the backward's first pass)
 __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
@@ -575,8 +607,11 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
                     pk[i / 2] = pack_bf16x2(a0, a1);
                     rk[i] = __float_as_uint(fmaf(-a0, s0, a0 + s0));  // silu' = sigma + silu (1 - sigma)
                     rk[i + 1] = __float_as_uint(fmaf(-a1, s1, a1 + s1));
+                    // Queries: the first kQueryFma columns of a block take the FMA-pipe tanh.
                     const float g0 = __uint_as_float(rq[i]), g1 = __uint_as_float(rq[i + 1]);
-                    pq[i / 2] = pack_bf16x2(fmaf(g0, tanh_approx(g0), g0), fmaf(g1, tanh_approx(g1), g1));
+                    const float q0 = i < kQueryFma ? silu_half_fma(g0) : fmaf(g0, tanh_approx(g0), g0);
+                    const float q1 = i + 1 < kQueryFma ? silu_half_fma(g1) : fmaf(g1, tanh_approx(g1), g1);
+                    pq[i / 2] = pack_bf16x2(q0, q1);
                 }
                 tmem_st16(t_work + 16 * blk, rk);
 #pragma unroll
@@ -800,6 +835,23 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
 }
 
 #undef DBG
+
+// Both SiLU routes of the chunk kernel, silu(2h) = h (1 + tanh h), on n arguments h.
+__global__ void silu_routes_kernel(const float* __restrict__ h, float* __restrict__ s_fma,
+                                   float* __restrict__ s_mufu, long n) {
+    for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < n; i += (long)gridDim.x * blockDim.x) {
+        const float x = h[i];
+        s_fma[i] = silu_half_fma(x);
+        s_mufu[i] = fmaf(x, tanh_approx(x), x);
+    }
+}
+
+cudaError_t launch_silu_routes(const float* h, float* s_fma, float* s_mufu, long n, cudaStream_t st) {
+    if (n <= 0) return cudaSuccess;
+    const long blocks = std::min<long>((n + 255) / 256, 148L * 8);
+    silu_routes_kernel<<<(unsigned)blocks, 256, 0, st>>>(h, s_fma, s_mufu, n);
+    return cudaGetLastError();
+}
 
 size_t chunk_tc_mlp64_smem_bytes() { return tc::kSmemBytes; }
 

@@ -37,6 +37,8 @@ cudaError_t launch_step_cluster(const ForwardArgs& a, cudaStream_t st);
 cudaError_t launch_chunk_tc_mlp64(const ForwardArgs& a, const CUtensorMap& tk, const CUtensorMap& tq,
                                   const CUtensorMap& tv, cudaStream_t st);
 size_t chunk_tc_mlp64_smem_bytes();
+// Both SiLU evaluations of the chunk kernel (FMA-pipe and special-function-unit tanh) on n values.
+cudaError_t launch_silu_routes(const float* h, float* s_fma, float* s_mufu, long n, cudaStream_t st);
 // Phased tensor-core chunk kernel of the wide memory (d = 128, h = 512, chunk <= 128, bf16): a
 // cooperative persistent launch over all SMs. Needs tc_phased_ws_bytes_per_unit() bytes of
 // workspace per unit (a.ws, a.ws_per_unit floats apart) and two device words `sync` for its grid

@@ -31,7 +31,7 @@ EXPORTED = ["titans_mem_init", "titans_mem_destroy", "titans_mem_forward", "tita
             "titans_mem_path", "titans_mem_sync_status", "titans_last_error_string", "titans_mem_version",
             "titans_mem_forward_noalloc", "titans_mem_forward_host", "titans_mem_forward_gated",
             "titans_mem_step_gated", "titans_mem_init_deep", "titans_mem_forward_deep", "titans_mem_backward",
-            "titans_mem_backward_workspace_bytes"]
+            "titans_mem_backward_workspace_bytes", "titans_silu_routes"]
 
 
 class TitansError(RuntimeError):
@@ -79,11 +79,12 @@ def lib():
         L.titans_mem_backward_workspace_bytes.restype = ctypes.c_size_t
         L.titans_mem_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, l, i] + [vp] * 20 + [ctypes.c_size_t, vp]
         L.titans_mem_sync_status.argtypes = [vp, vp]
+        L.titans_silu_routes.argtypes = [vp, vp, vp, l, vp]
         L.titans_last_error_string.restype = ctypes.c_char_p
         for f in ("titans_mem_init", "titans_mem_destroy", "titans_mem_forward", "titans_mem_step",
                   "titans_mem_path", "titans_mem_sync_status", "titans_mem_version", "titans_mem_forward_noalloc",
                   "titans_mem_forward_host", "titans_mem_forward_gated", "titans_mem_step_gated",
-                  "titans_mem_init_deep", "titans_mem_forward_deep", "titans_mem_backward"):
+                  "titans_mem_init_deep", "titans_mem_forward_deep", "titans_mem_backward", "titans_silu_routes"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -304,3 +305,13 @@ def forward_noalloc(k, q, v, alpha, eta, theta, state: Dict[str, torch.Tensor], 
                                             _ptr(theta), T, chunk, _ptr(state["W1"]), _ptr(state.get("W2")),
                                             _ptr(state["S1"]), _ptr(state.get("S2")), _ptr(y), _stream(stream)))
     return y
+
+
+def silu_routes(h: torch.Tensor):
+    """silu(2h) on the chunk kernel's two routes: (FMA-pipe tanh, hardware tanh.approx), fp32 on the device."""
+    if h.dtype != torch.float32 or not h.is_cuda:
+        raise TypeError("h must be a CUDA fp32 tensor")
+    h = h.contiguous()
+    a, b = torch.empty_like(h), torch.empty_like(h)
+    _check(lib().titans_silu_routes(_ptr(h), _ptr(a), _ptr(b), h.numel(), _stream(None)))
+    return a, b
