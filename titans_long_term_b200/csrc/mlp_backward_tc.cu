@@ -58,7 +58,7 @@ __host__ __device__ inline Layout layout(long nch) {
         return at;
     };
     L.ckpt = take((size_t)nch * 4 * kHD * 4);  // fp32 chunk-start states [nch][W1 | W2 | S1 | S2]
-    L.adj = take(2 * 4 * kHD * 4);             // fp32 adjoints at the chunk's end and start
+    L.adj = take(4 * kHD * 4);                 // fp32 adjoint, updated in place chunk by chunk
     L.w1b = take(kHD * 2);                     // bf16 W1 [h][d]
     L.w2b = take(kHD * 2);                     // bf16 W2 [d][h]
     L.dw1b = take(kHD * 2 * 2);                // bf16 [h][dW1' | dS1']
@@ -465,8 +465,9 @@ __global__ void __launch_bounds__(mbt::kThreads, 1) mlp_backward_tc_kernel(const
     }
 
     // ---- pass 2: backwards
-    float* dcur = adj;             // adjoint at the chunk's end: dW1', dW2', dS1', dS2'
-    float* dnext = adj + 4 * kHD;  // adjoint at its start
+    // The adjoint dW1', dW2', dS1', dS2' at the chunk's end; the update below turns it into the
+    // chunk-start adjoint in place (each element is read, then written, by the same thread).
+    float* dcur = adj;
     for (size_t i = tid; i < 4 * kHD; i += kThreads) {
         const float* src = i < kHD ? a.dW1 : (i < 2 * kHD ? a.dW2 : (i < 3 * kHD ? a.dS1 : a.dS2));
         dcur[i] = src ? src[u * kHD + (i % kHD)] : 0.f;
@@ -681,8 +682,8 @@ __global__ void __launch_bounds__(mbt::kThreads, 1) mlp_backward_tc_kernel(const
                         ps += dwv[e] * svv[e];
                         pe += dsv[e] * svv[e];
                     }
-                    *reinterpret_cast<float4*>(dnext + o + i) = make_float4(nw[0], nw[1], nw[2], nw[3]);
-                    *reinterpret_cast<float4*>(dnext + 2 * kHD + o + i) = make_float4(ns[0], ns[1], ns[2], ns[3]);
+                    *reinterpret_cast<float4*>(dcur + o + i) = make_float4(nw[0], nw[1], nw[2], nw[3]);
+                    *reinterpret_cast<float4*>(dcur + 2 * kHD + o + i) = make_float4(ns[0], ns[1], ns[2], ns[3]);
                     const uint2 bw = make_uint2(pack2(nw[0], nw[1]), pack2(nw[2], nw[3]));
                     const uint2 bs = make_uint2(pack2(ns[0], ns[1]), pack2(ns[2], ns[3]));
                     if (part == 0) {  // [h][dW1' | dS1'], row j = i / d
@@ -726,9 +727,6 @@ __global__ void __launch_bounds__(mbt::kThreads, 1) mlp_backward_tc_kernel(const
             }
         }
         __syncthreads();
-        float* tmp = dcur;
-        dcur = dnext;
-        dnext = tmp;
     }
     if (ok)
         for (size_t i = tid; i < 4 * kHD; i += kThreads) {
