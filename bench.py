@@ -165,7 +165,18 @@ def oracle_sample(w, core_seconds: float = 15.0, units_cap: int = 0):
     dt = time.perf_counter() - t
     return {"value": units * T / w.H / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
             "sample": f"{units} units x {T} tokens of {w.name} (fp64 token loop), {dt:.2f} s wall",
-            "seconds": dt}
+            "seconds": dt, "cpu_model": cpu_model()}
+
+
+def cpu_model() -> str:
+    """The host CPU's model name (/proc/cpuinfo), or "unknown"."""
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
 
 
 def reference_arm(args, w, rank, world):
