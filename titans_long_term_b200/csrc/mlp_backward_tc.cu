@@ -492,8 +492,8 @@ __global__ void __launch_bounds__(mbt::kThreads, 1) mlp_backward_tc_kernel(const
         forward(t0, n, true);
 
         // dG0 = -(c A dW2'^T + d A dS2'^T); dc, dd from -g . (dW2' a), -g . (dS2' a)
-        gemm(256, PQ + (size_t)128 * kH, kH, false, dW2b, kH, false, kD, kH);
-        gemm(256 + kD, PQ + (size_t)128 * kH, kH, false, dW2b + kHD, kH, false, kD, kH);
+        // (one N = 128 GEMM: rows 0..63 of [dW2'; dS2'] land in columns 256.., rows 64..127 in 256 + d..)
+        gemm(256, PQ + (size_t)128 * kH, kH, false, dW2b, kH, false, 2 * kD, kH);
         if (!ok) break;
         {
             float pc = 0.f, pd = 0.f;
@@ -591,8 +591,8 @@ __global__ void __launch_bounds__(mbt::kThreads, 1) mlp_backward_tc_kernel(const
             }
         }
         // dk = -(c Delta dW1' + d Delta dS1') + dz W1, dq = dzq W1; dc, dd from -k . (Delta dW1'), ...
-        gemm(0, DL, kH, false, dW1b, 2 * kD, true, kD, kH);
-        gemm(kD, DL, kH, false, dW1b + kD, 2 * kD, true, kD, kH);
+        // (one N = 128 GEMM for Delta [dW1' | dS1']: columns 0.. and d..)
+        gemm(0, DL, kH, false, dW1b, 2 * kD, true, 2 * kD, kH);
         gemm(2 * kD, DZ, kH, false, W1b, kD, true, kD, kH);
         if (!ok) break;
         {
