@@ -628,6 +628,13 @@ __global__ void __launch_bounds__(mbt::kThreads, 1) mlp_backward_tc_kernel(const
         }
         // chunk-start adjoints: dW1 = A dW1' + [dz; dzq]^T [K; Q], dW2^T = A dW2'^T + [db; A_q; A]^T [G; dy; dyhat],
         // dS = sigma dW' + E dS'; and the chunk scalars' adjoints <dW', W>, <dW', S>, <dS', S>
+        // The adjoint update below streams this chunk's checkpoint and the adjoint (256 KB each): they
+        // start moving into L2 now, while the four GEMMs run (16 KB pieces).
+        if (tid == 0)
+            for (int piece = 0; piece < 16; ++piece) {
+                prefetch_l2_bulk(X + (size_t)piece * kHD / 4, (uint32_t)(kHD / 4 * sizeof(float)));
+                prefetch_l2_bulk(dcur + (size_t)piece * kHD / 4, (uint32_t)(kHD / 4 * sizeof(float)));
+            }
         for (int mt = 0; mt < 2; ++mt) {
             gemm(kD * mt, DZ + 128 * mt, kH, true, XQ, kD, true, kD, 128);
             gemm(2 * kD + kD * mt, PQ + 128 * mt, kH, true, GQ, kD, true, kD, 192);
@@ -664,7 +671,7 @@ __global__ void __launch_bounds__(mbt::kThreads, 1) mlp_backward_tc_kernel(const
             for (int part = 0; part < 2; ++part) {
                 const size_t o = part == 0 ? 0 : kHD;
                 const float* st = part == 0 ? st1 : st2;
-#pragma unroll 4
+#pragma unroll 8
                 for (size_t i = 4 * tid; i < kHD; i += 4 * kThreads) {
                     const float4 dw = *reinterpret_cast<const float4*>(dcur + o + i);
                     const float4 ds = *reinterpret_cast<const float4*>(dcur + 2 * kHD + o + i);
