@@ -85,6 +85,8 @@ __host__ __device__ inline Layout layout(long nch) {
 
 namespace {
 
+using phc::cp_async16;
+using phc::cp_async_wait_all;
 using phc::load_kmajor;
 using phc::load_mnmajor;
 using phc::mma_steps;
@@ -234,31 +236,61 @@ __global__ void __launch_bounds__(mbt::kThreads, 1) mlp_backward_tc_kernel(const
         uint4* x = reinterpret_cast<uint4*>(p);
         for (size_t i = tid; i < bytes / 16; i += kThreads) x[i] = make_uint4(0, 0, 0, 0);
     };
-    // Gate scan of a chunk (sequential, division-free), as the CUDA-core backward.
+    // Gate scan of a chunk on warp 0, division-free, two tokens per lane (tokens j >= n are padding:
+    // they leave every product unchanged and get c_j = d_j = 0):
+    //   P_j = prod_{l>j} (1 - alpha_l), Q_j = prod_{l>j} eta_l,
+    //   r_j = P_j + eta_{j+1} r_{j+1} (r_{n-1} = 1; an affine suffix recurrence, scanned by composing
+    //   the maps r -> a r + b), c_j = theta_j r_j, d_j = theta_j Q_j,
+    //   A = prod_l (1 - alpha_l), E = prod_l eta_l, sigma = eta_0 r_0.
     auto scan = [&](long t0, int n) {
-        for (int i = tid; i < n; i += kThreads) {
-            s_a[i] = alpha[t0 + i];
-            s_e[i] = eta[t0 + i];
-            s_t[i] = theta[t0 + i];
-        }
-        for (int i = n + tid; i < kN; i += kThreads) s_c[i] = s_d[i] = 0.f;
-        __syncthreads();
-        if (tid == 0) {
-            float Pr = 1.f, Qr = 1.f, r_next = 0.f;
-            for (int j = n - 1; j >= 0; --j) {
-                const float r = Pr + (j + 1 < n ? s_e[j + 1] * r_next : 0.f);
-                s_r[j] = r;
-                s_P[j] = Pr;
-                s_Q[j] = Qr;
-                s_c[j] = s_t[j] * r;
-                s_d[j] = s_t[j] * Qr;
-                r_next = r;
-                Pr *= 1.f - s_a[j];
-                Qr *= s_e[j];
+        if (warp == 0) {
+            const unsigned FULL = 0xffffffffu;
+            const int j0 = 2 * lane, j1 = j0 + 1;
+            const float a0 = j0 < n ? alpha[t0 + j0] : 0.f, a1 = j1 < n ? alpha[t0 + j1] : 0.f;
+            const float e0 = j0 < n ? eta[t0 + j0] : 1.f, e1 = j1 < n ? eta[t0 + j1] : 1.f;
+            const float th0 = j0 < n ? theta[t0 + j0] : 0.f, th1 = j1 < n ? theta[t0 + j1] : 0.f;
+            const float om0 = 1.f - a0, om1 = 1.f - a1;
+            float pp = om0 * om1, pq = e0 * e1;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const float x = __shfl_down_sync(FULL, pp, off), y = __shfl_down_sync(FULL, pq, off);
+                if (lane + off < 32) {
+                    pp *= x;
+                    pq *= y;
+                }
             }
-            s_scal[0] = Pr;
-            s_scal[1] = Qr;
-            s_scal[2] = s_e[0] * r_next;
+            float exP = __shfl_down_sync(FULL, pp, 1), exQ = __shfl_down_sync(FULL, pq, 1);
+            if (lane == 31) exP = exQ = 1.f;
+            const float P1 = exP, P0 = exP * om1, Q1 = exQ, Q0 = exQ * e1;
+            const float b0 = j0 < n ? P0 : 0.f, b1 = j1 < n ? P1 : 0.f;
+            const float c0 = j1 < n ? e1 : 0.f;  // coefficient of r_{j0 + 1} = r_{j1}
+            const float e_next = __shfl_down_sync(FULL, e0, 1);
+            const float c1 = j1 + 1 < n ? e_next : 0.f;  // coefficient of r_{j1 + 1}
+            float A = c0 * c1, Bv = b0 + c0 * b1;  // this lane's pair as one map of r_{j1 + 1}
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const float A2 = __shfl_down_sync(FULL, A, off), B2 = __shfl_down_sync(FULL, Bv, off);
+                if (lane + off < 32) {
+                    Bv = Bv + A * B2;
+                    A = A * A2;
+                }
+            }
+            float r_after = __shfl_down_sync(FULL, Bv, 1);
+            if (lane == 31) r_after = 0.f;
+            const float r0 = Bv, r1 = b1 + c1 * r_after;
+            s_a[j0] = a0; s_a[j1] = a1;
+            s_e[j0] = e0; s_e[j1] = e1;
+            s_t[j0] = th0; s_t[j1] = th1;
+            s_r[j0] = r0; s_r[j1] = r1;
+            s_P[j0] = P0; s_P[j1] = P1;
+            s_Q[j0] = Q0; s_Q[j1] = Q1;
+            s_c[j0] = th0 * r0; s_c[j1] = th1 * r1;
+            s_d[j0] = th0 * Q0; s_d[j1] = th1 * Q1;
+            if (lane == 0) {
+                s_scal[0] = om0 * P0;
+                s_scal[1] = e0 * Q0;
+                s_scal[2] = e0 * r0;
+            }
         }
         __syncthreads();
     };
@@ -297,14 +329,21 @@ __global__ void __launch_bounds__(mbt::kThreads, 1) mlp_backward_tc_kernel(const
                 reinterpret_cast<uint4*>(GQ + (size_t)(64 + r) * kD)[p] = x;
             }
     };
+    // bf16 copies of the chunk-start W1, W2. The 128 KB of fp32 come into the (idle) operand region of
+    // shared memory with every copy in flight at once, then go out converted.
     auto state_bf16 = [&](const float* X) {
+        const uint8_t* src = reinterpret_cast<const uint8_t*>(X);
+        for (uint32_t o = 16u * tid; o < 2u * kHD * 4u; o += 16u * kThreads) cp_async16(sb + o, src + o);
+        cp_async_wait_all();
+        __syncthreads();
+        const float4* s4 = reinterpret_cast<const float4*>(sm);
 #pragma unroll 4
         for (size_t i = tid; i < kHD / 4; i += kThreads) {
-            const float4 w1 = reinterpret_cast<const float4*>(X)[i];
-            const float4 w2 = reinterpret_cast<const float4*>(X + kHD)[i];
+            const float4 w1 = s4[i], w2 = s4[kHD / 4 + i];
             reinterpret_cast<uint2*>(W1b)[i] = make_uint2(pack2(w1.x, w1.y), pack2(w1.z, w1.w));
             reinterpret_cast<uint2*>(W2b)[i] = make_uint2(pack2(w2.x, w2.y), pack2(w2.z, w2.w));
         }
+        __syncthreads();
     };
     // Keys' (and in pass 2 queries') forward at the chunk-start weights: silu and its derivatives,
     // G = 2 (Y - v) with its c-, d-scaled copy, B = G W2 and Delta = B * silu'(Z); pass 2 also
@@ -730,21 +769,59 @@ __global__ void __launch_bounds__(mbt::kThreads, 1) mlp_backward_tc_kernel(const
                 prefetch_l2_bulk(v + tp * kD, rows);
                 prefetch_l2_bulk(dy + tp * kD, rows);
             }
+        }
+        // The gates' adjoints through the scan, on warp 0 (two tokens per lane). With dr_{-1} = dsig:
+        //   dr_j = theta_j dc_j + eta_j dr_{j-1},
+        //   F_0 = dA, F_{j+1} = (1 - alpha_j) F_j + dr_j;  H_0 = dE, H_{j+1} = eta_j H_j + theta_j dd_j,
+        //   dtheta_j = dc_j r_j + dd_j Q_j, dalpha_j = -P_j F_j, deta_j = Q_j H_j + dr_{j-1} r_j.
+        // Each recurrence is a prefix scan of affine maps x -> a x + b over the lanes.
+        if (warp == 0) {
+            const unsigned FULL = 0xffffffffu;
             float dA = 0.f, dsig = 0.f, dE = 0.f;
             for (int w = 0; w < kThreads / 32; ++w) {
                 dA += s_red[4 * w];
                 dsig += s_red[4 * w + 1];
                 dE += s_red[4 * w + 2];
             }
-            float dr_prev = 0.f, F = dA, Hh = dE;
-            for (int j = 0; j < n; ++j) {
-                const float dr = s_t[j] * s_dc[j] + (j == 0 ? s_e[0] * dsig : s_e[j] * dr_prev);
-                a.dtheta[u * T + t0 + j] = s_dc[j] * s_r[j] + s_dd[j] * s_Q[j];
-                a.dalpha[u * T + t0 + j] = -s_P[j] * F;
-                a.deta[u * T + t0 + j] = s_Q[j] * Hh + (j == 0 ? dsig * s_r[0] : dr_prev * s_r[j]);
-                F = (1.f - s_a[j]) * F + dr;
-                Hh = s_e[j] * Hh + s_t[j] * s_dd[j];
-                dr_prev = dr;
+            const int j0 = 2 * lane, j1 = j0 + 1;
+            const bool in0 = j0 < n, in1 = j1 < n;
+            // padding tokens take the identity map
+            const float e0 = in0 ? s_e[j0] : 1.f, e1 = in1 ? s_e[j1] : 1.f;
+            const float om0 = in0 ? 1.f - s_a[j0] : 1.f, om1 = in1 ? 1.f - s_a[j1] : 1.f;
+            const float g0 = in0 ? s_t[j0] * s_dc[j0] : 0.f, g1 = in1 ? s_t[j1] * s_dc[j1] : 0.f;
+            const float h0 = in0 ? s_t[j0] * s_dd[j0] : 0.f, h1 = in1 ? s_t[j1] * s_dd[j1] : 0.f;
+            // inclusive prefix over lanes of the pair maps (later map after earlier: a = a2 a1, b = a2 b1 + b2),
+            // then the exclusive value at the lane's first token
+            auto prefix = [&](float a, float b, float x0) {
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    const float ap = __shfl_up_sync(FULL, a, off), bp = __shfl_up_sync(FULL, b, off);
+                    if (lane >= off) {
+                        b = a * bp + b;
+                        a = a * ap;
+                    }
+                }
+                float ae = __shfl_up_sync(FULL, a, 1), be = __shfl_up_sync(FULL, b, 1);
+                if (lane == 0) {
+                    ae = 1.f;
+                    be = 0.f;
+                }
+                return ae * x0 + be;
+            };
+            const float dr_in = prefix(e1 * e0, e1 * g0 + g1, dsig);  // dr_{j0 - 1}
+            const float dr0 = e0 * dr_in + g0, dr1 = e1 * dr0 + g1;
+            const float F0 = prefix(om1 * om0, om1 * dr0 + dr1, dA), F1 = om0 * F0 + dr0;
+            const float H0 = prefix(e1 * e0, e1 * h0 + h1, dE), H1 = e0 * H0 + h0;
+            const long g = u * T + t0;
+            if (in0) {
+                a.dtheta[g + j0] = s_dc[j0] * s_r[j0] + s_dd[j0] * s_Q[j0];
+                a.dalpha[g + j0] = -s_P[j0] * F0;
+                a.deta[g + j0] = s_Q[j0] * H0 + dr_in * s_r[j0];
+            }
+            if (in1) {
+                a.dtheta[g + j1] = s_dc[j1] * s_r[j1] + s_dd[j1] * s_Q[j1];
+                a.dalpha[g + j1] = -s_P[j1] * F1;
+                a.deta[g + j1] = s_Q[j1] * H1 + dr0 * s_r[j1];
             }
         }
         __syncthreads();
