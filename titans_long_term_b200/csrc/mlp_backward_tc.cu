@@ -320,6 +320,7 @@ __global__ void __launch_bounds__(mbt::kThreads, 1) mlp_backward_tc_kernel(const
                 o = make_uint4(y[0], y[1], y[2], y[3]);
             }
             reinterpret_cast<uint4*>(CK + (size_t)r * 2 * kD)[p] = o;
+            reinterpret_cast<uint4*>(CK + (size_t)(r + 64) * 2 * kD)[p] = o;  // copy in rows 64..127 (below)
         }
         if (with_dy)
             for (int i = tid; i < 64 * 8; i += kThreads) {
@@ -395,6 +396,8 @@ __global__ void __launch_bounds__(mbt::kThreads, 1) mlp_backward_tc_kernel(const
                 st16_bf16(GQ + (size_t)t * kD + col, g);
                 st16_bf16(CG + (size_t)t * 2 * kD + col, gc);
                 st16_bf16(CG + (size_t)t * 2 * kD + kD + col, gd);
+                st16_bf16(CG + (size_t)(64 + t) * 2 * kD + col, gc);  // copy in rows 64..127 (below)
+                st16_bf16(CG + (size_t)(64 + t) * 2 * kD + kD + col, gd);
             }
         }
         gemm(0, GQ, kD, false, W2b, kH, true, kH, kD);  // [G; dy] W2
@@ -419,7 +422,7 @@ __global__ void __launch_bounds__(mbt::kThreads, 1) mlp_backward_tc_kernel(const
         }
     };
 
-    // ---- set-up: zero the operand buffers whose padding rows must stay zero, chunk 0's state
+    // ---- set-up: zero the operand buffers (padding rows stay zero), chunk 0's state
     zero(XQ, (size_t)128 * kD * 2);
     zero(CK, (size_t)128 * 2 * kD * 2);
     zero(PQ, (size_t)256 * kH * 2);
@@ -563,13 +566,16 @@ __global__ void __launch_bounds__(mbt::kThreads, 1) mlp_backward_tc_kernel(const
             }
         }
         // dA0 = -[c G | d G] [dW2'; dS2'];  ddelta = -[c K | d K] [dW1' | dS1']^T -> db, dz0
+        // Rows 64..127 of [c G | d G] and [c K | d K] repeat rows 0..63, so TMEM lanes 64..127 hold a
+        // second copy of the products and all eight warps share the epilogue: lanes 0..63 take the
+        // first four 16-column blocks of their half, lanes 64..127 the last four.
         gemm(0, CG, 2 * kD, false, dW2b, kH, true, kH, 2 * kD);
         gemm(256, CK, 2 * kD, false, dW1b, 2 * kD, false, kH, 2 * kD);
         if (!ok) break;
-        if (row < 64) {
-            const int t = row;
+        {
+            const int t = row & 63, sub = row >> 6;
 #pragma unroll 1
-            for (int blk = 0; blk < 8; ++blk) {
+            for (int blk = 4 * sub; blk < 4 * sub + 4; ++blk) {
                 const int col = 128 * half + 16 * blk;
                 float x[16], y[16], s[16], b[16], s2[16], o[16];
                 tmem16(tmem + lane_off + col, x);
@@ -608,16 +614,18 @@ __global__ void __launch_bounds__(mbt::kThreads, 1) mlp_backward_tc_kernel(const
                     ov[e] = -2.f * g;
                 }
                 st16_bf16(GQ + (size_t)(128 + t) * kD + col, o);
+                st16_bf16(GQ + (size_t)(192 + t) * kD + col, o);  // copy in rows 192..255 (below)
                 if (t < n && DBG(t0 + t < T)) st16_bf16(dv + (t0 + t) * kD + col, ov);
             }
         }
         // dA = dA0 + dyhat W2;  dz = dz0 + dA * silu'(Z)
+        // (rows 192..255 of GQ repeat dyhat: lanes 64..127 hold a copy, shared out as above)
         gemm(0, GQ + (size_t)128 * kD, kD, false, W2b, kH, true, kH, kD);
         if (!ok) break;
-        if (row < 64) {
-            const int t = row;
+        {
+            const int t = row & 63, sub = row >> 6;
 #pragma unroll 1
-            for (int blk = 0; blk < 8; ++blk) {
+            for (int blk = 4 * sub; blk < 4 * sub + 4; ++blk) {
                 const int col = 128 * half + 16 * blk;
                 float x[16], a0[16], s[16], z0[16], o[16];
                 tmem16(tmem + lane_off + col, x);
