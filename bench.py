@@ -68,7 +68,10 @@ def state_bytes_per_unit(w) -> float:
 # ---------------------------------------------------------------- clocks
 
 class ClockSampler:
-    """nvidia-smi samples (every 50 ms) bracketing the timed region."""
+    """SM clocks and clock-event reasons around and inside the timed region: nvidia-smi samples
+    every 50 ms from start() to stop(), and NVML reads (read-only queries) about every millisecond
+    between mark_start() and mark_stop(), so that a timed region of a few milliseconds still has
+    samples of its own."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -79,8 +82,20 @@ class ClockSampler:
         self.proc = None
         self.lines = []
         self.t_start = self.t_stop = None
+        self.nvml = None       # pynvml module once initialised
+        self.nvml_rows = []    # (sm MHz, event-reason bitmask) inside the timed region
+        self._poll = None
+        self._polling = False
 
     def start(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._handle = pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
+            self._max_sm = float(pynvml.nvmlDeviceGetMaxClockInfo(self._handle, pynvml.NVML_CLOCK_SM))
+            self.nvml = pynvml
+        except Exception:  # no NVML: nvidia-smi samples only
+            self.nvml = None
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "50",
@@ -96,10 +111,28 @@ class ClockSampler:
         for line in self.proc.stdout:
             self.lines.append((time.time(), line.strip()))
 
+    def _poll_nvml(self):
+        nv, h = self.nvml, self._handle
+        reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while self._polling:
+            try:
+                self.nvml_rows.append((nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM), int(reasons(h))))
+            except Exception:
+                return
+            time.sleep(0.005)
+
     def mark_start(self):
         self.t_start = time.time()
+        if self.nvml is not None:
+            self._polling = True
+            self._poll = threading.Thread(target=self._poll_nvml, daemon=True)
+            self._poll.start()
 
     def mark_stop(self):
+        if self._poll is not None:
+            self._polling = False
+            self._poll.join(timeout=1.0)
         self.t_stop = time.time()
 
     def stop(self):
@@ -110,6 +143,23 @@ class ClockSampler:
                 self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
+        if self.nvml is not None:
+            try:
+                self.nvml.nvmlShutdown()
+            except Exception:
+                pass
+
+    def _nvml_reasons(self, mask: int):
+        nv = self.nvml
+        names = {"hw_slowdown": "HwSlowdown", "hw_thermal_slowdown": "HwThermalSlowdown",
+                 "sw_thermal_slowdown": "SwThermalSlowdown", "sw_power_cap": "SwPowerCap",
+                 "hw_power_brake_slowdown": "HwPowerBrakeSlowdown"}
+        out = set()
+        for key, suffix in names.items():
+            bit = getattr(nv, "nvmlClocksEventReason" + suffix, None) or getattr(nv, "nvmlClocksThrottleReason" + suffix, 0)
+            if mask & bit:
+                out.add(key)
+        return out
 
     def summary(self):
         rows = []
@@ -120,7 +170,7 @@ class ClockSampler:
             rows.append((ts, parts))
         inside = [p for ts, p in rows if self.t_start and self.t_stop and self.t_start - 0.1 <= ts <= self.t_stop + 0.1]
         use = inside or [p for _, p in rows]
-        if not use:
+        if not use and not self.nvml_rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no nvidia-smi samples"], "samples": 0}
 
         def num(x):
@@ -135,9 +185,18 @@ class ClockSampler:
             for name, val in zip(names, p[5:9]):
                 if val.strip().lower() == "active":
                     reasons.add(name)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": num(use[0][2]),
-                "reasons": sorted(reasons), "samples": len(use), "samples_in_timed_region": len(inside),
-                "power_w_max": max((num(p[3]) or 0.0) for p in use)}
+        for _, mask in self.nvml_rows:
+            reasons |= self._nvml_reasons(mask)
+        nvml_sm = [float(c) for c, _ in self.nvml_rows]
+        out = {"sm_mhz": statistics.median(nvml_sm) if nvml_sm else (statistics.median(sm) if sm else None),
+               "sm_max_mhz": num(use[0][2]) if use else getattr(self, "_max_sm", None), "reasons": sorted(reasons),
+               "samples": len(use), "samples_in_timed_region": len(inside) + len(nvml_sm),
+               "nvml_samples_in_timed_region": len(nvml_sm)}
+        if use:
+            out["power_w_max"] = max((num(p[3]) or 0.0) for p in use)
+        if nvml_sm:
+            out["sm_mhz_min_in_timed_region"] = min(nvml_sm)
+        return out
 
 
 # ---------------------------------------------------------------- oracle (CPU baseline / reference arm)
