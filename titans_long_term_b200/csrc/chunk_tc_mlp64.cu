@@ -118,6 +118,23 @@ static_assert(tc::kSmemBytes <= 232448, "shared memory budget");
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
+// 16-byte global -> shared copy (cached in L2 only) and the wait for all of a thread's copies.
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit_wait() {
+    asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;" ::: "memory");
+}
+__device__ __forceinline__ float ld_shared_f32(uint32_t a) {
+    float x;
+    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(x) : "r"(a) : "memory");
+    return x;
+}
+__device__ __forceinline__ void st_shared_f32(uint32_t a, float x) {
+    asm volatile("st.shared.f32 [%0], %1;" ::"r"(a), "f"(x) : "memory");
+}
+// Named barrier of one epilogue warpgroup (tile t: barrier 1 + t, its 128 threads).
+__device__ __forceinline__ void tile_bar(int tile) { asm volatile("bar.sync %0, 128;" ::"r"(1 + tile) : "memory"); }
 
 // Writes 16 fp32 values as bf16 into columns [16 blk, 16 blk + 16) of row `row` of a
 // swizzled [rows][64] tile (two 16-byte chunks).
@@ -540,31 +557,76 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
         const uint32_t t_work = tmem + lane_off + tile * 128;     // this tile's working columns
         const uint32_t t_s = tmem + lane_off + 256 + tile * 128;  // S1 at +0, S2^T at +64
         float w1[64], w2[64];
+        // The unit's state moves between global memory and the threads' rows through shared memory
+        // that the tile does not use at entry or exit, so that every global access is coalesced:
+        //   region A (this tile's AT0 and AT1 rows, 32 KB): a row-major [128][64] fp32 block of W1 or S1,
+        //     row r at r * 256 B with its 16-byte pieces XORed by r & 15 (conflict-free row reads);
+        //   region B (this tile's bf16 W1 and W2^T rows, 32 KB): the tile's 128 columns of W2 or S2,
+        //     [64][128] fp32 (a thread's column reads are conflict-free as they stand).
+        const int it = hrow - 128 * tile;  // the thread's row within the tile
+        auto a_addr = [&](int r, int c) -> uint32_t {
+            return sb + (r < 64 ? AT0 : AT1) + (uint32_t)tile * 16384u + (uint32_t)(r & 63) * 256u +
+                   ((uint32_t)(c ^ (r & 15)) << 4);
+        };
+        auto b_addr = [&](int d, int col) -> uint32_t {
+            return sb + (d < 32 ? W1 : W2T) + (uint32_t)tile * 16384u + (uint32_t)(d & 31) * 512u + (uint32_t)col * 4u;
+        };
+        // global -> regions A, B: the tile's rows of a [256][64] matrix (32 KB, contiguous) and the
+        // tile's columns of a [64][256] matrix (64 rows of 512 B), 16-byte copies all in flight
+        auto stage_in_state = [&](const float* rows, const float* cols) {
+            const float* ga = rows + (u * kH + 128 * tile) * kD;
+            const float* gb = cols + u * kD * kH + 128 * tile;
+            for (int q = it; q < 2048; q += 128) {
+                cp_async_16(a_addr(q >> 4, q & 15), ga + 4 * q);
+                cp_async_16(b_addr(q >> 5, 4 * (q & 31)), gb + (q >> 5) * kH + 4 * (q & 31));
+            }
+            cp_async_commit_wait();
+            tile_bar(tile);
+        };
+        // regions A, B -> global, the same layouts, coalesced 16-byte stores
+        auto stage_out_state = [&](float* rows, float* cols) {
+            tile_bar(tile);
+            float* ga = rows + (u * kH + 128 * tile) * kD;
+            float* gb = cols + u * kD * kH + 128 * tile;
+            for (int q = it; q < 2048; q += 128) {
+                const uint4 x = ld_shared_v4(a_addr(q >> 4, q & 15));
+                *reinterpret_cast<uint4*>(ga + 4 * q) = x;
+                const uint4 y2 = ld_shared_v4(b_addr(q >> 5, 4 * (q & 31)));
+                *reinterpret_cast<uint4*>(gb + (q >> 5) * kH + 4 * (q & 31)) = y2;
+            }
+            tile_bar(tile);
+        };
         {
-            const float4* p = reinterpret_cast<const float4*>(W1g + (u * kH + hrow) * kD);
+            stage_in_state(W1g, W2g);
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-                const float4 x = p[i];
-                w1[4 * i] = 0.5f * x.x;
-                w1[4 * i + 1] = 0.5f * x.y;
-                w1[4 * i + 2] = 0.5f * x.z;
-                w1[4 * i + 3] = 0.5f * x.w;
+                const uint4 x = ld_shared_v4(a_addr(it, i));
+                w1[4 * i] = 0.5f * __uint_as_float(x.x);
+                w1[4 * i + 1] = 0.5f * __uint_as_float(x.y);
+                w1[4 * i + 2] = 0.5f * __uint_as_float(x.z);
+                w1[4 * i + 3] = 0.5f * __uint_as_float(x.w);
             }
-            const float* q2 = W2g + u * kD * kH + hrow;
 #pragma unroll
-            for (int i = 0; i < 64; ++i) w2[i] = q2[(size_t)i * kH];
-            const float* p1 = S1g + (u * kH + hrow) * kD;
-            const float* p2 = S2g + u * kD * kH + hrow;
+            for (int i = 0; i < 64; ++i) w2[i] = ld_shared_f32(b_addr(i, it));
+            tile_bar(tile);  // every row read before the regions take S
+            stage_in_state(S1g, S2g);
 #pragma unroll
             for (int blk = 0; blk < 4; ++blk) {
                 uint32_t r[16];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(0.5f * p1[16 * blk + i]);
+                for (int j = 0; j < 4; ++j) {
+                    const uint4 x = ld_shared_v4(a_addr(it, 4 * blk + j));
+                    r[4 * j] = __float_as_uint(0.5f * __uint_as_float(x.x));
+                    r[4 * j + 1] = __float_as_uint(0.5f * __uint_as_float(x.y));
+                    r[4 * j + 2] = __float_as_uint(0.5f * __uint_as_float(x.z));
+                    r[4 * j + 3] = __float_as_uint(0.5f * __uint_as_float(x.w));
+                }
                 tmem_st16(t_s + 16 * blk, r);
 #pragma unroll
-                for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(p2[(size_t)(16 * blk + i) * kH]);
+                for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(ld_shared_f32(b_addr(16 * blk + i, it)));
                 tmem_st16(t_s + 64 + 16 * blk, r);
             }
+            tile_bar(tile);  // region B is the bf16 W1 and W2^T rows written next
 #pragma unroll
             for (int blk = 0; blk < 4; ++blk) {
                 store16_bf16(sb + W1, hrow, blk, w1 + 16 * blk);
@@ -799,30 +861,34 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
             mbar_arrive(&bars[B_W0 + tile]);
         }
 
-        // Final state of this hidden row, once the last chunk's S accumulations have completed.
+        // Final state of this tile, once the last chunk's S accumulations (the last readers of the
+        // tile's AT0 and AT1 rows) have completed; its bf16 weight rows are no longer read either.
         if (nchunks > 0 && !*abort_flag) wait(B_SA0 + tile, (uint32_t)(nchunks - 1) & 1u);
         {
-            float4* p = reinterpret_cast<float4*>(W1g + (u * kH + hrow) * kD);
 #pragma unroll
             for (int i = 0; i < 16; ++i)
-                p[i] = make_float4(2.f * w1[4 * i], 2.f * w1[4 * i + 1], 2.f * w1[4 * i + 2], 2.f * w1[4 * i + 3]);
-            float* q2 = W2g + u * kD * kH + hrow;
+                st_shared_v4(a_addr(it, i), __float_as_uint(2.f * w1[4 * i]), __float_as_uint(2.f * w1[4 * i + 1]),
+                             __float_as_uint(2.f * w1[4 * i + 2]), __float_as_uint(2.f * w1[4 * i + 3]));
 #pragma unroll
-            for (int i = 0; i < 64; ++i) q2[(size_t)i * kH] = w2[i];
-            float* p1 = S1g + (u * kH + hrow) * kD;
-            float* p2 = S2g + u * kD * kH + hrow;
+            for (int i = 0; i < 64; ++i) st_shared_f32(b_addr(i, it), w2[i]);
+            stage_out_state(W1g, W2g);
 #pragma unroll
             for (int blk = 0; blk < 4; ++blk) {
                 uint32_t r[16];
                 tmem_ld16(t_s + 16 * blk, r);
                 tmem_wait_ld();
 #pragma unroll
-                for (int i = 0; i < 16; ++i) p1[16 * blk + i] = 2.f * __uint_as_float(r[i]);
+                for (int j = 0; j < 4; ++j)
+                    st_shared_v4(a_addr(it, 4 * blk + j), __float_as_uint(2.f * __uint_as_float(r[4 * j])),
+                                 __float_as_uint(2.f * __uint_as_float(r[4 * j + 1])),
+                                 __float_as_uint(2.f * __uint_as_float(r[4 * j + 2])),
+                                 __float_as_uint(2.f * __uint_as_float(r[4 * j + 3])));
                 tmem_ld16(t_s + 64 + 16 * blk, r);
                 tmem_wait_ld();
 #pragma unroll
-                for (int i = 0; i < 16; ++i) p2[(size_t)(16 * blk + i) * kH] = __uint_as_float(r[i]);
+                for (int i = 0; i < 16; ++i) st_shared_f32(b_addr(16 * blk + i, it), __uint_as_float(r[i]));
             }
+            stage_out_state(S1g, S2g);
         }
     }
 
