@@ -319,14 +319,15 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
         tc_fence_after();
         const float En = s_scal[4 * p + 1];
         const uint32_t tq = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + 256;
+        // 32 columns per TMEM round trip (16 measured 1% slower per launch; 64 spill at 88 registers)
 #pragma unroll 1
-        for (int col = 0; col < 256; col += 16) {
-            uint32_t r[16];
-            tmem_ld16(tq + col, r);
+        for (int col = 0; col < 256; col += 32) {
+            uint32_t r[32];
+            tmem_ld32(tq + col, r);
             tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(En * __uint_as_float(r[i]));
-            tmem_st16(tq + col, r);
+            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(En * __uint_as_float(r[i]));
+            tmem_st32(tq + col, r);
         }
         tmem_wait_st();
         tc_fence_before();
