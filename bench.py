@@ -201,17 +201,24 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- oracle (CPU baseline / reference arm)
 
-def oracle_sample(w, core_seconds: float = 15.0, units_cap: int = 0):
-    """Time the fp64 oracle (token loop, OpenMP over units, all host cores) on a bounded
-    sample of the workload: the first U units x the first T tokens, sized from a short
-    calibration run to about `core_seconds` of CPU work."""
+def oracle_rate(w) -> float:
+    """Head-tokens per second of the fp64 oracle on this host, from a short calibration run."""
     import oracle
     cores = oracle.threads()
     cal = synth.make_inputs(w, units=range(min(w.units, cores)), T=min(w.T, 2 * w.chunk))
     st = {n: cal[n] for n in cal if n[0] in "WS"}
     t = time.perf_counter()
     oracle.forward(*(cal[n] for n in ("k", "q", "v", "alpha", "eta", "theta")), st, w.chunk)
-    rate = cal["k"].shape[0] * cal["k"].shape[1] / max(time.perf_counter() - t, 1e-6)  # head-tokens/s
+    return cal["k"].shape[0] * cal["k"].shape[1] / max(time.perf_counter() - t, 1e-6)
+
+
+def oracle_sample(w, core_seconds: float = 15.0, units_cap: int = 0, rate: float = 0.0):
+    """Time the fp64 oracle (token loop, OpenMP over units, all host cores) on a bounded
+    sample of the workload: the first U units x the first T tokens, sized from a short
+    calibration run (or the given rate, head-tokens/s) to about `core_seconds` of CPU work."""
+    import oracle
+    cores = oracle.threads()
+    rate = rate or oracle_rate(w)
     want = rate * core_seconds / cores  # head-tokens for the target wall time
     units = min(w.units, units_cap or w.units, max(1, cores))
     T = int(min(w.T, max(w.chunk, (want / units) // w.chunk * w.chunk)))
@@ -246,11 +253,12 @@ def reference_arm(args, w, rank, world):
     import oracle
     per_step = 120.0 * oracle.threads() / max(1, args.steps + args.warmup)
     per_step = min(per_step, 30.0 * oracle.threads())
+    rate = oracle_rate(w)  # calibrated once, so that many short steps stay cheap
     for _ in range(args.warmup):
-        oracle_sample(w, core_seconds=per_step / 4)
+        oracle_sample(w, core_seconds=per_step / 4, rate=rate)
     vals, base = [], None
     for _ in range(args.steps):
-        base = oracle_sample(w, core_seconds=per_step)
+        base = oracle_sample(w, core_seconds=per_step, rate=rate)
         vals.append(base["value"])
     value = statistics.median(vals)
     base["value"] = value
