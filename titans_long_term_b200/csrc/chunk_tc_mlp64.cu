@@ -873,6 +873,10 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
         // Final state of this tile, once the last chunk's S accumulations (the last readers of the
         // tile's AT0 and AT1 rows) have completed; its bf16 weight rows are no longer read either.
         if (nchunks > 0 && !*abort_flag) wait(B_SA0 + tile, (uint32_t)(nchunks - 1) & 1u);
+        // Region B is this tile's bf16 weight rows, which every thread of the tile rewrote in the
+        // last chunk's weight update; the wait above does not order those stores, so all of the
+        // tile's threads finish them before any staging write.
+        tile_bar(tile);
         {
 #pragma unroll
             for (int i = 0; i < 16; ++i)
