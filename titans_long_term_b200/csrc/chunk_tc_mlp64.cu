@@ -863,11 +863,15 @@ __global__ void __launch_bounds__(tc::kThreads, 1) chunk_fwd_tc_mlp64(
                     w2[16 * blk + i] += __uint_as_float(r2[i]);
                 }
                 store16_bf16(sb + W1, hrow, blk, w1 + 16 * blk);
-                store16_bf16(sb + W2T, hrow, blk, w2 + 16 * blk);
             }
+            // The next chunk's Z^T needs only the W1 rows; every TMEM read of dW1, dW2^T is done.
             fence_proxy_async_smem();
             tc_fence_before();
             mbar_arrive(&bars[B_W0 + tile]);
+            // W2^T rows after the arrival: their readers, Y and (GW2)^T, wait for this thread's later
+            // arrivals (the SiLU's and G's), which follow these stores and a proxy fence.
+#pragma unroll
+            for (int blk = 0; blk < 4; ++blk) store16_bf16(sb + W2T, hrow, blk, w2 + 16 * blk);
         }
 
         // Final state of this tile, once the last chunk's S accumulations (the last readers of the
