@@ -184,7 +184,7 @@ typedef struct {
 /*
  * titans_mem_forward with the token streams and y in HOST memory and the state on the
  * device: the gates are copied whole first, then T is cut into segments of t_seg tokens (a multiple of `chunk`; 0 picks about
- * sixteen segments), and each segment's host-to-device copy, forward and device-to-host copy
+ * five segments), and each segment's host-to-device copy, forward and device-to-host copy
  * of y run on three streams, so the copies of one segment overlap the compute and copies of
  * the others. Running a stream in segments gives exactly the result of one call over T (a
  * segment boundary is a chunk boundary).

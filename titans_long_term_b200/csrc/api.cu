@@ -370,7 +370,10 @@ titans_status_t titans_mem_forward_host(titans_mem_t m, const void* k, const voi
     if (chunk < 1 || chunk > m->cfg.chunk)
         return fail(TITANS_EUNSUPPORTED, "chunk must be in 1..config.chunk");
     if (t_seg < 0 || t_seg % chunk != 0) return fail(TITANS_EINVAL, "t_seg must be a non-negative multiple of chunk");
-    if (t_seg == 0) t_seg = ((T + 15) / 16 + chunk - 1) / chunk * chunk;  // about 16 segments
+    // Automatic length: three times a sixteenth of T, in whole chunks (about five segments). On the
+    // 128-unit, 4096-token stream it measured 4.36-4.40 ms per call against 4.50-4.52 ms with
+    // sixteen segments: fewer, larger copies outweigh the longer last segment.
+    if (t_seg == 0) t_seg = 3 * (((T + 15) / 16 + chunk - 1) / chunk * chunk);
     const long nseg = (T + t_seg - 1) / t_seg;
     if (nseg > 4096) return fail(TITANS_EINVAL, "more than 4096 segments: raise t_seg");
     int cur = -1;
